@@ -1,0 +1,309 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with:
+  * the hand-worked cases in ``tests/golden/hand_cases.txt`` (values computed by hand
+    from the pages' definitions),
+  * closed forms (E[gamma] for Gaussian weights, the share of zero codes),
+  * invariants (code alphabet, sign symmetry, absmax -> +-127, all-zero inputs,
+    K-permutation invariance, linearity),
+  * independent library routines (numpy integer matmul, torch round/clamp in fp32,
+    torch's bf16 conversion, a float64 matmul of the dequantised operands).
+They are plain functions so that ``test_oracle_mutants`` can run the same pins
+against deliberately broken builds of the oracle and show that each break is caught.
+"""
+import math
+
+import numpy as np
+import torch
+
+from conftest import parse_golden
+
+EPS = 1e-5
+
+
+def _floats(v):
+    return np.array([float(x) for x in v.split(",")], dtype=np.float32)
+
+
+def _ints(v, dt=np.int64):
+    return np.array([int(x, 0) for x in v.split(",")], dtype=dt)
+
+
+def _bf16_bits(x_f32):
+    t = torch.from_numpy(np.asarray(x_f32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------- hand cases --
+
+def pin_hand_ternarise(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "ternarise":
+            continue
+        W = _floats(r["W"])[None, :]
+        got = O.ternarise(W, np.float32(float(r["gamma"])))
+        assert np.array_equal(got[0].astype(np.int64), _ints(r["codes"])), (r, got)
+        n += 1
+    assert n >= 2
+
+
+def pin_hand_absmean(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "absmean":
+            continue
+        N, K = int(r["N"]), int(r["K"])
+        W = _floats(r["W"]).reshape(N, K)
+        g = O.absmean_gamma(W, float(r["eps"]))
+        assert g == np.float32(float(r["gamma"])), (r, g)
+        codes = O.ternarise(W, g)
+        assert np.array_equal(codes.reshape(-1).astype(np.int64), _ints(r["codes"])), (r, codes)
+        n += 1
+    assert n >= 2
+
+
+def pin_hand_act(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "act":
+            continue
+        x = _floats(r["x"])[None, :]
+        bits = _bf16_bits(x)
+        # every hand value is exactly representable in bf16
+        assert np.array_equal(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+                              .float().numpy(), x)
+        xq, s = O.quantize_act(bits, EPS)
+        assert s[0] == np.float32(float(r["s"])), (r, s)
+        assert np.array_equal(xq[0].astype(np.int64), _ints(r["xq"])), (r, xq)
+        n += 1
+    assert n >= 3
+
+
+def pin_hand_pack(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "pack":
+            continue
+        codes = _ints(r["codes"], np.int8)[None, :]
+        packed, bad = O.pack(codes)
+        assert bad == 0
+        assert int(packed[0, 0]) == int(r["byte"], 16), (r, hex(packed[0, 0]))
+        assert np.array_equal(O.unpack(packed, 4), codes)
+        n += 1
+    assert n >= 8
+
+
+def pin_hand_matmul(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "matmul":
+            continue
+        K = int(r["K"])
+        xq = _ints(r["xq"], np.int8)[None, :]
+        codes = np.array([[int(v) for v in row.split(",")] for row in r["codes"].split(";")],
+                         dtype=np.int8)
+        acc = O.int_matmul(xq, codes)
+        assert np.array_equal(acc[0].astype(np.int64), _ints(r["acc"])), (r, acc)
+        s = np.array([float(r["s"])], np.float32)
+        y = O.dequant(acc, s, np.float32(float(r["gamma"])))
+        want = np.array([int(a) / int(r["y_den"]) for a in r["y_num"].split(",")])
+        assert np.allclose(y[0].astype(np.float64), want, rtol=1e-7, atol=0), (y, want)
+        packed, _ = O.pack(codes)
+        y2 = O.forward(xq, s, packed, np.float32(float(r["gamma"])), K)
+        assert np.array_equal(y2, y)
+        n += 1
+    assert n >= 1
+
+
+# --------------------------------------------------------------- closed forms --
+
+def pin_gaussian_statistics(O):
+    """W ~ N(0, sigma): E|w| = sigma sqrt(2/pi); a weight codes to 0 iff |w| <= gamma/2,
+    so the zero share is erf(gamma / (2 sigma sqrt 2)) for the sample's own gamma."""
+    sigma = 0.02
+    for seed in (0, 1, 2):
+        g = torch.Generator().manual_seed(seed)
+        W = (torch.randn(256, 512, generator=g) * sigma).numpy()
+        gamma = float(O.absmean_gamma(W, EPS))
+        n = W.size
+        mean_abs = sigma * math.sqrt(2 / math.pi)
+        sd_mean = sigma * math.sqrt(1 - 2 / math.pi) / math.sqrt(n)
+        assert abs((gamma - EPS) - mean_abs) < 5 * sd_mean, (gamma, mean_abs)
+        codes = O.ternarise(W, np.float32(gamma))
+        zero = float(np.mean(codes == 0))
+        p0 = math.erf(gamma / (2 * sigma * math.sqrt(2)))
+        assert abs(zero - p0) < 5 * math.sqrt(p0 * (1 - p0) / n), (zero, p0)
+        assert abs(zero - 0.3101) < 0.01
+        # the two signs are equally likely
+        plus, minus = float(np.mean(codes == 1)), float(np.mean(codes == -1))
+        assert abs(plus - minus) < 5 * math.sqrt(0.7 / n)
+
+
+def pin_constant_magnitude(O):
+    """|W| constant -> gamma = that constant + eps, codes = sign(W)."""
+    rng = np.random.default_rng(5)
+    for c in (0.25, 0.015625, 3.0):
+        W = np.where(rng.random((64, 128)) < 0.5, -c, c).astype(np.float32)
+        g = O.absmean_gamma(W, 2.0 ** -20)
+        assert g == np.float32(np.float32(c) + np.float32(2.0 ** -20))
+        assert np.array_equal(O.ternarise(W, g), np.sign(W).astype(np.int8))
+
+
+# ----------------------------------------------------------------- invariants --
+
+def pin_zero_weights(O):
+    W = np.zeros((16, 32), np.float32)
+    g = O.absmean_gamma(W, EPS)
+    assert g == np.float32(EPS)
+    codes = O.ternarise(W, g)
+    assert not codes.any()
+    packed, bad = O.pack(codes)
+    assert bad == 0 and not packed.any()
+    xq, s = O.quantize_act(_bf16_bits(np.random.default_rng(1).normal(size=(3, 32))), EPS)
+    assert not O.forward(xq, s, packed, g, 32).any()
+
+
+def pin_zero_token(O):
+    X = np.random.default_rng(2).normal(size=(4, 64)).astype(np.float32)
+    X[2] = 0.0
+    xq, s = O.quantize_act(_bf16_bits(X), EPS)
+    assert not xq[2].any()
+    codes = np.random.default_rng(3).integers(-1, 2, size=(8, 64)).astype(np.int8)
+    packed, _ = O.pack(codes)
+    y = O.forward(xq, s, packed, np.float32(0.03), 64)
+    assert not y[2].any() and y[[0, 1, 3]].any()
+
+
+def pin_code_alphabet_and_sign_symmetry(O):
+    g = torch.Generator().manual_seed(11)
+    W = (torch.randn(64, 256, generator=g) * 0.02).numpy()
+    gamma = O.absmean_gamma(W, EPS)
+    c = O.ternarise(W, gamma)
+    assert set(np.unique(c).tolist()) <= {-1, 0, 1}
+    assert O.absmean_gamma(-W, EPS) == gamma
+    assert np.array_equal(O.ternarise(-W, gamma), -c)
+
+
+def pin_act_range_and_symmetry(O):
+    g = torch.Generator().manual_seed(12)
+    X = torch.randn(32, 300, generator=g)
+    X[:, 7] *= 20
+    bits = _bf16_bits(X.numpy())
+    xq, s = O.quantize_act(bits, EPS)
+    xf = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    assert np.abs(xq.astype(np.int64)).max() <= 127
+    am = np.argmax(np.abs(xf), axis=1)
+    rows = np.arange(xf.shape[0])
+    assert np.array_equal(xq[rows, am].astype(np.int64), (127 * np.sign(xf[rows, am])).astype(np.int64))
+    xqn, sn = O.quantize_act(bits ^ np.uint16(0x8000), EPS)
+    assert np.array_equal(sn, s) and np.array_equal(xqn, -xq)
+
+
+def pin_permutation_and_linearity(O):
+    rng = np.random.default_rng(4)
+    M, N, K = 5, 7, 96
+    xa = rng.integers(-63, 64, size=(M, K)).astype(np.int8)
+    xb = rng.integers(-63, 64, size=(M, K)).astype(np.int8)
+    c = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    acc = O.int_matmul(xa, c)
+    perm = rng.permutation(K)
+    assert np.array_equal(O.int_matmul(xa[:, perm], c[:, perm]), acc)
+    assert np.array_equal(O.int_matmul((xa + xb).astype(np.int8), c), acc + O.int_matmul(xb, c))
+    # swapping the roles of two token rows swaps the output rows
+    assert np.array_equal(O.int_matmul(xa[[1, 0, 2, 3, 4]], c), acc[[1, 0, 2, 3, 4]])
+
+
+# -------------------------------------------------- independent implementations --
+
+def pin_matmul_vs_numpy(O):
+    rng = np.random.default_rng(6)
+    for (M, N, K) in [(1, 1, 4), (3, 17, 64), (16, 40, 260), (33, 9, 1000)]:
+        xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+        c = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        want = xq.astype(np.int64) @ c.astype(np.int64).T
+        assert np.array_equal(O.int_matmul(xq, c).astype(np.int64), want)
+        packed, _ = O.pack(c)
+        assert np.array_equal(O.forward(xq, np.ones(M, np.float32), packed, 1.0, K, 2), want)
+
+
+def pin_ternarise_vs_torch(O):
+    g = torch.Generator().manual_seed(7)
+    W = torch.randn(128, 192, generator=g) * 0.02
+    for gamma in (0.015, 0.0173, 0.02, 1e-3):
+        want = torch.round(W / torch.tensor(gamma, dtype=torch.float32)).clamp(-1, 1)
+        got = O.ternarise(W.numpy(), np.float32(gamma))
+        assert np.array_equal(got, want.to(torch.int8).numpy())
+    # values sitting exactly on the +-0.5 boundary
+    gamma = np.float32(0.0625)
+    Wt = np.array([[0.03125, -0.03125, 0.09375, -0.09375, 0.0312500037]], np.float32)
+    want = torch.round(torch.from_numpy(Wt) / torch.tensor(gamma)).clamp(-1, 1).to(torch.int8)
+    assert np.array_equal(O.ternarise(Wt, gamma), want.numpy())
+    # weights a few ulps either side of gamma/2 for many gammas: here an IEEE division
+    # and a multiply by a rounded reciprocal disagree on some codes
+    rng = np.random.default_rng(13)
+    for gamma in rng.uniform(0.005, 0.05, size=64).astype(np.float32):
+        half = np.float32(gamma * np.float32(0.5))
+        w = half + np.arange(-8, 9, dtype=np.float32) * np.spacing(half)
+        Wb = np.concatenate([w, -w]).astype(np.float32)[None, :]
+        want = torch.round(torch.from_numpy(Wb) / torch.tensor(gamma)).clamp(-1, 1).to(torch.int8)
+        assert np.array_equal(O.ternarise(Wb, gamma), want.numpy()), gamma
+
+
+def pin_act_vs_torch(O):
+    g = torch.Generator().manual_seed(8)
+    X = (torch.randn(64, 512, generator=g) * 3).to(torch.bfloat16)
+    X[5] = 0
+    X[6, :] = torch.tensor(1e-7).to(torch.bfloat16)
+    bits = X.view(torch.int16).numpy().view(np.uint16)
+    xf = X.float()
+    a = xf.abs().amax(dim=1)
+    s = torch.tensor(127.0) / torch.clamp(a, min=EPS)
+    xq = torch.round(xf * s[:, None]).clamp(-128, 127).to(torch.int8)
+    got_q, got_s = O.quantize_act(bits, EPS)
+    assert np.array_equal(got_s, s.numpy())
+    assert np.array_equal(got_q, xq.numpy())
+
+
+def pin_pack_vs_numpy(O):
+    rng = np.random.default_rng(9)
+    c = rng.integers(-1, 2, size=(13, 88)).astype(np.int8)
+    enc = np.where(c == 1, 1, np.where(c == -1, 2, 0)).astype(np.uint8)
+    want = (enc[:, 0::4] | (enc[:, 1::4] << 2) | (enc[:, 2::4] << 4) | (enc[:, 3::4] << 6))
+    packed, bad = O.pack(c)
+    assert bad == 0 and np.array_equal(packed, want.astype(np.uint8))
+    assert np.array_equal(O.unpack(packed, 88), c)
+    # invalid codes are counted and written as 00
+    cb = c.copy()
+    cb[0, 0], cb[3, 5] = 2, -7
+    packed_b, bad_b = O.pack(cb)
+    assert bad_b == 2
+    # byte 11 decodes to 0 everywhere
+    assert not O.unpack(np.full((2, 3), 0xFF, np.uint8), 12).any()
+
+
+def pin_dequant_vs_float64(O):
+    """y equals the float64 product of the dequantised operands (x_q / s)(gamma c)^T."""
+    rng = np.random.default_rng(10)
+    M, N, K = 9, 21, 320
+    xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    s = (rng.random(M) * 50 + 1).astype(np.float32)
+    c = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    gamma = np.float32(0.0173)
+    packed, _ = O.pack(c)
+    y = O.forward(xq, s, packed, gamma, K)
+    want = (xq.astype(np.float64) / s.astype(np.float64)[:, None]) @ (float(gamma) * c.astype(np.float64)).T
+    assert np.allclose(y.astype(np.float64), want, rtol=2e-7, atol=1e-12)
+    # bf16 output is torch's round-to-nearest-even of the fp32 output
+    yb = O.forward(xq, s, packed, gamma, K, 1)
+    assert np.array_equal(yb, torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+ALL_PINS = [
+    pin_hand_ternarise, pin_hand_absmean, pin_hand_act, pin_hand_pack, pin_hand_matmul,
+    pin_gaussian_statistics, pin_constant_magnitude, pin_zero_weights, pin_zero_token,
+    pin_code_alphabet_and_sign_symmetry, pin_act_range_and_symmetry,
+    pin_permutation_and_linearity, pin_matmul_vs_numpy, pin_ternarise_vs_torch,
+    pin_act_vs_torch, pin_pack_vs_numpy, pin_dequant_vs_float64,
+]

@@ -1,0 +1,67 @@
+"""The CPU oracle against its pins (hand cases, closed forms, invariants, independent
+library routines), and a check that those pins catch plausible mistakes planted in a
+copy of the oracle source."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+import oracle_pins
+
+pytestmark = pytest.mark.cpu
+
+
+@pytest.mark.parametrize("pin", oracle_pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(orc, pin):
+    pin(orc)
+
+
+# Each mutant is one plausible slip in the oracle: (name, text in the source, replacement).
+MUTANTS = [
+    ("round_half_away", "float q = rintf(W[i] / gamma);", "float q = roundf(W[i] / gamma);"),
+    ("reciprocal_multiply", "float q = rintf(W[i] / gamma);",
+     "float q = rintf(W[i] * (1.0f / gamma));"),
+    ("no_abs_in_gamma", "sum += fabs((double)W[n * K + k]);", "sum += (double)W[n * K + k];"),
+    ("eps_dropped", "float gamma = mean + eps;", "float gamma = mean;"),
+    ("mean_over_K_only", "float mean = (float)(sum / (double)(N * K));",
+     "float mean = (float)(sum / (double)K);"),
+    ("clip_to_two", "if (q > 1.0f) q = 1.0f;", "if (q > 2.0f) q = 2.0f;"),
+    ("codes_swapped", "if (c == 1) return 1;\n    if (c == -1) return 2;",
+     "if (c == 1) return 2;\n    if (c == -1) return 1;"),
+    ("msb_first", "byte |= (unsigned)e << (2 * i);", "byte |= (unsigned)e << (6 - 2 * i);"),
+    ("qb_128", "float s = 127.0f / fmaxf(a, eps);", "float s = 128.0f / fmaxf(a, eps);"),
+    ("act_round_away", "float q = rintf(bf16_bits_to_float(X[m * K + k]) * s);",
+     "float q = roundf(bf16_bits_to_float(X[m * K + k]) * s);"),
+    ("act_no_abs", "float v = fabsf(bf16_bits_to_float(X[m * K + k]));",
+     "float v = bf16_bits_to_float(X[m * K + k]);"),
+    ("transposed_codes", "int8_t c = codes[n * K + k];", "int8_t c = codes[k * N + n];"),
+    ("minus_is_plus", "else if (c == -1) sum -= xq[m * K + k];", "else if (c == -1) sum += xq[m * K + k];"),
+    ("scale_inverted", "(double)acc[m * N + n] * (double)gamma / (double)s[m]",
+     "(double)acc[m * N + n] * (double)gamma * (double)s[m]"),
+    ("gamma_dropped", "(double)acc[m * N + n] * (double)gamma / (double)s[m]",
+     "(double)acc[m * N + n] / (double)s[m]"),
+    ("bf16_truncate", "u += 0x7FFFu + lsb;", "u += 0u * lsb;"),
+    ("unpack_wrong_shift", "unsigned c = (byte >> (2 * (k % 4))) & 3u;",
+     "unsigned c = (byte >> (2 * (3 - k % 4))) & 3u;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_oracle_mutant_is_caught(tmp_path, name, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, "mutation anchor not found: %s" % name
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / ("lib_%s.so" % name)
+    subprocess.run(["gcc", *obuild.CFLAGS, str(mutated), "-o", str(lib), "-lm"], check=True,
+                   stderr=subprocess.DEVNULL)
+    M = oracle.Oracle(str(lib))
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(M)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, "no pin caught mutant %s" % name
