@@ -1,0 +1,405 @@
+"""Benchmark of the BitLinear forward hot path on B200.
+
+One step = one pass of every stage of the hot path over the seven BitLinear projections
+of one LLaMA-700M-shaped layer (hidden 1536, FFN 4096: q/k/v/o 1536x1536, up/gate
+1536->4096, down 4096->1536), fp32 N(0, 0.02) weights, bf16 heavy-tailed activations
+(1% of channels x20), at M = 1, 8, 512 and 4096 tokens:
+  a1+a2  absmean ternarisation + 2-bit packing of the 7 weight matrices,
+  a3     packing of 7 int8 code matrices of the same shapes,
+  a4     per-token int8 quantisation of each projection's input at every M,
+  a5-a7  the forward (decode GEMV for M <= 16, tcgen05 kind::i8 otherwise) with the
+         fused gamma / s epilogue, bf16 output.
+`value` is the forward work of the step (2 M N K ops summed over projections and M)
+divided by the device time of the whole step, in TOPS, summed over ranks (each rank
+runs its own step: weak scaling, no collective on the data path).
+
+Timing: the step is captured once in a CUDA graph with timing events around every
+library call; each timed replay is bracketed by events, L2 is flushed (256 MiB write)
+between replays outside the events, and K replays are bracketed by a barrier and a
+device synchronisation.  `e2e` repeats the step with its inputs copied from pinned
+host memory and its outputs copied back inside the timed region.
+
+--impl reference runs the CPU oracle (plain C, one core) on a bounded sample of the
+same workload and reports the same metric.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+EPS = 1e-5
+METRIC = "BitLinear fwd TOPS & weight GB/s at M=1..8192 vs B200 roofline"
+WORKLOAD = "llama700m"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ref-tokens", type=int, default=4,
+                   help="token rows per M in one reference-arm (oracle) step")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload():
+    from ternary_weight_bit_absmean_b200 import synth
+    spec = synth.WORKLOADS[WORKLOAD]
+    return spec["proj"], spec["M"], spec["outlier_frac"]
+
+
+def fwd_ops(projs, Ms):
+    return sum(2 * M * N * K for M in Ms for (_, N, K) in projs)
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % self.index)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ ours --
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from ternary_weight_bit_absmean_b200 import binding as B
+    from ternary_weight_bit_absmean_b200 import build_lib, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build_lib.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    projs, Ms, ofrac = workload()
+    # inputs: weights are the same model replica on every rank; tokens differ per rank
+    W = [synth.weight(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
+    C = [synth.codes(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
+    X = {(pi, M): synth.activations(M, K, seed=pi + 97 * M + 7919 * rank, outlier_frac=ofrac).to(dev)
+         for M in Ms for pi, (_, N, K) in enumerate(projs)}
+    gam = [torch.empty(1, dtype=torch.float32, device=dev) for _ in projs]
+    pk = [torch.empty(N, K // 4, dtype=torch.uint8, device=dev) for (_, N, K) in projs]
+    pk2 = [torch.empty(N, K // 4, dtype=torch.uint8, device=dev) for (_, N, K) in projs]
+    ws = [torch.empty(B.bitlinear_workspace_size(N, K), dtype=torch.uint8, device=dev) for (_, N, K) in projs]
+    xq = {(pi, M): torch.empty(M, K, dtype=torch.int8, device=dev) for M in Ms for pi, (_, N, K) in enumerate(projs)}
+    sc = {(pi, M): torch.empty(M, dtype=torch.float32, device=dev) for M in Ms for pi, _ in enumerate(projs)}
+    Y = {(pi, M): torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms for pi, (_, N, K) in enumerate(projs)}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # (label, callable) list in step order; labels name the hot-path row
+    calls = []
+    for pi, (_, N, K) in enumerate(projs):
+        calls.append((("a1a2", pi, 0), lambda pi=pi: B.bitlinear_quantize_weights(W[pi], EPS, gam[pi], pk[pi], ws[pi])))
+    for pi, _ in enumerate(projs):
+        calls.append((("a3", pi, 0), lambda pi=pi: B.bitlinear_pack(C[pi], pk2[pi])))
+    for M in sorted(Ms, reverse=True):
+        for pi, _ in enumerate(projs):
+            calls.append((("a4", pi, M), lambda pi=pi, M=M: B.bitlinear_quantize_act(X[pi, M], EPS, xq[pi, M], sc[pi, M])))
+            calls.append((("fwd", pi, M), lambda pi=pi, M=M: B.bitlinear_forward(xq[pi, M], sc[pi, M], pk[pi], gam[pi], Y[pi, M])))
+    launches_per_call = {"a1a2": 2, "a3": 1, "a4": 1, "fwd": 1}
+    launches_per_step = sum(launches_per_call[lab[0]] for lab, _ in calls)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(2):  # eager warm-up: first-call set-up (attributes, entry points)
+            for _, fn in calls:
+                fn()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in calls]
+    ev_step = (torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        ev_step[0].record()
+        for (lab, fn), (e0, e1) in zip(calls, ev):
+            e0.record()
+            fn()
+            e1.record()
+        ev_step[1].record()
+    torch.cuda.synchronize()
+
+    def one_step():
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            graph.replay()
+        torch.cuda.synchronize()
+        return ev_step[0].elapsed_time(ev_step[1]), [e0.elapsed_time(e1) for e0, e1 in ev]
+
+    for _ in range(max(3, args.warmup)):
+        one_step()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, call_ms = [], [0.0] * len(calls)
+    for _ in range(args.steps):
+        t, per = one_step()
+        step_ms.append(t)
+        call_ms = [a + b for a, b in zip(call_ms, per)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = sum(step_ms)
+    call_ms = [c / args.steps for c in call_ms]
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t.item()
+
+    # ---- end to end: pinned host inputs -> device, step, outputs -> pinned host
+    h_W = [w.cpu().pin_memory() for w in W]
+    h_C = [c.cpu().pin_memory() for c in C]
+    h_X = {k: v.cpu().pin_memory() for k, v in X.items()}
+    h_Y = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in Y.items()}
+    h2d = sum(t.numel() * t.element_size() for t in h_W + h_C + list(h_X.values()))
+    d2h = sum(t.numel() * t.element_size() for t in h_Y.values())
+    e2e_ms = []
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(args.e2e_steps + 1):
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            e_a.record()
+            for d, h in zip(W, h_W):
+                d.copy_(h, non_blocking=True)
+            for d, h in zip(C, h_C):
+                d.copy_(h, non_blocking=True)
+            for k, h in h_X.items():
+                X[k].copy_(h, non_blocking=True)
+            graph.replay()
+            for k, h in h_Y.items():
+                h.copy_(Y[k], non_blocking=True)
+            e_b.record()
+        torch.cuda.synchronize()
+        if i > 0:
+            e2e_ms.append(e_a.elapsed_time(e_b))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = t.item()
+
+    ops_step = fwd_ops(projs, Ms)
+    value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
+    e2e_value = ops_step * len(e2e_ms) * world / (e2e_total * 1e-3) / 1e12
+
+    # ---- per-row breakdown and the dominant kernel's roofline
+    pk_bytes = {pi: N * K // 4 for pi, (_, N, K) in enumerate(projs)}
+    by = {}
+    for (lab, _), ms in zip(calls, call_ms):
+        key = lab[0] if lab[0] in ("a1a2", "a3") else "%s_M%d" % (lab[0], lab[2])
+        by[key] = by.get(key, 0.0) + ms
+    fwd = {}
+    for M in Ms:
+        t_ms = by["fwd_M%d" % M]
+        ops = sum(2 * M * N * K for (_, N, K) in projs)
+        wbytes = sum(pk_bytes.values())
+        fwd[str(M)] = {"us": round(t_ms * 1e3, 2), "tops": round(ops / (t_ms * 1e-3) / 1e12, 2),
+                       "weight_gbs": round(wbytes / (t_ms * 1e-3) / 1e9, 1),
+                       "path": "gemv" if M <= 16 else "tcgen05"}
+    P = peaks()
+    int8_peak = 2.0 * P["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio 4.5 / 2.25 POPS)
+    Mbig = max(Ms)
+    dom_ms = by["fwd_M%d" % Mbig] / len(projs)
+    dom_ops = sum(2 * Mbig * N * K for (_, N, K) in projs) / len(projs)
+    achieved = dom_ops / (dom_ms * 1e-3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            tj = json.load(open(tpath))
+            from ternary_weight_bit_absmean_b200 import build_lib as _bl
+            if tj.get("source_digest") == _bl.source_digest():
+                traffic = tj.get("gemm_tc_M%d_bytes_per_launch" % Mbig)
+        except (ValueError, KeyError, AttributeError):
+            traffic = None
+    roofline = {"kernel": "gemm_tc (tcgen05 kind::i8), M=%d, mean over the 7 projections" % Mbig,
+                "bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4), "traffic": traffic,
+                "peak_note": "int8 dense = 2 x %s bf16 %.0f TFLOP/s (burst)" % (P["source"], P["bf16_tflops"])}
+    step_mean = total_ms / args.steps
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_mean, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+        "data": "synthetic (seeded N(0,0.02) fp32 weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
+        "config": {"workload": "llama700m BitLinear set: q/k/v/o 1536x1536, up/gate 1536->4096, down 4096->1536",
+                   "M": Ms, "out_dtype": "bf16", "eps": EPS,
+                   "stages": "a1+a2 quantize_weights x7, a3 pack x7, a4 quantize_act x28, a5/a6 forward x28",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "timing": "CUDA graph replay, device events, sum over steps, max over ranks",
+                   "parallelism": "dp%d (independent token batches per GPU, replicated weights)" % world},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": round(e2e_value, 4), "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "roofline": roofline,
+        "breakdown_us_per_step": {k: round(v * 1e3, 2) for k, v in sorted(by.items())},
+        "forward_by_M": fwd,
+        "hbm_peak_gbs": P["hbm_gbs"],
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(projs, Ms, ofrac, tokens=48)
+    graph.reset()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ---------------------------------------------------------- CPU oracle --
+
+def oracle_sample(projs, Ms, ofrac, tokens, seed_base=0):
+    """Run the oracle on a bounded sample of one step: the full weight quantisation of
+    every projection, plus activation quantisation and forward of min(M, tokens) token
+    rows at every M.  Returns (forward ops in the sample, seconds)."""
+    import numpy as np
+
+    import oracle
+    from ternary_weight_bit_absmean_b200 import synth
+    inputs = []
+    for pi, (_, N, K) in enumerate(projs):
+        Wn = synth.weight(N, K, seed=pi).numpy()
+        Xs = {M: synth.bf16_bits(synth.activations(min(M, tokens), K, seed=seed_base + pi + 97 * M,
+                                                   outlier_frac=ofrac)) for M in Ms}
+        inputs.append((Wn, Xs, K))
+    oracle.default()
+    t0 = time.perf_counter()
+    ops = 0
+    for Wn, Xs, K in inputs:
+        g, codes, packed = oracle.quantize_weights(Wn, EPS)
+        for M in Ms:
+            xq, s = oracle.quantize_act(Xs[M], EPS)
+            y = oracle.forward(xq, s, packed, g, K, oracle.OUT_BF16)
+            ops += 2 * xq.shape[0] * packed.shape[0] * K
+            assert y.shape[0] == xq.shape[0]
+    return ops, time.perf_counter() - t0, np
+
+
+def cpu_baseline(projs, Ms, ofrac, tokens):
+    ops, secs, _ = oracle_sample(projs, Ms, ofrac, tokens)
+    return {"value": round(ops / secs / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": "full weight quantisation of the 7 projections + act quantisation and forward of "
+                      "min(M, %d) token rows at each M (%.2f GOP forward, %.1f s)" % (tokens, ops / 1e9, secs)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    projs, Ms, ofrac = workload()
+    for i in range(args.warmup):
+        oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=i)
+    total_ops, total_s = 0, 0.0
+    for i in range(args.steps):
+        ops, secs, _ = oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=1000 + i)
+        total_ops += ops
+        total_s += secs
+    value = total_ops / total_s / 1e12
+    sample = ("per step: full weight quantisation of the 7 projections + act quantisation and forward "
+              "of min(M, %d) token rows at each M (CPU oracle, plain C, one core)" % args.ref_tokens)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_s / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+        "data": "synthetic", "config": {"workload": "llama700m BitLinear set (bounded oracle sample)",
+                                        "M": Ms, "tokens_per_M": args.ref_tokens},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,168 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so, the B200 (sm_100a) BitNet b1.58 BitLinear
+ * forward pass.
+ *
+ * Conventions shared by every entry point
+ *   - Data pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates, frees or copies on these calls and never synchronises; each call only
+ *     enqueues kernels on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) and returns.
+ *   - Dimensions are int64_t.  Matrices are dense row-major: W is [N, K] (nn.Linear
+ *     convention, N = out features, K = in features), X / x_q are [M, K], y is [M, N].
+ *   - Base pointers must be 16-byte aligned (cudaMalloc and PyTorch allocations are).
+ *   - Argument errors are detected on the host before any launch and leave every
+ *     output untouched.  A launch error returns BL_ERR_CUDA (the CUDA error code is
+ *     kept for bitlinear_last_cuda_error()).  Faults inside a kernel surface at the
+ *     caller's next synchronisation of `stream`, as for any CUDA kernel.
+ *   - Optional `err_word` (device int32, may be NULL): kernels OR status bits into it
+ *     (BL_ERRBIT_*) for conditions only the device can see.  The caller zeroes it.
+ *   - Calls are reentrant: there is no hidden state besides the last CUDA error code.
+ *
+ * Packed ternary weight format (the only weight format the forward reads)
+ *   uint8 [N, K/4], row-major, K % 4 == 0.  Byte j of row n holds the codes of
+ *   elements k = 4j + i (i = 0..3) in bits 2i..2i+1, least significant first:
+ *   00 -> 0, 01 -> +1, 10 -> -1.  11 is never written by this library; the forward
+ *   reads it as 0.
+ *
+ * Sources (page title -- section):
+ *   [B158] "1-bit & Ternary LLMs (BitNet b1.58)" -- "How it works (real mechanics)",
+ *          block "BitNet b1.58 (Feb 2024)": gamma = (1/nm) sum |W_ij|,
+ *          W~ = RoundClip(W / (gamma + eps), -1, 1).
+ *   [BIN]  same page, block "BitNet (Oct 2023)": absmax per-token activation
+ *          quantisation and y = W~ . Quant(LN(x)) . (beta gamma / Q_b).
+ *   [STE]  same page, "Training: shadow weights + the straight-through estimator":
+ *          y = (W_eff @ x_q) * scale, an integer matmul plus one float rescale.
+ *   [CH2]  "What 1.58 Bits Actually Changes" -- "How the low-bit linear path works":
+ *          per-token signed 8-bit activations without a zero point; +1 adds, -1
+ *          subtracts, 0 skips; packed ternary values are loaded and unpacked.
+ *
+ * Readings where the pages are silent: round = half to even; gamma includes eps
+ * everywhere (division and output scale); Q_b = 127 with clip [-128, 127]; true IEEE
+ * division for W / gamma and 127 / absmax; y = acc * gamma / s_m.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BL_API __attribute__((visibility("default")))
+#else
+#define BL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_INVALID_ARG = 1,       /* NULL pointer, non-positive size, eps <= 0 or not finite */
+    BL_ERR_UNSUPPORTED_SHAPE = 2, /* K % 4 != 0, or a size whose int32 sums could overflow */
+    BL_ERR_MISALIGNED = 3,        /* a base pointer is not 16-byte aligned */
+    BL_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than bitlinear_workspace_size */
+    BL_ERR_CUDA = 5,              /* a launch or attribute call failed */
+    BL_ERR_TIMEOUT = 6,           /* (err_word bit) a bounded device wait gave up */
+    BL_ERR_BAD_CODE = 7           /* (err_word bit) an input code outside {-1, 0, +1} */
+} bl_status;
+
+/* Bits OR-ed into the optional device err_word. */
+#define BL_ERRBIT_BAD_CODE 0x1
+#define BL_ERRBIT_TIMEOUT 0x2
+
+typedef enum {
+    BL_OUT_F32 = 0,  /* y as fp32 */
+    BL_OUT_BF16 = 1, /* y as bf16 (round to nearest even of the fp32 value) */
+    BL_OUT_I32 = 2   /* the raw int32 accumulators acc = x_q . c^T, no rescale */
+} bl_dtype;
+
+typedef enum {
+    BL_PATH_AUTO = 0, /* GEMV for M <= 16 (or shapes the tensor-core path cannot tile), else tcgen05 */
+    BL_PATH_GEMV = 1, /* register-unpack GEMV, any M (token tiles of 16) */
+    BL_PATH_TC = 2    /* tcgen05 kind::i8 tiled path; needs K % 64 == 0 */
+} bl_path;
+
+/* Bytes of device workspace bitlinear_quantize_weights needs for an [N, K] matrix
+ * (fp64 partial sums of |W|).  Depends on N*K only; 0 for a non-positive size. */
+BL_API size_t bitlinear_workspace_size(int64_t N, int64_t K);
+
+/* [B158] absmean ternarisation and packing of one weight matrix.
+ *   W          in  : fp32 [N, K] row-major, device.
+ *   eps        in  : > 0, finite; gamma = fp32(mean|W|) + eps (fp32 add).
+ *   gamma_out  out : device fp32 scalar; written by the kernels, never read back here.
+ *   packed_out out : device uint8 [N, K/4] in the packed format above.
+ *   ws, ws_bytes   : device workspace of at least bitlinear_workspace_size(N, K) bytes,
+ *                    scratch for the duration of the enqueued work.
+ * The sum of |W| is accumulated in fp64 per thread and per block, and the block
+ * partials are summed in a fixed order, so gamma is deterministic from run to run.
+ * Codes: clip(rint(W / gamma), -1, 1) with an IEEE fp32 division.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 4), BL_ERR_MISALIGNED,
+ * BL_ERR_WORKSPACE, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_quantize_weights(const float *W, int64_t N, int64_t K, float eps,
+                                     float *gamma_out, uint8_t *packed_out,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* [B158] the RoundClip step alone, with the scale supplied by the caller.
+ *   W      in  : fp32 [N, K], device.
+ *   gamma  in  : device fp32 scalar, the full divisor (mean|W| + eps), > 0.
+ *   packed_out out : device uint8 [N, K/4].
+ * Errors: as bitlinear_quantize_weights, without BL_ERR_WORKSPACE. */
+BL_API bl_status bitlinear_quantize_weights_with_scale(const float *W, int64_t N, int64_t K,
+                                                const float *gamma, uint8_t *packed_out,
+                                                void *stream);
+
+/* [CH2] pack ternary codes given as int8.
+ *   codes      in  : int8 [N, K] in {-1, 0, +1}, device.
+ *   packed_out out : device uint8 [N, K/4].
+ *   err_word   out : optional; BL_ERRBIT_BAD_CODE is OR-ed in if any code is outside
+ *                    {-1, 0, +1}; such a code is written as 00 (zero).
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_pack(const int8_t *codes, int64_t N, int64_t K, uint8_t *packed_out,
+                         int32_t *err_word, void *stream);
+
+/* [BIN] + [CH2] per-token absmax int8 quantisation with no zero point.
+ *   X      in  : bf16 [M, K] as raw uint16 bit patterns, device.  Finite values.
+ *   eps    in  : > 0, finite.
+ *   xq_out out : int8 [M, K], device: clip(rint(x * s_m), -128, 127).
+ *   s_out  out : fp32 [M], device: s_m = 127 / max(max_k |x_mk|, eps) (IEEE division).
+ * Any K >= 1 is accepted.  Errors: BL_ERR_INVALID_ARG, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_quantize_act(const uint16_t *X, int64_t M, int64_t K, float eps,
+                                 int8_t *xq_out, float *s_out, void *stream);
+
+/* [BIN] + [STE] + [CH2] the BitLinear forward from quantised operands:
+ *   acc[m, n] = sum_k x_q[m, k] * c[n, k]   (exact, int32)
+ *   y[m, n]   = float(acc[m, n]) * (gamma / s[m])   (fp32: the quotient and the product
+ *               are each rounded to nearest, so y is within 2^-23 relative of the exact
+ *               value; bf16 output is the round-to-nearest-even of that fp32 value)
+ *   xq      in  : int8 [M, K], device.
+ *   s       in  : fp32 [M], device (ignored for BL_OUT_I32 but must be valid).
+ *   packed  in  : uint8 [N, K/4] packed codes, device.
+ *   gamma   in  : device fp32 scalar.
+ *   out     out : [M, N] of out_dtype, device.
+ *   err_word out: optional; BL_ERRBIT_TIMEOUT if a bounded device wait gave up (the
+ *                 output is then incomplete).
+ * M <= 16 runs the register-unpack GEMV; larger M runs the tcgen05 kind::i8 path when
+ * K % 64 == 0 (else the GEMV).  K * 127 must stay below 2^31.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_forward(const int8_t *xq, const float *s, const uint8_t *packed,
+                            const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
+                            bl_dtype out_dtype, int32_t *err_word, void *stream);
+
+/* bitlinear_forward with the kernel choice forced (testing both paths at any M). */
+BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const uint8_t *packed,
+                                 const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
+                                 bl_dtype out_dtype, int32_t *err_word, bl_path path,
+                                 void *stream);
+
+/* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
+BL_API int bitlinear_last_cuda_error(void);
+
+/* Static string naming a bl_status value. */
+BL_API const char *bitlinear_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

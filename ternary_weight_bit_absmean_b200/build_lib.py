@@ -1,0 +1,70 @@
+"""Build ``libbitlinear.so`` (the CUDA kernels and the C ABI) in-tree for sm_100a.
+
+``python -m ternary_weight_bit_absmean_b200.build_lib [--force] [--verbose]``
+
+The library is compiled with nvcc for ``sm_100a`` only, position independent, with the
+CUDA runtime linked statically (no dependency on the runtime that PyTorch ships) and
+without linking the driver library (the tensor-map encoder is fetched through the
+runtime's driver entry point), so it loads on a machine without a GPU.
+"""
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libbitlinear.so")
+SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemm_tc.cu"]
+HEADERS = ["bl_device.cuh", "bl_internal.h"]
+
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+         "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-cudart", "static"]
+
+
+def _inputs():
+    return ([os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+            + [os.path.join(INCLUDE, "bitlinear.h"), os.path.abspath(__file__)])
+
+
+def source_digest() -> str:
+    """SHA-256 over the library's sources and header (identifies a kernel build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "bitlinear.h")]:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(p) <= t for p in _inputs())
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return LIB
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    objs = []
+    for src in SOURCES:
+        obj = os.path.join(objdir, src.replace(".cu", ".o"))
+        cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        subprocess.run(cmd, check=True)
+        objs.append(obj)
+    tmp = LIB + ".tmp.%d" % os.getpid()
+    subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
+                    *objs, "-o", tmp], check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

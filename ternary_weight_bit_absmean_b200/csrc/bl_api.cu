@@ -1,0 +1,148 @@
+// bl_api.cu -- the C ABI of libbitlinear.so (declared in include/bitlinear.h): argument
+// validation on the host, workspace checks, and dispatch to the kernels.  No call here
+// allocates, frees, copies or synchronises; every kernel is enqueued on the caller's
+// stream.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "bitlinear.h"
+#include "bl_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool eps_ok(float eps) { return std::isfinite(eps) && eps > 0.0f; }
+
+bl_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return BL_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return BL_ERR_CUDA;
+}
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Shapes shared by the weight entry points.
+bl_status check_weight_shape(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (N > (int64_t(1) << 40) / K) return BL_ERR_UNSUPPORTED_SHAPE;
+    return BL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitlinear_workspace_size(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return 0;
+    return static_cast<size_t>(bl::absmean_num_partials(N * K)) * sizeof(double);
+}
+
+bl_status bitlinear_quantize_weights(const float* W, int64_t N, int64_t K, float eps, float* gamma_out,
+                                     uint8_t* packed_out, void* ws, size_t ws_bytes, void* stream) {
+    if (W == nullptr || gamma_out == nullptr || packed_out == nullptr || !eps_ok(eps))
+        return BL_ERR_INVALID_ARG;
+    bl_status st = check_weight_shape(N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(W) || !aligned16(packed_out) || !aligned16(gamma_out)) return BL_ERR_MISALIGNED;
+    const size_t need = bitlinear_workspace_size(N, K);
+    if (ws == nullptr || ws_bytes < need) return BL_ERR_WORKSPACE;
+    if (!aligned16(ws)) return BL_ERR_MISALIGNED;
+    const int64_t numel = N * K;
+    const int nparts = bl::absmean_num_partials(numel);
+    double* partials = static_cast<double*>(ws);
+    cudaError_t e = bl::launch_absmean_partials(W, numel, partials, nparts, as_stream(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    e = bl::launch_ternarise_pack(W, numel, nullptr, partials, nparts, eps, gamma_out, packed_out,
+                                  as_stream(stream));
+    return cuda_status(e);
+}
+
+bl_status bitlinear_quantize_weights_with_scale(const float* W, int64_t N, int64_t K, const float* gamma,
+                                                uint8_t* packed_out, void* stream) {
+    if (W == nullptr || gamma == nullptr || packed_out == nullptr) return BL_ERR_INVALID_ARG;
+    bl_status st = check_weight_shape(N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(W) || !aligned16(packed_out)) return BL_ERR_MISALIGNED;
+    cudaError_t e = bl::launch_ternarise_pack(W, N * K, gamma, nullptr, 0, 0.0f, nullptr, packed_out,
+                                              as_stream(stream));
+    return cuda_status(e);
+}
+
+bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, uint8_t* packed_out, int32_t* err_word,
+                         void* stream) {
+    if (codes == nullptr || packed_out == nullptr) return BL_ERR_INVALID_ARG;
+    bl_status st = check_weight_shape(N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(codes) || !aligned16(packed_out)) return BL_ERR_MISALIGNED;
+    cudaError_t e = bl::launch_pack_codes(codes, N * K, packed_out, err_word, as_stream(stream));
+    return cuda_status(e);
+}
+
+bl_status bitlinear_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
+                                 float* s_out, void* stream) {
+    if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 40) / K) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(X) || !aligned16(xq_out) || !aligned16(s_out)) return BL_ERR_MISALIGNED;
+    cudaError_t e = bl::launch_quantize_act(X, M, K, eps, xq_out, s_out, as_stream(stream));
+    return cuda_status(e);
+}
+
+bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                                 int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                 int32_t* err_word, bl_path path, void* stream) {
+    if (xq == nullptr || s == nullptr || packed == nullptr || gamma == nullptr || out == nullptr)
+        return BL_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32)
+        return BL_ERR_INVALID_ARG;
+    if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC) return BL_ERR_INVALID_ARG;
+    if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    // |acc| <= 128 K must fit in int32; sizes must fit the kernels' 32-bit indexing.
+    if (K > (int64_t(1) << 31) / 128 - 1) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(xq) || !aligned16(s) || !aligned16(packed) || !aligned16(out)) return BL_ERR_MISALIGNED;
+    const bool k64 = (K % 64) == 0;
+    if (path == BL_PATH_TC && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (path == BL_PATH_AUTO) path = (M <= 16 || !k64) ? BL_PATH_GEMV : BL_PATH_TC;
+    const int kind = static_cast<int>(out_dtype);
+    cudaError_t e;
+    if (path == BL_PATH_TC) {
+        e = bl::launch_gemm_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+    } else if (k64 && M <= int64_t(65535) * 16) {
+        e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, as_stream(stream));
+    } else {
+        e = bl::launch_gemv_generic(xq, s, packed, gamma, M, N, K, out, kind, as_stream(stream));
+    }
+    return cuda_status(e);
+}
+
+bl_status bitlinear_forward(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                            int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                            int32_t* err_word, void* stream) {
+    return bitlinear_forward_path(xq, s, packed, gamma, M, N, K, out, out_dtype, err_word, BL_PATH_AUTO,
+                                  stream);
+}
+
+int bitlinear_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* bitlinear_status_string(int status) {
+    switch (status) {
+        case BL_OK: return "BL_OK";
+        case BL_ERR_INVALID_ARG: return "BL_ERR_INVALID_ARG";
+        case BL_ERR_UNSUPPORTED_SHAPE: return "BL_ERR_UNSUPPORTED_SHAPE";
+        case BL_ERR_MISALIGNED: return "BL_ERR_MISALIGNED";
+        case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE";
+        case BL_ERR_CUDA: return "BL_ERR_CUDA";
+        case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT";
+        case BL_ERR_BAD_CODE: return "BL_ERR_BAD_CODE";
+        default: return "BL_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// bl_internal.h -- launchers shared between the kernel files and the C-ABI layer.
+// Every launcher enqueues on `stream` and returns the cudaError_t of its launch.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bl {
+
+// Weight quantisation (absmean partial sums, ternarise + pack, pack of int8 codes).
+int absmean_num_partials(int64_t numel);
+cudaError_t launch_absmean_partials(const float* W, int64_t numel, double* partials, int nparts,
+                                    cudaStream_t stream);
+// gamma from the partials (gamma_in == nullptr) or given (gamma_in != nullptr).
+cudaError_t launch_ternarise_pack(const float* W, int64_t numel, const float* gamma_in,
+                                  const double* partials, int nparts, float eps,
+                                  float* gamma_out, uint8_t* packed, cudaStream_t stream);
+cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packed, int32_t* err,
+                              cudaStream_t stream);
+
+// Per-token absmax int8 activation quantisation.
+cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
+                                float* s, cudaStream_t stream);
+
+// Output kinds (mirror bl_dtype).
+enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
+
+// Decode GEMV: register unpack + mma.sync, any M (token groups of 16), K % 64 == 0.
+cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
+                        const float* gamma, int64_t M, int64_t N, int64_t K, void* out, int kind,
+                        cudaStream_t stream);
+// Plain fallback for K % 64 != 0 (one output per thread).
+cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
+                                const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
+                                int kind, cudaStream_t stream);
+
+// Tiled tcgen05 kind::i8 path (K % 64 == 0).
+cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed,
+                           const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
+                           int kind, int32_t* err, cudaStream_t stream);
+
+}  // namespace bl

@@ -1,0 +1,396 @@
+// k_gemm_tc.cu -- prefill-regime BitLinear forward on the 5th-generation tensor cores
+// (tcgen05.mma kind::i8, int32 accumulators in tensor memory).
+//
+// What is computed ("1-bit & Ternary LLMs (BitNet b1.58)", block "BitNet (Oct 2023)":
+// y = W~ . Quant(x) . scale, an integer product and one float rescale; block
+// "BitNet b1.58 (Feb 2024)": W~ in {-1, 0, +1}; "1.58 bits: what BitNet promised and what
+// it required", "What you get on today's hardware": on GPUs the packed weights are
+// unpacked and then multiplied):
+//   acc[m, n] = sum_k x_q[m, k] * c[n, k]   (int32, exact)
+//   y[m, n]   = acc[m, n] * gamma / s[m]
+//
+// Tile: 128 output features (MMA M, TMEM lanes) x BT tokens (MMA N, TMEM columns), K in
+// stages of 128 bytes.  The weights are the A operand so that the expansion work per
+// MMA is 128 x 32 codes whatever the token tile, and each expanded code is reused by BT
+// tokens.  Per stage:
+//   warp 0 (one lane)  TMA: x_q tile [BT x 128 B] (128-byte swizzle) and the packed
+//                      weight tile [128 x 32 B] into shared memory, one mbarrier;
+//   warps 2-5          expanders: thread e unpacks packed row e (128 codes) into int8 and
+//                      writes it in the same 128-byte-swizzled K-major layout;
+//   warp 1 (one lane)  MMA issuer: four tcgen05.mma (K = 32 each) per stage into a TMEM
+//                      accumulator, tcgen05.commit frees the stage;
+//   warps 6-9          epilogue: tcgen05.ld of the finished accumulator (one feature row
+//                      per thread), y = acc * (gamma / s_m), coalesced stores along N.
+// Two TMEM accumulators let the epilogue of one tile overlap the main loop of the next
+// (persistent blocks, one per SM, static round-robin over tiles).  Ragged M, N and K
+// edges come from TMA zero fill: a zero packed byte is four zero codes.
+//
+// Every wait is bounded: a role that waits longer than kWaitTimeoutNs raises an abort
+// flag, the other roles leave their loops, outstanding TMA loads and MMAs are drained,
+// TMEM is freed and BL_ERRBIT_TIMEOUT is OR-ed into the caller's error word.
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "bl_device.cuh"
+#include "bl_internal.h"
+
+namespace bl {
+namespace {
+
+constexpr int kBN = 128;          // output features per tile (MMA M)
+constexpr int kBK = 128;          // K bytes per stage (one 128-byte swizzle row)
+constexpr int kThreads = 320;     // 10 warps
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2, kWarpEpi = 6;
+constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
+
+template <int BT>
+struct TcCfg {
+    static_assert(BT == 32 || BT == 64 || BT == 128 || BT == 256, "token tile");
+    static constexpr int kXBytes = BT * kBK;
+    static constexpr int kABytes = kBN * kBK;
+    static constexpr int kPBytes = kBN * (kBK / 4);
+    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes;
+    static constexpr int kStagesRaw = (220 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kTmemCols = 2 * BT;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 5) + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
+    static_assert(kStages >= 2, "stages");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct TcArgs {
+    const float* s;
+    const float* gamma;
+    int M, N, K;
+    int n_tiles_n, num_tiles;
+    void* out;
+    int kind;
+    int32_t* err;
+};
+
+__device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
+    if (kind == kOutI32) {
+        static_cast<int*>(out)[idx] = acc;
+        return;
+    }
+    const float y = __fmul_rn(__int2float_rn(acc), fac);
+    if (kind == kOutF32)
+        static_cast<float*>(out)[idx] = y;
+    else
+        static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(y);
+}
+
+// Wait for the given phase parity of `bar`, giving up after `limit_ns` regardless of
+// the abort flag (used only to drain after an abort).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kDrainTimeoutNs) return;
+    }
+}
+
+template <int BT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
+                   const TcArgs a) {
+    using C = TcCfg<BT>;
+    constexpr int ST = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sX = base;
+    const uint32_t sA = sX + ST * C::kXBytes;
+    const uint32_t sP = sA + ST * C::kABytes;
+    const uint32_t sBar = sP + ST * C::kPBytes;
+    auto full = [&](int s) { return sBar + 8u * s; };
+    auto afull = [&](int s) { return sBar + 8u * (ST + s); };
+    auto empty = [&](int s) { return sBar + 8u * (2 * ST + s); };
+    auto tfull = [&](int b) { return sBar + 8u * (3 * ST + b); };
+    auto tempty = [&](int b) { return sBar + 8u * (3 * ST + 2 + b); };
+    const uint32_t drain_bar = sBar + 8u * (3 * ST + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (sBar - base) + 8 * (3 * ST + 5));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(afull(s), 4);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 4);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_p);
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nK = (a.K + kBK - 1) / kBK;
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ producer --
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+                const int n0 = (tile % a.n_tiles_n) * kBN;
+                const int t0 = (tile / a.n_tiles_n) * BT;
+                for (int kt = 0; kt < nK; ++kt) {
+                    if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full(stage), C::kXBytes + C::kPBytes);
+                    tma_load_2d(sX + stage * C::kXBytes, &tmap_x, full(stage), kt * kBK, t0);
+                    tma_load_2d(sP + stage * C::kPBytes, &tmap_p, full(stage), kt * (kBK / 4), n0);
+                    ++issued;
+                    if (++stage == ST) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // wait for every load still in flight before the block may exit
+                for (int s = 0; s < ST; ++s) {
+                    const long long fills = (issued - s + ST - 1) / ST;  // loads issued into stage s
+                    if (fills > 0) mbar_drain(full(s), static_cast<uint32_t>((fills - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc = idesc_i8(kBN, BT);
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+                if (!mbar_wait_bounded(tempty(buf), bphase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BT);
+                for (int kt = 0; kt < nK; ++kt) {
+                    if (!mbar_wait_bounded(full(stage), phase, abort_flag) ||
+                        !mbar_wait_bounded(afull(stage), phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = sA + stage * C::kABytes;
+                    const uint32_t b_addr = sX + stage * C::kXBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        tc_mma_i8(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32),
+                                  idesc, (kt | kk) != 0 ? 1u : 0u);
+                    tc_commit(empty(stage));
+                    if (++stage == ST) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(tfull(buf));
+                if (++buf == 2) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+            if (!ok) {
+                // let every MMA already issued finish before TMEM is released
+                tc_commit(drain_bar);
+                mbar_drain(drain_bar, 0);
+            }
+        }
+    } else if (warp < kWarpEpi) {
+        // ------------------------------------------------------------- expanders --
+        const int e = threadIdx.x - 32 * kWarpExp;  // weight row within the tile, 0..127
+        const uint32_t sw = static_cast<uint32_t>(e & 7);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+            for (int kt = 0; kt < nK; ++kt) {
+                if (!mbar_wait_bounded(full(stage), phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* pp = gbase + (sP - base) + stage * C::kPBytes + e * (kBK / 4);
+                const uint4 p0 = *reinterpret_cast<const uint4*>(pp);
+                const uint4 p1 = *reinterpret_cast<const uint4*>(pp + 16);
+                uint8_t* ap = gbase + (sA - base) + stage * C::kABytes + e * kBK;
+                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 u;
+                    unpack16_natural(words[c], u.x, u.y, u.z, u.w);
+                    *reinterpret_cast<uint4*>(ap + ((static_cast<uint32_t>(c) ^ sw) << 4)) = u;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(afull(stage));
+                if (++stage == ST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue --
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+            const int n0 = (tile % a.n_tiles_n) * kBN;
+            const int t0 = (tile / a.n_tiles_n) * BT;
+            if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag)) break;
+            tc_fence_after();
+            const int row = n0 + 32 * q + lane;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BT; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(buf * BT + c0),
+                                   r);
+                tmem_ld_wait();
+                const int tk = t0 + c0 + lane;
+                const float fac = (a.kind != kOutI32 && tk < a.M) ? __fdiv_rn(gamma, a.s[tk]) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float fj = __shfl_sync(0xffffffffu, fac, j);
+                    const int tok = t0 + c0 + j;
+                    if (tok < a.M && row < a.N)
+                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
+                                static_cast<int>(r[j]), fj);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty(buf));
+            if (++buf == 2) {
+                buf = 0;
+                bphase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && a.err != nullptr) atomicOr(a.err, kErrBitTimeout);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool encode_2d_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer, CUtensorMapSwizzle swz) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BT>
+cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms, cudaStream_t stream) {
+    using C = TcCfg<BT>;
+    CUtensorMap tx, tp;
+    if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, BT,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d_u8(&tp, packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
+                      kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+    }
+    const int grid = a.num_tiles < sms ? a.num_tiles : sms;
+    gemm_tc_kernel<BT><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                           int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                           cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t nN = (N + kBN - 1) / kBN;
+    // Token tile: per K step an MMA of 128 x BT costs ~BT/2 cycles at peak while the
+    // expansion of 128 x 32 codes costs a fixed ~64; pick the tile with the fewest
+    // waves x cycles per tile.
+    int bt = 256;
+    if (M <= 32) {
+        bt = 32;
+    } else if (M <= 64) {
+        bt = 64;
+    } else {
+        auto cost = [&](int b) {
+            const int64_t tiles = nN * ((M + b - 1) / b);
+            const int64_t waves = (tiles + sms - 1) / sms;
+            const int64_t per = (b / 2 > 64 ? b / 2 : 64) + 16;
+            return waves * per;
+        };
+        bt = cost(128) < cost(256) ? 128 : 256;
+    }
+    TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
+             0, out, kind, err};
+    a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
+    switch (bt) {
+        case 32: return launch_bt<32>(xq, packed, a, sms, stream);
+        case 64: return launch_bt<64>(xq, packed, a, sms, stream);
+        case 128: return launch_bt<128>(xq, packed, a, sms, stream);
+        default: return launch_bt<256>(xq, packed, a, sms, stream);
+    }
+}
+
+}  // namespace bl

@@ -1,0 +1,314 @@
+// k_quant.cu -- the HBM-bound quantisation kernels of the BitLinear forward:
+//   * absmean partial sums of |W| (fp64) and the fused gamma + ternarise + 2-bit pack,
+//   * packing of caller-supplied int8 ternary codes,
+//   * per-token absmax int8 activation quantisation.
+//
+// Definitions ("1-bit & Ternary LLMs (BitNet b1.58)", "How it works", block
+// "BitNet b1.58 (Feb 2024)"): gamma = (1/nm) sum |W_ij| (+ eps),
+// W~ = RoundClip(W / gamma, -1, 1).  Block "BitNet (Oct 2023)" and "What 1.58 Bits
+// Actually Changes" ("How the low-bit linear path works"): activations scaled per token
+// by their absmax to signed 8 bits with no zero point.
+//
+// Bit-exactness: every float step is the IEEE operation the definition names --
+// __fdiv_rn for W / gamma and 127 / absmax, __fmul_rn for x * s, __float2int_rn
+// (round half to even) for round(); nothing here is compiled with fast-math.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "bl_device.cuh"
+#include "bl_internal.h"
+
+namespace bl {
+namespace {
+
+constexpr int kAbsThreads = 256;
+constexpr int kAbsMaxParts = 148 * 8;
+
+// 2-bit code of round-half-even(t) clipped to [-1, 1]: 01 for +1, 10 for -1, 00 for 0.
+__device__ __forceinline__ uint32_t code_of_ratio(float t) {
+    const int q = __float2int_rn(t);
+    return q >= 1 ? 1u : (q <= -1 ? 2u : 0u);
+}
+
+__device__ __forceinline__ uint32_t pack4_codes(float4 w, float gamma) {
+    return code_of_ratio(__fdiv_rn(w.x, gamma)) | (code_of_ratio(__fdiv_rn(w.y, gamma)) << 2) |
+           (code_of_ratio(__fdiv_rn(w.z, gamma)) << 4) | (code_of_ratio(__fdiv_rn(w.w, gamma)) << 6);
+}
+
+// ---------------------------------------------------------- absmean partials --
+// Each block accumulates |W| over a grid-stride range of float4s in fp64 and writes
+// one fp64 partial.  The partials are summed in a fixed order by the pack kernel.
+__global__ void __launch_bounds__(kAbsThreads) absmean_partials_kernel(const float4* __restrict__ W4,
+                                                                      int64_t n4,
+                                                                      double* __restrict__ partials) {
+    double acc = 0.0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kAbsThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kAbsThreads + threadIdx.x; i < n4;
+         i += stride) {
+        const float4 v = __ldg(W4 + i);
+        acc += static_cast<double>(fabsf(v.x));
+        acc += static_cast<double>(fabsf(v.y));
+        acc += static_cast<double>(fabsf(v.z));
+        acc += static_cast<double>(fabsf(v.w));
+    }
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    __shared__ double warp_sum[kAbsThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < kAbsThreads / 32; ++w) t += warp_sum[w];
+        partials[blockIdx.x] = t;
+    }
+}
+
+// -------------------------------------------------------- ternarise + pack --
+// Every block first forms gamma: from the caller's device scalar, or by summing the
+// absmean partials in a fixed order (identical in every block), dividing by N*K in
+// fp64, rounding to fp32 and adding eps in fp32.  Block 0 stores it.  Then each thread
+// turns 16 weights (four float4) into one 32-bit word of packed codes.
+__global__ void __launch_bounds__(256) ternarise_pack_kernel(
+    const float4* __restrict__ W4, int64_t numel, const float* __restrict__ gamma_in,
+    const double* __restrict__ partials, int nparts, float eps, float* __restrict__ gamma_out,
+    uint8_t* __restrict__ packed) {
+    __shared__ float s_gamma;
+    if (threadIdx.x < 32) {
+        float g;
+        if (gamma_in != nullptr) {
+            g = *gamma_in;
+        } else {
+            double sum = 0.0;
+            for (int i = threadIdx.x; i < nparts; i += 32) sum += partials[i];
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            g = __fadd_rn(__double2float_rn(sum / static_cast<double>(numel)), eps);
+            if (blockIdx.x == 0 && threadIdx.x == 0) *gamma_out = g;
+        }
+        if (threadIdx.x == 0) s_gamma = g;
+    }
+    __syncthreads();
+    const float gamma = s_gamma;
+
+    const int64_t ngroups = numel / 16;
+    uint32_t* packed32 = reinterpret_cast<uint32_t*>(packed);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ngroups;
+         i += stride) {
+        const float4* src = W4 + 4 * i;
+        const float4 a = __ldg(src), b = __ldg(src + 1), c = __ldg(src + 2), d = __ldg(src + 3);
+        packed32[i] = pack4_codes(a, gamma) | (pack4_codes(b, gamma) << 8) |
+                      (pack4_codes(c, gamma) << 16) | (pack4_codes(d, gamma) << 24);
+    }
+    // tail: numel % 16 weights (numel is a multiple of 4), one byte per float4
+    const int64_t done4 = ngroups * 4, n4 = numel / 4;
+    for (int64_t j = done4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n4;
+         j += stride)
+        packed[j] = static_cast<uint8_t>(pack4_codes(__ldg(W4 + j), gamma));
+}
+
+// -------------------------------------------------------------- pack codes --
+__device__ __forceinline__ uint32_t encode_byte_code(uint32_t b, bool& bad) {
+    if (b == 0x01u) return 1u;
+    if (b == 0xFFu) return 2u;
+    if (b != 0u) bad = true;
+    return 0u;
+}
+
+__device__ __forceinline__ uint32_t pack_word_codes(uint32_t w, bool& bad) {
+    return encode_byte_code(w & 0xFFu, bad) | (encode_byte_code((w >> 8) & 0xFFu, bad) << 2) |
+           (encode_byte_code((w >> 16) & 0xFFu, bad) << 4) |
+           (encode_byte_code(w >> 24, bad) << 6);
+}
+
+__global__ void __launch_bounds__(256) pack_codes_kernel(const uint4* __restrict__ codes16,
+                                                         int64_t numel,
+                                                         uint8_t* __restrict__ packed,
+                                                         int32_t* __restrict__ err) {
+    bool bad = false;
+    const int64_t ngroups = numel / 16;
+    uint32_t* packed32 = reinterpret_cast<uint32_t*>(packed);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ngroups;
+         i += stride) {
+        const uint4 v = __ldg(codes16 + i);
+        packed32[i] = pack_word_codes(v.x, bad) | (pack_word_codes(v.y, bad) << 8) |
+                      (pack_word_codes(v.z, bad) << 16) | (pack_word_codes(v.w, bad) << 24);
+    }
+    const uint32_t* codes4 = reinterpret_cast<const uint32_t*>(codes16);
+    for (int64_t j = ngroups * 4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+         j < numel / 4; j += stride)
+        packed[j] = static_cast<uint8_t>(pack_word_codes(__ldg(codes4 + j), bad));
+    if (bad && err != nullptr) atomicOr(err, kErrBitBadCode);
+}
+
+// --------------------------------------------------- activation quantisation --
+// bf16 pairs -> int8: x * s rounded half to even, clipped to [-128, 127].
+__device__ __forceinline__ uint32_t quant_pair(uint32_t w, float s) {
+    const float lo = __uint_as_float(w << 16);
+    const float hi = __uint_as_float(w & 0xFFFF0000u);
+    int ql = __float2int_rn(__fmul_rn(lo, s));
+    int qh = __float2int_rn(__fmul_rn(hi, s));
+    ql = max(-128, min(127, ql));
+    qh = max(-128, min(127, qh));
+    return (static_cast<uint32_t>(ql) & 0xFFu) | ((static_cast<uint32_t>(qh) & 0xFFu) << 8);
+}
+
+__device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+    uint2 r;
+    r.x = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
+    r.y = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+    return r;
+}
+
+// |x| of two bf16 at once as unsigned 16-bit lanes; for finite values the integer
+// order of |x| bit patterns is the float order.
+__device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
+    m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    return m;
+}
+
+// One group of G threads per token row; each thread keeps up to NV 16-byte vectors of
+// its row in registers between the absmax pass and the quantise pass (longer rows are
+// re-read for the remainder).  Needs K % 8 == 0.
+template <int G>
+__global__ void __launch_bounds__(G > 256 ? G : 256)
+    act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
+                         uint2* __restrict__ xq, float* __restrict__ s_out) {
+    constexpr int CTA = G > 256 ? G : 256;
+    constexpr int RPC = CTA / G;   // rows per block
+    constexpr int WPG = G / 32;    // warps per row group
+    constexpr int NV = 8;
+    __shared__ uint32_t red[CTA / 32];
+
+    const int sub = threadIdx.x / G;
+    const int j = threadIdx.x % G;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + sub;
+    const int nvec = K / 8;
+    const bool active = row < M;
+    const uint4* xr = X + (active ? row : 0) * nvec;
+
+    uint4 v[NV];
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int idx = j + u * G;
+        if (active && idx < nvec) {
+            v[u] = __ldg(xr + idx);
+            m2 = absmax_vec(m2, v[u]);
+        } else {
+            v[u] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    for (int idx = j + NV * G; active && idx < nvec; idx += G) m2 = absmax_vec(m2, __ldg(xr + idx));
+
+    uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+    for (int off = 16; off > 0; off >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
+    if constexpr (WPG > 1) {
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+        __syncthreads();
+        am = 0;
+#pragma unroll
+        for (int w = 0; w < WPG; ++w) am = max(am, red[sub * WPG + w]);
+    }
+    const float a = __uint_as_float(am << 16);
+    const float s = __fdiv_rn(127.0f, fmaxf(a, eps));
+    if (!active) return;
+    if (j == 0) s_out[row] = s;
+    uint2* qr = xq + row * nvec;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int idx = j + u * G;
+        if (idx < nvec) qr[idx] = quant8(v[u], s);
+    }
+    for (int idx = j + NV * G; idx < nvec; idx += G) qr[idx] = quant8(__ldg(xr + idx), s);
+}
+
+// Any K: one warp per row, scalar loads.
+__global__ void __launch_bounds__(256) act_quant_scalar_kernel(const uint16_t* __restrict__ X,
+                                                              int64_t M, int64_t K, float eps,
+                                                              int8_t* __restrict__ xq,
+                                                              float* __restrict__ s_out) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const uint16_t* xr = X + row * K;
+    uint32_t am = 0;
+    for (int64_t k = lane; k < K; k += 32) am = max(am, static_cast<uint32_t>(xr[k] & 0x7FFFu));
+    for (int off = 16; off > 0; off >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
+    const float s = __fdiv_rn(127.0f, fmaxf(__uint_as_float(am << 16), eps));
+    if (lane == 0) s_out[row] = s;
+    for (int64_t k = lane; k < K; k += 32) {
+        int q = __float2int_rn(__fmul_rn(__uint_as_float(static_cast<uint32_t>(xr[k]) << 16), s));
+        xq[row * K + k] = static_cast<int8_t>(max(-128, min(127, q)));
+    }
+}
+
+int grid_for(int64_t work, int per_block, int cap) {
+    int64_t g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return static_cast<int>(g);
+}
+
+}  // namespace
+
+int absmean_num_partials(int64_t numel) {
+    const int64_t n4 = numel / 4;
+    int64_t want = (n4 + kAbsThreads * 8 - 1) / (kAbsThreads * 8);
+    if (want < 1) want = 1;
+    if (want > kAbsMaxParts) want = kAbsMaxParts;
+    return static_cast<int>(want);
+}
+
+cudaError_t launch_absmean_partials(const float* W, int64_t numel, double* partials, int nparts,
+                                    cudaStream_t stream) {
+    absmean_partials_kernel<<<nparts, kAbsThreads, 0, stream>>>(
+        reinterpret_cast<const float4*>(W), numel / 4, partials);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ternarise_pack(const float* W, int64_t numel, const float* gamma_in,
+                                  const double* partials, int nparts, float eps,
+                                  float* gamma_out, uint8_t* packed, cudaStream_t stream) {
+    const int grid = grid_for(numel / 16, 256 * 4, 148 * 16);
+    ternarise_pack_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), numel,
+                                                     gamma_in, partials, nparts, eps, gamma_out,
+                                                     packed);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packed, int32_t* err,
+                              cudaStream_t stream) {
+    const int grid = grid_for(numel / 16, 256 * 4, 148 * 16);
+    pack_codes_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(codes), numel,
+                                                packed, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
+                                float* s, cudaStream_t stream) {
+    if (K % 8 != 0 || K > (int64_t(1) << 30)) {
+        act_quant_scalar_kernel<<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X, M, K, eps, xq, s);
+        return cudaGetLastError();
+    }
+    const int nvec = static_cast<int>(K / 8);
+    const uint4* X4 = reinterpret_cast<const uint4*>(X);
+    uint2* q8 = reinterpret_cast<uint2*>(xq);
+    const int Ki = static_cast<int>(K);
+    if (nvec <= 128) {
+        act_quant_vec_kernel<32><<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    } else if (nvec <= 256) {
+        act_quant_vec_kernel<64><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    } else if (nvec <= 512) {
+        act_quant_vec_kernel<128><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    } else if (nvec <= 1024) {
+        act_quant_vec_kernel<256><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    } else {
+        act_quant_vec_kernel<512><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace bl

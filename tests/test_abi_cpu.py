@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol that ``include/bitlinear.h`` declares, reports workspace sizes, and rejects bad
+arguments before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+pytestmark = pytest.mark.cpu
+
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from ternary_weight_bit_absmean_b200 import build_lib, binding
+    build_lib.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"BL_API\s+[\w\s\*]+?\b(bitlinear_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ["bitlinear_quantize_weights", "bitlinear_quantize_weights_with_scale",
+                 "bitlinear_pack", "bitlinear_quantize_act", "bitlinear_forward",
+                 "bitlinear_workspace_size"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from ternary_weight_bit_absmean_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+    # nothing but the declared API is exported
+    assert {n for n in exported if n.startswith("bitlinear_")} == set(declared_functions())
+
+
+def test_library_has_no_driver_or_torch_dependency():
+    from ternary_weight_bit_absmean_b200 import binding
+    out = subprocess.run(["ldd", binding.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out and "libcudart" not in out
+
+
+def test_header_compiles_as_c():
+    src = '#include "bitlinear.h"\nint main(void){ return (int)bitlinear_workspace_size(1, 4) < 0; }\n'
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I",
+                    os.path.join(ROOT, "include"), "-x", "c", "-"], input=src, text=True, check=True)
+
+
+def test_workspace_size(L):
+    assert L.bitlinear_workspace_size(0, 4) == 0
+    assert L.bitlinear_workspace_size(4, 0) == 0
+    assert L.bitlinear_workspace_size(1, 4) == 8
+    sizes = [L.bitlinear_workspace_size(n, 4096) for n in (1, 64, 4096, 65536)]
+    assert sizes == sorted(sizes) and sizes[-1] <= 148 * 8 * 8
+
+
+BL_OK, INVALID, SHAPE, MISALIGNED, WORKSPACE = 0, 1, 2, 3, 4
+FAKE = 1 << 20          # 16-byte aligned, never dereferenced: every case fails validation first
+ODD = FAKE + 4
+
+
+def test_quantize_weights_validation(L):
+    f = L.bitlinear_quantize_weights
+    ws = L.bitlinear_workspace_size(8, 64)
+    assert f(None, 8, 64, 1e-5, FAKE, FAKE, FAKE, ws, None) == INVALID
+    assert f(FAKE, 0, 64, 1e-5, FAKE, FAKE, FAKE, ws, None) == INVALID
+    assert f(FAKE, 8, -4, 1e-5, FAKE, FAKE, FAKE, ws, None) == INVALID
+    assert f(FAKE, 8, 64, 0.0, FAKE, FAKE, FAKE, ws, None) == INVALID
+    assert f(FAKE, 8, 64, float("nan"), FAKE, FAKE, FAKE, ws, None) == INVALID
+    assert f(FAKE, 8, 66, 1e-5, FAKE, FAKE, FAKE, ws, None) == SHAPE
+    assert f(ODD, 8, 64, 1e-5, FAKE, FAKE, FAKE, ws, None) == MISALIGNED
+    assert f(FAKE, 8, 64, 1e-5, FAKE, ODD, FAKE, ws, None) == MISALIGNED
+    assert f(FAKE, 8, 64, 1e-5, FAKE, FAKE, None, ws, None) == WORKSPACE
+    assert f(FAKE, 8, 64, 1e-5, FAKE, FAKE, FAKE, ws - 1, None) == WORKSPACE
+
+
+def test_other_entry_points_validation(L):
+    assert L.bitlinear_quantize_weights_with_scale(FAKE, 8, 64, None, FAKE, None) == INVALID
+    assert L.bitlinear_quantize_weights_with_scale(FAKE, 8, 6, FAKE, FAKE, None) == SHAPE
+    assert L.bitlinear_pack(FAKE, 8, 10, FAKE, None, None) == SHAPE
+    assert L.bitlinear_pack(ODD, 8, 64, FAKE, None, None) == MISALIGNED
+    assert L.bitlinear_quantize_act(FAKE, 0, 64, 1e-5, FAKE, FAKE, None) == INVALID
+    assert L.bitlinear_quantize_act(FAKE, 4, 64, -1.0, FAKE, FAKE, None) == INVALID
+    assert L.bitlinear_quantize_act(FAKE, 4, 64, 1e-5, ODD, FAKE, None) == MISALIGNED
+    fwd = L.bitlinear_forward
+    assert fwd(None, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, None) == INVALID
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 4, 8, 66, FAKE, 0, None, None) == SHAPE
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 7, None, None) == INVALID
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 4, 8, 1 << 25, FAKE, 0, None, None) == SHAPE
+    assert fwd(FAKE, ODD, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, None) == MISALIGNED
+    path = L.bitlinear_forward_path
+    assert path(FAKE, FAKE, FAKE, FAKE, 40, 8, 96, FAKE, 0, None, 2, None) == SHAPE  # tcgen05 needs K % 64
+    assert path(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 9, None) == INVALID
+    assert L.bitlinear_status_string(3) == b"BL_ERR_MISALIGNED"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from ternary_weight_bit_absmean_b200 import binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.lib()

@@ -1,0 +1,301 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded
+inputs.  Integer and byte results (packed codes, x_q, int32 accumulators) must be
+bit-exact; gamma within 1e-6 relative; float outputs within 1e-5 relative / 1e-6
+absolute; bf16 outputs equal the oracle's except next to a rounding midpoint."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (EPS, assert_bf16_match, assert_float_close, bits, check_guard,
+                      guarded_empty)
+from ternary_weight_bit_absmean_b200 import binding as B
+from ternary_weight_bit_absmean_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from ternary_weight_bit_absmean_b200 import build_lib
+    build_lib.build()
+    B.lib()
+
+
+def sync():
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------- activations (a4) --
+
+ACT_SHAPES = [(1, 1), (3, 7), (5, 100), (2, 4), (17, 8), (8192, 256), (4096, 1536), (512, 4096),
+              (64, 3200), (16, 8640), (8, 8192), (3, 28672), (33, 1032), (7, 36000)]
+
+
+@pytest.mark.parametrize("M,K", ACT_SHAPES)
+def test_quantize_act_bit_exact(M, K):
+    X = synth.activations(M, K, seed=M * 7 + K, outlier_frac=0.01, outlier_scale=20.0)
+    if M > 2:
+        X[1] = 0  # an all-zero token
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    Xd = X.to(DEV)
+    xq = guarded_empty((M, K), torch.int8)
+    s = guarded_empty((M,), torch.float32)
+    B.bitlinear_quantize_act(Xd, EPS, xq, s)
+    sync()
+    check_guard(xq)
+    check_guard(s)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+
+
+def test_quantize_act_tiny_rows_use_eps():
+    X = torch.full((4, 64), 1e-7, dtype=torch.float32).to(torch.bfloat16)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    xq, s = B.quantize_act(X.to(DEV), EPS)
+    sync()
+    assert np.array_equal(s.cpu().numpy(), s_ref) and np.array_equal(xq.cpu().numpy(), xq_ref)
+
+
+# ------------------------------------------------------- weights (a1, a2, a3) --
+
+W_SHAPES = [(1, 4), (3, 12), (7, 20), (512, 256), (1536, 1536), (4096, 1536), (1536, 4096),
+            (3200, 3200), (8640, 3200), (1024, 8192), (33, 1000)]
+
+
+@pytest.mark.parametrize("N,K", W_SHAPES)
+def test_quantize_weights(N, K):
+    W = synth.weight(N, K, seed=N + 3 * K)
+    g_ref, codes_ref, packed_ref = oracle.quantize_weights(W.numpy(), EPS)
+    Wd = W.to(DEV)
+    gamma = torch.empty(1, dtype=torch.float32, device=DEV)
+    packed = guarded_empty((N, K // 4), torch.uint8)
+    ws = torch.empty(B.bitlinear_workspace_size(N, K), dtype=torch.uint8, device=DEV)
+    B.bitlinear_quantize_weights(Wd, EPS, gamma, packed, ws)
+    sync()
+    check_guard(packed)
+    g = np.float32(gamma.item())
+    assert abs(float(g) - float(g_ref)) <= 1e-6 * float(g_ref)
+    # codes are compared with the oracle's gamma through the given-scale entry
+    g_dev = torch.tensor([g_ref], dtype=torch.float32, device=DEV)
+    packed2 = guarded_empty((N, K // 4), torch.uint8)
+    B.bitlinear_quantize_weights_with_scale(Wd, g_dev, packed2)
+    sync()
+    check_guard(packed2)
+    assert np.array_equal(packed2.cpu().numpy(), packed_ref)
+    if g == g_ref:
+        assert np.array_equal(packed.cpu().numpy(), packed_ref)
+    # gamma is reproducible from run to run
+    gamma2 = torch.empty(1, dtype=torch.float32, device=DEV)
+    B.bitlinear_quantize_weights(Wd, EPS, gamma2, packed, ws)
+    sync()
+    assert gamma2.item() == gamma.item()
+
+
+def test_quantize_weights_given_scale_ties_and_zero_share():
+    # weights on the +-gamma/2 rounding boundary and beyond the clip
+    gamma = np.float32(0.0625)
+    row = np.array([0.03125, -0.03125, 0.09375, -0.09375, 0.5, -0.5, 0.0, 0.0312500037] * 2, np.float32)
+    W = torch.from_numpy(np.tile(row, (3, 1)))
+    want, _ = oracle.pack(oracle.ternarise(W.numpy(), gamma))
+    packed = torch.empty(3, 4, dtype=torch.uint8, device=DEV)
+    B.bitlinear_quantize_weights_with_scale(W.to(DEV), torch.tensor([gamma], device=DEV), packed)
+    sync()
+    assert np.array_equal(packed.cpu().numpy(), want)
+    # zero-code share of the 50% / 70% mixtures (reported by the oracle) is reproduced
+    for frac in (0.378, 0.664):
+        Wm = synth.weight(256, 1024, seed=5, small_frac=frac)
+        g_ref, codes, packed_ref = oracle.quantize_weights(Wm.numpy(), EPS)
+        g_dev, p_dev = B.quantize_weights(Wm.to(DEV), EPS)
+        sync()
+        pk = oracle.unpack(p_dev.cpu().numpy(), 1024)
+        assert abs(float(np.mean(pk == 0)) - float(np.mean(codes == 0))) < 1e-3
+
+
+def test_zero_weights():
+    W = torch.zeros(64, 256, device=DEV)
+    gamma, packed = B.quantize_weights(W, EPS)
+    sync()
+    assert gamma.item() == np.float32(EPS) and not packed.any().item()
+
+
+@pytest.mark.parametrize("N,K", [(1, 4), (5, 12), (64, 256), (1536, 4096), (7, 100)])
+def test_pack_codes(N, K):
+    c = synth.codes(N, K, seed=N * K)
+    want, bad = oracle.pack(c.numpy())
+    assert bad == 0
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    packed = guarded_empty((N, K // 4), torch.uint8)
+    B.bitlinear_pack(c.to(DEV), packed, err)
+    sync()
+    check_guard(packed)
+    assert err.item() == 0
+    assert np.array_equal(packed.cpu().numpy(), want)
+
+
+def test_pack_reports_bad_codes():
+    c = synth.codes(16, 64, seed=3)
+    c[3, 5] = 2
+    c[9, 63] = -100
+    want, bad = oracle.pack(c.numpy())
+    assert bad == 2
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    packed = torch.empty(16, 16, dtype=torch.uint8, device=DEV)
+    B.bitlinear_pack(c.to(DEV), packed, err)
+    sync()
+    assert err.item() & B.BL_ERRBIT_BAD_CODE
+    assert np.array_equal(packed.cpu().numpy(), want)
+
+
+# ------------------------------------------------------------ forward (a5-a7) --
+
+def make_problem(M, N, K, seed, zero_row=False):
+    W = synth.weight(N, K, seed=seed)
+    X = synth.activations(M, K, seed=seed, outlier_frac=0.01, outlier_scale=20.0)
+    if zero_row and M > 1:
+        X[M // 2] = 0
+    g_ref, _, packed_ref = oracle.quantize_weights(W.numpy(), EPS)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    return g_ref, packed_ref, xq_ref, s_ref
+
+
+def run_forward(xq_ref, s_ref, packed_ref, g_ref, out_dtype, path):
+    M, K = xq_ref.shape
+    N = packed_ref.shape[0]
+    xq = torch.from_numpy(xq_ref).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], dtype=torch.float32, device=DEV)
+    out = guarded_empty((M, N), out_dtype)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.bitlinear_forward(xq, s, packed, gamma, out, err, path=path)
+    sync()
+    check_guard(out)
+    assert err.item() == 0
+    return out
+
+
+def check_forward(M, N, K, path, seed=0, rows=None, zero_row=True):
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed, zero_row)
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    acc_ref = oracle.forward(xq_ref[sel], s_ref[sel], packed_ref, g_ref, K, oracle.OUT_I32)
+    y_ref = oracle.dequant(acc_ref, s_ref[sel], g_ref)
+    yb_ref = oracle.f32_to_bf16(y_ref)
+    acc = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, path).cpu().numpy()
+    assert np.array_equal(acc[sel], acc_ref), "int32 accumulators differ"
+    y = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.float32, path).cpu().numpy()
+    assert_float_close(y[sel], y_ref, "fp32 y")
+    yb = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.bfloat16, path)
+    yb = yb.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert_bf16_match(yb[sel], y_ref, yb_ref, "bf16 y")
+    if rows is not None:
+        # every row: the integer accumulators are linear in x_q, so the product of the
+        # accumulator matrix with a random vector equals x_q times (codes^T times it)
+        codes = oracle.unpack(packed_ref, K).astype(np.int64)
+        v = np.random.default_rng(seed).integers(-3, 4, size=N).astype(np.int64)
+        assert np.array_equal(acc.astype(np.int64) @ v, xq_ref.astype(np.int64) @ (codes.T @ v))
+
+
+GEMV_CASES = [(1, 1, 64), (1, 256, 64), (2, 300, 192), (3, 512, 256), (8, 1536, 1536),
+              (9, 100, 320), (16, 4096, 1536), (16, 3200, 8640), (5, 1024, 8192), (1, 8192, 8192),
+              (13, 8640, 3200), (16, 1000, 4160), (40, 200, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMV_CASES)
+def test_forward_gemv(M, N, K):
+    check_forward(M, N, K, B.BL_PATH_GEMV, seed=M + N + K)
+
+
+TC_CASES = [(17, 128, 128), (32, 256, 256), (64, 512, 256), (100, 300, 192), (256, 128, 1536),
+            (300, 200, 320), (512, 1536, 1536), (513, 4096, 1536), (1000, 1536, 4096),
+            (8192, 512, 256), (130, 640, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", TC_CASES)
+def test_forward_tc(M, N, K):
+    check_forward(M, N, K, B.BL_PATH_TC, seed=M * 3 + N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 64, 100), (3, 33, 4), (20, 17, 36), (5, 7, 1000)])
+def test_forward_generic_k(M, N, K):
+    """K % 64 != 0 runs the plain kernel through the automatic dispatch."""
+    check_forward(M, N, K, B.BL_PATH_AUTO, seed=M + 2 * N + K)
+
+
+def test_forward_paths_agree_and_are_deterministic():
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(48, 768, 2048, 11)
+    a = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_GEMV)
+    b = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_TC)
+    c = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_TC)
+    assert torch.equal(a, b) and torch.equal(b, c)
+
+
+def test_forward_zero_weights_give_zero():
+    M, N, K = 300, 256, 512
+    xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=DEV)
+    s = torch.ones(M, device=DEV)
+    packed = torch.zeros(N, K // 4, dtype=torch.uint8, device=DEV)
+    gamma = torch.tensor([EPS], device=DEV)
+    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC):
+        y = B.forward(xq, s, packed, gamma, torch.float32, path=path)
+        sync()
+        assert not y.any().item()
+
+
+def test_forward_extreme_accumulators():
+    """All codes +1 against x_q = -128 or +127 everywhere: |acc| reaches 128 K."""
+    M, N, K = 64, 256, 8192
+    xq = torch.full((M, K), 127, dtype=torch.int8, device=DEV)
+    xq[::2] = -128
+    packed = torch.full((N, K // 4), 0x55, dtype=torch.uint8, device=DEV)  # all +1
+    packed[::3] = 0xAA                                                     # all -1
+    s = torch.ones(M, device=DEV)
+    gamma = torch.tensor([1.0], device=DEV)
+    want = (xq.long().sum(1)[:, None] * torch.where(torch.arange(N, device=DEV) % 3 == 0, -1, 1)[None, :])
+    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC):
+        acc = B.forward(xq, s, packed, gamma, torch.int32, path=path)
+        sync()
+        assert torch.equal(acc.long(), want)
+
+
+# -------------------------------------------------- the workloads' own sizes --
+
+@pytest.mark.parametrize("name", ["toy", "llama700m", "llama3b", "llama70b"])
+def test_workload_sizes(name):
+    """Every projection of each workload at its decode and prefill token counts, in the
+    configuration the benchmark times (automatic dispatch); large problems are checked
+    on sampled token rows plus the linearity property over all rows."""
+    spec = synth.WORKLOADS[name]
+    projs = spec["proj"]
+    if name == "llama70b":
+        projs = [p for p in projs if p[0] in ("k", "up", "down")]
+    for pi, (pname, N, K) in enumerate(projs):
+        W = synth.weight(N, K, seed=pi)
+        g_ref, _, packed_ref = oracle.quantize_weights(W.numpy(), EPS)
+        g_dev, p_dev = B.quantize_weights(W.to(DEV), EPS)
+        sync()
+        assert abs(g_dev.item() - float(g_ref)) <= 1e-6 * float(g_ref)
+        if g_dev.item() == float(g_ref):
+            assert np.array_equal(p_dev.cpu().numpy(), packed_ref)
+        Ms = spec["M"] if name != "llama70b" else [1, 16, 64]
+        for M in Ms:
+            X = synth.activations(M, K, seed=pi + 100 * M, outlier_frac=spec["outlier_frac"])
+            xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+            xq, s = B.quantize_act(X.to(DEV), EPS)
+            sync()
+            assert np.array_equal(xq.cpu().numpy(), xq_ref) and np.array_equal(s.cpu().numpy(), s_ref)
+            rows = np.arange(M) if M * N * K <= 4e9 else np.unique(
+                np.r_[0, M - 1, np.random.default_rng(M).integers(0, M, 6)])
+            acc_ref = oracle.forward(xq_ref[rows], s_ref[rows], packed_ref, g_ref, K, oracle.OUT_I32)
+            y_ref = oracle.dequant(acc_ref, s_ref[rows], g_ref)
+            gamma = torch.tensor([g_ref], device=DEV)
+            pk = torch.from_numpy(packed_ref).to(DEV)
+            acc = B.forward(xq, s, pk, gamma, torch.int32).cpu().numpy()
+            y = B.forward(xq, s, pk, gamma, torch.float32).cpu().numpy()
+            assert np.array_equal(acc[rows], acc_ref), (name, pname, M)
+            assert_float_close(y[rows], y_ref, "%s %s M=%d" % (name, pname, M))
