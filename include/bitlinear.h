@@ -155,6 +155,28 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
                                  bl_dtype out_dtype, int32_t *err_word, bl_path path,
                                  void *stream);
 
+/* bitlinear_quantize_weights for callers that cannot allocate device memory.  The
+ * source pages have no counterpart to this entry point; it exists for the library's
+ * users.  Callers such as a serving loop that must not call cudaMalloc (which can
+ * synchronise the whole device), a plug-in whose host framework owns all device
+ * memory, or a deployment with a device memory budget fixed at start-up have no
+ * workspace to pass.  This variant keeps the fp64 partial sums of |W| in a fixed
+ * array inside the library instead:
+ *   - The array holds 1184 doubles (9472 bytes).  Every GPU that loads the library
+ *     keeps it until the process exits.  Every shape accepted by
+ *     bitlinear_quantize_weights fits; a shape that would need more partial sums
+ *     than the array holds returns BL_ERR_WORKSPACE.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current) and caches it.  Make that first call before any stream capture.
+ *   - Nothing is allocated or freed, by this library or by any library it calls.
+ *   - All calls share the one array.  Calls that run at the same time on the GPU
+ *     (for example on two streams) race and corrupt each other's gamma.  Serialise
+ *     them.  A call never reads what an earlier call left in the array.
+ * Arguments, results and the other errors are those of bitlinear_quantize_weights. */
+BL_API bl_status bitlinear_quantize_weights_noalloc(const float *W, int64_t N, int64_t K, float eps,
+                                                    float *gamma_out, uint8_t *packed_out,
+                                                    void *stream);
+
 /* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
 BL_API int bitlinear_last_cuda_error(void);
 

@@ -35,6 +35,10 @@ bl_status check_weight_shape(int64_t N, int64_t K) {
 
 }  // namespace
 
+namespace bl {
+void record_cuda_error(int code) { g_last_cuda_error = code; }
+}  // namespace bl
+
 extern "C" {
 
 size_t bitlinear_workspace_size(int64_t N, int64_t K) {

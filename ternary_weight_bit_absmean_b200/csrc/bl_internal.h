@@ -40,4 +40,7 @@ cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* pack
                            const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                            int kind, int32_t* err, cudaStream_t stream);
 
+// Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
+void record_cuda_error(int code);
+
 }  // namespace bl
