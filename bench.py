@@ -48,6 +48,14 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ref-tokens", type=int, default=4,
                    help="token rows per M in one reference-arm (oracle) step")
+    p.add_argument("--single", choices=["forward", "quantize_act", "quantize_weights", "pack"],
+                   help="time one entry point on one shape instead of the step (kernel study, ncu)")
+    p.add_argument("--M", type=int, default=4096)
+    p.add_argument("--N", type=int, default=4096)
+    p.add_argument("--K", type=int, default=4096)
+    p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2"], default="auto")
+    p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
+    p.add_argument("--iters", type=int, default=20)
     return p.parse_args()
 
 
@@ -262,7 +270,7 @@ def run_ours(args):
 
     ops_step = fwd_ops(projs, Ms)
     value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
-    e2e_value = ops_step * len(e2e_ms) * world / (e2e_total * 1e-3) / 1e12
+    e2e_value = ops_step * len(e2e_ms) * world / (e2e_total * 1e-3) / 1e12 if e2e_ms else None
 
     # ---- per-row breakdown and the dominant kernel's roofline
     pk_bytes = {pi: N * K // 4 for pi, (_, N, K) in enumerate(projs)}
@@ -311,8 +319,8 @@ def run_ours(args):
                    "timing": "CUDA graph replay, device events, sum over steps, max over ranks",
                    "parallelism": "dp%d (independent token batches per GPU, replicated weights)" % world},
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": round(e2e_value, 4), "unit": "TOPS", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "e2e": {"value": round(e2e_value, 4) if e2e_value is not None else None, "unit": "TOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roofline,
         "breakdown_us_per_step": {k: round(v * 1e3, 2) for k, v in sorted(by.items())},
         "forward_by_M": fwd,
@@ -393,9 +401,82 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_single(args):
+    """Time one entry point on one shape: CUDA events around each call, L2 flushed in
+    between (outside the events); prints one JSON line with the mean time and the
+    achieved rate against its roofline."""
+    import torch
+
+    from ternary_weight_bit_absmean_b200 import binding as B
+    from ternary_weight_bit_absmean_b200 import build_lib, synth
+
+    build_lib.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M, N, K = args.M, args.N, args.K
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    P = peaks()
+    if args.single == "forward":
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        s = torch.rand(M, device=dev) + 1.0
+        c = synth.codes(N, K, seed=1).to(dev)
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+        B.bitlinear_pack(c, packed)
+        del c
+        gamma = torch.tensor([0.02], device=dev)
+        odt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[args.out_dtype]
+        out = torch.empty(M, N, dtype=odt, device=dev)
+        path = {"auto": B.BL_PATH_AUTO, "gemv": B.BL_PATH_GEMV, "tc": B.BL_PATH_TC, "tc1": B.BL_PATH_TC_1SM,
+                "tc2": B.BL_PATH_TC_2SM}[args.path]
+        fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path)
+        ops = 2 * M * N * K
+        nbytes = N * K // 4 + M * K + 4 * M + M * N * out.element_size()
+    elif args.single == "quantize_act":
+        X = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        s = torch.empty(M, device=dev)
+        fn = lambda: B.bitlinear_quantize_act(X, EPS, xq, s)
+        ops, nbytes = 0, 3 * M * K + 4 * M
+    elif args.single == "quantize_weights":
+        W = torch.randn(N, K, device=dev) * 0.02
+        gamma = torch.empty(1, device=dev)
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+        ws = torch.empty(B.bitlinear_workspace_size(N, K), dtype=torch.uint8, device=dev)
+        fn = lambda: B.bitlinear_quantize_weights(W, EPS, gamma, packed, ws)
+        ops, nbytes = 0, 8 * N * K + N * K // 4
+    else:
+        c = synth.codes(N, K, seed=1).to(dev)
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+        fn = lambda: B.bitlinear_pack(c, packed)
+        ops, nbytes = 0, N * K + N * K // 4
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(args.iters):
+        flush.fill_(1)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    t = statistics.median(ts) * 1e-3
+    rec = {"single": args.single, "M": M, "N": N, "K": K, "path": args.path, "out_dtype": args.out_dtype,
+           "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
+           "gbs": round(nbytes / t / 1e9, 1), "hbm_frac": round(nbytes / t / 1e9 / P["hbm_gbs"], 4),
+           "weight_gbs": round((N * K // 4) / t / 1e9, 1) if args.single == "forward" else None}
+    if ops:
+        rec["tops"] = round(ops / t / 1e12, 2)
+        rec["int8_frac"] = round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4)
+    print(json.dumps(rec), flush=True)
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.single:
+        run_single(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

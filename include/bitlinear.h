@@ -78,9 +78,11 @@ typedef enum {
 } bl_dtype;
 
 typedef enum {
-    BL_PATH_AUTO = 0, /* GEMV for M <= 16 (or shapes the tensor-core path cannot tile), else tcgen05 */
-    BL_PATH_GEMV = 1, /* register-unpack GEMV, any M (token tiles of 16) */
-    BL_PATH_TC = 2    /* tcgen05 kind::i8 tiled path; needs K % 64 == 0 */
+    BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core path cannot tile), else tcgen05 */
+    BL_PATH_GEMV = 1,   /* register-unpack GEMV, any M (token tiles of 16) */
+    BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
+    BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
+    BL_PATH_TC_2SM = 4  /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
 } bl_path;
 
 /* Bytes of device workspace bitlinear_quantize_weights needs for an [N, K] matrix

@@ -105,19 +105,26 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
     if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32)
         return BL_ERR_INVALID_ARG;
-    if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC) return BL_ERR_INVALID_ARG;
+    if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
+        path != BL_PATH_TC_2SM)
+        return BL_ERR_INVALID_ARG;
     if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
     // |acc| <= 128 K must fit in int32; sizes must fit the kernels' 32-bit indexing.
     if (K > (int64_t(1) << 31) / 128 - 1) return BL_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(xq) || !aligned16(s) || !aligned16(packed) || !aligned16(out)) return BL_ERR_MISALIGNED;
     const bool k64 = (K % 64) == 0;
-    if (path == BL_PATH_TC && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
+    const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM;
+    if (tc && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
     if (path == BL_PATH_AUTO) path = (M <= 16 || !k64) ? BL_PATH_GEMV : BL_PATH_TC;
     const int kind = static_cast<int>(out_dtype);
     cudaError_t e;
     if (path == BL_PATH_TC) {
         e = bl::launch_gemm_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+    } else if (path == BL_PATH_TC_1SM) {
+        e = bl::launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+    } else if (path == BL_PATH_TC_2SM) {
+        e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
     } else if (k64 && M <= int64_t(65535) * 16) {
         e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, as_stream(stream));
     } else {

@@ -59,6 +59,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the warp (up to `hint_ns`) until the phase
+// completes, instead of spinning and taking issue slots from the working warps.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 200000;  // 0.2 ms per suspended try_wait
+
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up after
 // kWaitTimeoutNs, or as soon as another role of the CTA has raised *abort; returns
 // false then (and raises *abort itself on a timeout).
@@ -66,14 +82,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                *abort = 1;
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            *abort = 1;
+            return false;
         }
     }
 }
@@ -186,6 +200,91 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// ----------------------------------------------------- CTA pairs (cta_group::2) --
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address, in the shared::cluster window, of the variable at CTA-local shared address
+// `addr` in the CTA of the cluster with rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier that may live in another CTA of the cluster (default
+// semantics: release at CTA scope; a cluster-scope release costs a full fence).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity);
+}
+
+// As mbar_wait_bounded, for barriers that also receive arrivals from the peer CTA.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity,
+                                                          volatile int* abort) {
+    return mbar_wait_bounded(bar, parity, abort);
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// 2-D tiled TMA load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A * B^T over a CTA pair: A's rows and B's rows are split
+// between the two CTAs' shared memory at the same offsets.  Issued by one thread of the
+// even CTA.
+__device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier at shared offset `bar` in every CTA of `cta_mask` when all
+// pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair_multicast(uint32_t bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"(cta_mask)
+        : "memory");
+}
+
 // ------------------------------------------------------------ legacy mma.sync --
 
 // D = A(16x32, row) * B(32x8, col) + C, int8 inputs, int32 accumulate (warp-wide).
@@ -243,6 +342,21 @@ __device__ __forceinline__ void unpack16_evenodd(uint32_t p, uint32_t& e0, uint3
     e1 = __byte_perm(kCodeTable, 0u, sa >> 16);
     o0 = __byte_perm(kCodeTable, 0u, sb);
     o1 = __byte_perm(kCodeTable, 0u, sb >> 16);
+}
+
+// unpack16_evenodd with its three right shifts done as high-half multiplies by
+// 2^(32 - shift), which run on the FMA pipe instead of the integer ALU pipe.  The
+// multipliers come in as runtime values (mul2 = 2^30, mul16 = 2^16) so that they stay
+// multiplies.
+__device__ __forceinline__ void unpack16_evenodd_fma(uint32_t p, uint32_t mul2, uint32_t mul16,
+                                                     uint32_t& e0, uint32_t& e1, uint32_t& o0,
+                                                     uint32_t& o1) {
+    const uint32_t sa = p & 0x33333333u;
+    const uint32_t sb = __umulhi(p, mul2) & 0x33333333u;
+    e0 = __byte_perm(kCodeTable, 0u, sa);
+    e1 = __byte_perm(kCodeTable, 0u, __umulhi(sa, mul16));
+    o0 = __byte_perm(kCodeTable, 0u, sb);
+    o1 = __byte_perm(kCodeTable, 0u, __umulhi(sb, mul16));
 }
 
 // The matching permutation of 16 activation bytes (v = bytes 0..15 little-endian):

@@ -35,10 +35,17 @@ cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t*
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                                 int kind, cudaStream_t stream);
 
-// Tiled tcgen05 kind::i8 path (K % 64 == 0).
+// Tiled tcgen05 kind::i8 paths (K % 64 == 0): launch_gemm_tc picks between the
+// single-SM kernel (tc1) and the CTA-pair kernel (tc2).
 cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed,
                            const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                            int kind, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* packed,
+                            const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
+                            int kind, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed,
+                            const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
+                            int kind, int32_t* err, cudaStream_t stream);
 
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);

@@ -15,12 +15,15 @@
 // tokens.  Per stage:
 //   warp 0 (one lane)  TMA: x_q tile [BT x 128 B] (128-byte swizzle) and the packed
 //                      weight tile [128 x 32 B] into shared memory, one mbarrier;
-//   warps 2-5          expanders: thread e unpacks packed row e (128 codes) into int8 and
-//                      writes it in the same 128-byte-swizzled K-major layout;
+//   warps 2-9          expanders: two threads per packed row, each unpacking 64 codes
+//                      into int8 and writing them in the same 128-byte-swizzled K-major
+//                      layout (two expander warps per SM sub-partition keep the
+//                      unpack off the critical path of a stage);
 //   warp 1 (one lane)  MMA issuer: four tcgen05.mma (K = 32 each) per stage into a TMEM
 //                      accumulator, tcgen05.commit frees the stage;
-//   warps 6-9          epilogue: tcgen05.ld of the finished accumulator (one feature row
-//                      per thread), y = acc * (gamma / s_m), coalesced stores along N.
+//   warps 10-17        epilogue: tcgen05.ld of the finished accumulator (one feature row
+//                      per thread, two warps per lane quarter taking alternate 32-column
+//                      chunks), y = acc * (gamma / s_m), coalesced stores along N.
 // Two TMEM accumulators let the epilogue of one tile overlap the main loop of the next
 // (persistent blocks, one per SM, static round-robin over tiles).  Ragged M, N and K
 // edges come from TMA zero fill: a zero packed byte is four zero codes.
@@ -42,8 +45,10 @@ namespace {
 
 constexpr int kBN = 128;          // output features per tile (MMA M)
 constexpr int kBK = 128;          // K bytes per stage (one 128-byte swizzle row)
-constexpr int kThreads = 320;     // 10 warps
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2, kWarpEpi = 6;
+constexpr int kThreads = 576;     // 18 warps
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2, kWarpEpi = 10;
+constexpr int kExpWarps = kWarpEpi - kWarpExp;
+constexpr int kEpiWarps = 8;      // two per TMEM lane quarter, alternating 32-column chunks
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
 
 template <int BT>
@@ -121,12 +126,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(afull(s), 4);
+            mbar_init(afull(s), kExpWarps);
             mbar_init(empty(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
-            mbar_init(tempty(b), 4);
+            mbar_init(tempty(b), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -227,8 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kWarpEpi) {
         // ------------------------------------------------------------- expanders --
-        const int e = threadIdx.x - 32 * kWarpExp;  // weight row within the tile, 0..127
-        const uint32_t sw = static_cast<uint32_t>(e & 7);
+        // Thread e owns half `half` (64 codes = 16 packed bytes) of weight row `row`;
+        // neighbouring lanes read neighbouring 16-byte pieces, so both the packed reads
+        // and the swizzled writes are free of bank conflicts.
+        const int e = threadIdx.x - 32 * kWarpExp;  // 0 .. 32 * kExpWarps - 1
+        const int row = e >> 1, half = e & 1;
+        const uint32_t sw = static_cast<uint32_t>(row & 7);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -238,16 +247,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const uint8_t* pp = gbase + (sP - base) + stage * C::kPBytes + e * (kBK / 4);
+                const uint8_t* pp = gbase + (sP - base) + stage * C::kPBytes + row * (kBK / 4) + half * 16;
                 const uint4 p0 = *reinterpret_cast<const uint4*>(pp);
-                const uint4 p1 = *reinterpret_cast<const uint4*>(pp + 16);
-                uint8_t* ap = gbase + (sA - base) + stage * C::kABytes + e * kBK;
-                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                uint8_t* ap = gbase + (sA - base) + stage * C::kABytes + row * kBK;
+                const uint32_t words[4] = {p0.x, p0.y, p0.z, p0.w};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     uint4 u;
                     unpack16_natural(words[c], u.x, u.y, u.z, u.w);
-                    *reinterpret_cast<uint4*>(ap + ((static_cast<uint32_t>(c) ^ sw) << 4)) = u;
+                    const uint32_t chunk = static_cast<uint32_t>(4 * half + c);
+                    *reinterpret_cast<uint4*>(ap + ((chunk ^ sw) << 4)) = u;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -260,32 +269,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue --
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;                   // TMEM lane quarter this warp may access
+        const int first = 32 * ((warp - kWarpEpi) >> 2);  // this warp's first column chunk
         const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
             const int n0 = (tile % a.n_tiles_n) * kBN;
             const int t0 = (tile / a.n_tiles_n) * BT;
+            // s of the first chunk's tokens is fetched before the accumulator is ready;
+            // each chunk then fetches the next chunk's while it converts and stores
+            float s_next = (a.kind != kOutI32 && t0 + first + lane < a.M) ? __ldg(a.s + t0 + first + lane) : 1.0f;
             if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag)) break;
             tc_fence_after();
             const int row = n0 + 32 * q + lane;
+            const bool row_ok = row < a.N;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BT; c0 += 32) {
+            for (int c0 = first; c0 < BT; c0 += 64) {
+                const float fac = __fdiv_rn(gamma, s_next);
+                const int tk = t0 + c0 + 64 + lane;
+                if (c0 + 64 < BT) s_next = (a.kind != kOutI32 && tk < a.M) ? __ldg(a.s + tk) : 1.0f;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
                                        static_cast<uint32_t>(buf * BT + c0),
                                    r);
                 tmem_ld_wait();
-                const int tk = t0 + c0 + lane;
-                const float fac = (a.kind != kOutI32 && tk < a.M) ? __fdiv_rn(gamma, a.s[tk]) : 0.0f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float fj = __shfl_sync(0xffffffffu, fac, j);
                     const int tok = t0 + c0 + j;
-                    if (tok < a.M && row < a.N)
-                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
-                                static_cast<int>(r[j]), fj);
+                    if (tok < a.M && row_ok)
+                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row, static_cast<int>(r[j]), fj);
                 }
             }
             tc_fence_before();
@@ -320,8 +334,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-bool encode_2d_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                  uint32_t box_outer, CUtensorMapSwizzle swz) {
+}  // namespace
+
+// 2-D uint8 tensor map over a row-major [outer, inner] byte matrix with a
+// [box_outer, box_inner] box; 128-byte swizzle or none.
+bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer, bool swizzle128) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t dims[2] = {inner, outer};
@@ -329,18 +347,19 @@ bool encode_2d_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t ou
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <int BT>
 cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms, cudaStream_t stream) {
     using C = TcCfg<BT>;
     CUtensorMap tx, tp;
-    if (!encode_2d_u8(&tx, xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, BT,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d_u8(&tp, packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4,
-                      kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), kBK, BT, true) ||
+        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4, kBN,
+                           false))
         return cudaErrorInvalidValue;
     static bool attr_done[64] = {};
     int dev = 0;
@@ -358,30 +377,35 @@ cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms
 
 }  // namespace
 
-cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                           int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
-                           cudaStream_t stream) {
+// Token tile of the single-SM kernel and its cost (cycles of the busiest SM, up to a
+// constant): a 128-byte K stage costs ~2 BT cycles of MMA at peak but never less than a
+// fixed pipeline floor (TMA + expansion latency spread over the stages in flight).
+static int tc1_tile(int64_t M, int64_t N, int sms, int64_t* cost) {
+    const int64_t nN = (N + kBN - 1) / kBN;
+    const int64_t nK = 1;
+    auto c = [&](int b) {
+        const int64_t tiles = nN * ((M + b - 1) / b);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        const int64_t per_stage = 2 * b > 400 ? 2 * b : 400;
+        return waves * per_stage * nK;
+    };
+    int bt = 256;
+    if (M <= 32) bt = 32;
+    else if (M <= 64) bt = 64;
+    else bt = c(128) < c(256) ? 128 : 256;
+    *cost = c(bt);
+    return bt;
+}
+
+cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                            cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t nN = (N + kBN - 1) / kBN;
-    // Token tile: per K step an MMA of 128 x BT costs ~BT/2 cycles at peak while the
-    // expansion of 128 x 32 codes costs a fixed ~64; pick the tile with the fewest
-    // waves x cycles per tile.
-    int bt = 256;
-    if (M <= 32) {
-        bt = 32;
-    } else if (M <= 64) {
-        bt = 64;
-    } else {
-        auto cost = [&](int b) {
-            const int64_t tiles = nN * ((M + b - 1) / b);
-            const int64_t waves = (tiles + sms - 1) / sms;
-            const int64_t per = (b / 2 > 64 ? b / 2 : 64) + 16;
-            return waves * per;
-        };
-        bt = cost(128) < cost(256) ? 128 : 256;
-    }
+    int64_t cost = 0;
+    const int bt = tc1_tile(M, N, sms, &cost);
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
              0, out, kind, err};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
@@ -391,6 +415,25 @@ cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* pack
         case 128: return launch_bt<128>(xq, packed, a, sms, stream);
         default: return launch_bt<256>(xq, packed, a, sms, stream);
     }
+}
+
+// The pair kernel moves half the activation bytes per SM and stores 16-byte vectors;
+// it is preferred unless its coarser 256 x 256 tiles leave more waves than the
+// single-SM kernel's.
+cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                           int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                           cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t cost1 = 0;
+    tc1_tile(M, N, sms, &cost1);
+    const int64_t tiles2 = ((N + 255) / 256) * ((M + 255) / 256);
+    const int64_t pairs = sms / 2;
+    const int64_t cost2 = (tiles2 + pairs - 1) / pairs * 512;
+    if (M > 128 && cost2 <= cost1)
+        return launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
+    return launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
 }
 
 }  // namespace bl

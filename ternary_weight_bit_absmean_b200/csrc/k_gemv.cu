@@ -50,6 +50,7 @@ struct GemvArgs {
     int xs_bytes;  // shared bytes reserved for staged activations (the reduction buffer follows)
     void* out;
     int kind;
+    uint32_t mul2, mul16;  // 2^30 and 2^16: right shifts by 2 and 16 as high-half multiplies
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -64,8 +65,130 @@ __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int ac
         static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(y);
 }
 
+// One K step of 16 codes per row for the thread's four rows (word w_r of each row):
+// the even/odd unpack of the four words (masks on the ALU pipe, shifts as high-half
+// multiplies on the FMA pipe, one prmt table lookup per output register) feeding the
+// warp MMAs of both 16-row tiles directly, written as one block so that the unpacked
+// registers are the MMA operands.  acc0/acc1: tiles 0/1 against token tile 0 (B = b0..b3);
+// with MT == 2 also acc2/acc3 against token tile 1 (B = c0..c3).
+// One K step of 16 codes per row for the thread's four rows (word w_r of each row):
+// the even/odd unpack of the four words (masks on the ALU pipe, shifts as high-half
+// multiplies on the FMA pipe, one prmt table lookup per output register) feeding the
+// warp MMAs of both 16-row tiles directly, written as one block so that the unpacked
+// registers are the MMA operands.  acc[0]/acc[1]: the two 16-row tiles; token tile 0
+// uses B = b, token tile 1 (MT == 2) uses B = bb.
 template <int MT>
-__global__ void __launch_bounds__(kGvThreads) gemv_kernel(GemvArgs a) {
+__device__ __forceinline__ void gemv_step(int (&acc)[2][MT][4], uint32_t w0, uint32_t w1, uint32_t w2,
+                                          uint32_t w3, uint4 b, uint4 bb, uint32_t mul2, uint32_t mul16) {
+    if constexpr (MT == 1) {
+        asm volatile(
+            "{\n\t.reg .b32 sa0,sa1,sa2,sa3,sb0,sb1,sb2,sb3,tt0,tt1,tt2,tt3,ha0,ha1,ha2,ha3,hb0,hb1,hb2,hb3;\n\t"
+            ".reg .b32 e00,e01,e02,e03,e10,e11,e12,e13,o00,o01,o02,o03,o10,o11,o12,o13;\n\t"
+            "and.b32 sa0, %8, 0x33333333;\n\t"
+            "mul.hi.u32 tt0, %8, %16;\n\t"
+            "and.b32 sb0, tt0, 0x33333333;\n\t"
+            "mul.hi.u32 ha0, sa0, %17;\n\t"
+            "mul.hi.u32 hb0, sb0, %17;\n\t"
+            "prmt.b32 e00, %18, 0, sa0;\n\t"
+            "prmt.b32 e10, %18, 0, ha0;\n\t"
+            "prmt.b32 o00, %18, 0, sb0;\n\t"
+            "prmt.b32 o10, %18, 0, hb0;\n\t"
+            "and.b32 sa1, %9, 0x33333333;\n\t"
+            "mul.hi.u32 tt1, %9, %16;\n\t"
+            "and.b32 sb1, tt1, 0x33333333;\n\t"
+            "mul.hi.u32 ha1, sa1, %17;\n\t"
+            "mul.hi.u32 hb1, sb1, %17;\n\t"
+            "prmt.b32 e01, %18, 0, sa1;\n\t"
+            "prmt.b32 e11, %18, 0, ha1;\n\t"
+            "prmt.b32 o01, %18, 0, sb1;\n\t"
+            "prmt.b32 o11, %18, 0, hb1;\n\t"
+            "and.b32 sa2, %10, 0x33333333;\n\t"
+            "mul.hi.u32 tt2, %10, %16;\n\t"
+            "and.b32 sb2, tt2, 0x33333333;\n\t"
+            "mul.hi.u32 ha2, sa2, %17;\n\t"
+            "mul.hi.u32 hb2, sb2, %17;\n\t"
+            "prmt.b32 e02, %18, 0, sa2;\n\t"
+            "prmt.b32 e12, %18, 0, ha2;\n\t"
+            "prmt.b32 o02, %18, 0, sb2;\n\t"
+            "prmt.b32 o12, %18, 0, hb2;\n\t"
+            "and.b32 sa3, %11, 0x33333333;\n\t"
+            "mul.hi.u32 tt3, %11, %16;\n\t"
+            "and.b32 sb3, tt3, 0x33333333;\n\t"
+            "mul.hi.u32 ha3, sa3, %17;\n\t"
+            "mul.hi.u32 hb3, sb3, %17;\n\t"
+            "prmt.b32 e03, %18, 0, sa3;\n\t"
+            "prmt.b32 e13, %18, 0, ha3;\n\t"
+            "prmt.b32 o03, %18, 0, sb3;\n\t"
+            "prmt.b32 o13, %18, 0, hb3;\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {e00,e01,o00,o01}, {%12,%13}, {%0,%1,%2,%3};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {e10,e11,o10,o11}, {%14,%15}, {%0,%1,%2,%3};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%4,%5,%6,%7}, {e02,e03,o02,o03}, {%12,%13}, {%4,%5,%6,%7};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%4,%5,%6,%7}, {e12,e13,o12,o13}, {%14,%15}, {%4,%5,%6,%7};\n\t"
+            "}\n"
+            : "+r"(acc[0][0][0]), "+r"(acc[0][0][1]), "+r"(acc[0][0][2]), "+r"(acc[0][0][3]),
+              "+r"(acc[1][0][0]), "+r"(acc[1][0][1]), "+r"(acc[1][0][2]), "+r"(acc[1][0][3])
+            : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w),
+              "r"(mul2), "r"(mul16), "r"(kCodeTable));
+    } else {
+        asm volatile(
+            "{\n\t.reg .b32 sa0,sa1,sa2,sa3,sb0,sb1,sb2,sb3,tt0,tt1,tt2,tt3,ha0,ha1,ha2,ha3,hb0,hb1,hb2,hb3;\n\t"
+            ".reg .b32 e00,e01,e02,e03,e10,e11,e12,e13,o00,o01,o02,o03,o10,o11,o12,o13;\n\t"
+            "and.b32 sa0, %16, 0x33333333;\n\t"
+            "mul.hi.u32 tt0, %16, %28;\n\t"
+            "and.b32 sb0, tt0, 0x33333333;\n\t"
+            "mul.hi.u32 ha0, sa0, %29;\n\t"
+            "mul.hi.u32 hb0, sb0, %29;\n\t"
+            "prmt.b32 e00, %30, 0, sa0;\n\t"
+            "prmt.b32 e10, %30, 0, ha0;\n\t"
+            "prmt.b32 o00, %30, 0, sb0;\n\t"
+            "prmt.b32 o10, %30, 0, hb0;\n\t"
+            "and.b32 sa1, %17, 0x33333333;\n\t"
+            "mul.hi.u32 tt1, %17, %28;\n\t"
+            "and.b32 sb1, tt1, 0x33333333;\n\t"
+            "mul.hi.u32 ha1, sa1, %29;\n\t"
+            "mul.hi.u32 hb1, sb1, %29;\n\t"
+            "prmt.b32 e01, %30, 0, sa1;\n\t"
+            "prmt.b32 e11, %30, 0, ha1;\n\t"
+            "prmt.b32 o01, %30, 0, sb1;\n\t"
+            "prmt.b32 o11, %30, 0, hb1;\n\t"
+            "and.b32 sa2, %18, 0x33333333;\n\t"
+            "mul.hi.u32 tt2, %18, %28;\n\t"
+            "and.b32 sb2, tt2, 0x33333333;\n\t"
+            "mul.hi.u32 ha2, sa2, %29;\n\t"
+            "mul.hi.u32 hb2, sb2, %29;\n\t"
+            "prmt.b32 e02, %30, 0, sa2;\n\t"
+            "prmt.b32 e12, %30, 0, ha2;\n\t"
+            "prmt.b32 o02, %30, 0, sb2;\n\t"
+            "prmt.b32 o12, %30, 0, hb2;\n\t"
+            "and.b32 sa3, %19, 0x33333333;\n\t"
+            "mul.hi.u32 tt3, %19, %28;\n\t"
+            "and.b32 sb3, tt3, 0x33333333;\n\t"
+            "mul.hi.u32 ha3, sa3, %29;\n\t"
+            "mul.hi.u32 hb3, sb3, %29;\n\t"
+            "prmt.b32 e03, %30, 0, sa3;\n\t"
+            "prmt.b32 e13, %30, 0, ha3;\n\t"
+            "prmt.b32 o03, %30, 0, sb3;\n\t"
+            "prmt.b32 o13, %30, 0, hb3;\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {e00,e01,o00,o01}, {%20,%21}, {%0,%1,%2,%3};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {e10,e11,o10,o11}, {%22,%23}, {%0,%1,%2,%3};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%4,%5,%6,%7}, {e02,e03,o02,o03}, {%20,%21}, {%4,%5,%6,%7};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%4,%5,%6,%7}, {e12,e13,o12,o13}, {%22,%23}, {%4,%5,%6,%7};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%8,%9,%10,%11}, {e00,e01,o00,o01}, {%24,%25}, {%8,%9,%10,%11};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%8,%9,%10,%11}, {e10,e11,o10,o11}, {%26,%27}, {%8,%9,%10,%11};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%12,%13,%14,%15}, {e02,e03,o02,o03}, {%24,%25}, {%12,%13,%14,%15};\n\t"
+            "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%12,%13,%14,%15}, {e12,e13,o12,o13}, {%26,%27}, {%12,%13,%14,%15};\n\t"
+            "}\n"
+            : "+r"(acc[0][0][0]), "+r"(acc[0][0][1]), "+r"(acc[0][0][2]), "+r"(acc[0][0][3]),
+              "+r"(acc[1][0][0]), "+r"(acc[1][0][1]), "+r"(acc[1][0][2]), "+r"(acc[1][0][3]),
+              "+r"(acc[0][MT - 1][0]), "+r"(acc[0][MT - 1][1]), "+r"(acc[0][MT - 1][2]), "+r"(acc[0][MT - 1][3]),
+              "+r"(acc[1][MT - 1][0]), "+r"(acc[1][MT - 1][1]), "+r"(acc[1][MT - 1][2]), "+r"(acc[1][MT - 1][3])
+            : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(bb.x), "r"(bb.y), "r"(bb.z), "r"(bb.w),
+              "r"(mul2), "r"(mul16), "r"(kCodeTable));
+    }
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
     constexpr int MP = 8 * MT;  // tokens per block (padded)
     extern __shared__ __align__(16) uint8_t smem[];
     // xs: for window chunk c, word i (0..3), token m, thread-in-group t: 16 permuted bytes
@@ -79,14 +202,14 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(GemvArgs a) {
     const int k_end = min(a.K, k_begin + a.Kc);
     const int64_t m0 = static_cast<int64_t>(blockIdx.z) * MP;
     const int64_t KB = a.K / 4;
+    const uint32_t mul2 = a.mul2, mul16 = a.mul16;
 
+    // Rows past N read the last row (always valid memory); their sums are never stored.
     const uint8_t* wrow[4];
-    bool wok[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int64_t row = row0 + g + 8 * r;
-        wok[r] = row < a.N;
-        wrow[r] = a.packed + (wok[r] ? row : 0) * KB;
+        wrow[r] = a.packed + (row < a.N ? row : a.N - 1) * KB + 16 * t;
     }
 
     int acc[2][MT][4];
@@ -97,46 +220,34 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(GemvArgs a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][j][e] = 0;
 
+    auto compute_chunk = [&](const uint4 (&buf)[4], int c) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint8_t* xb = xs + ((((c * 4 + i) * MP) + g) * 4 + t) * 16;
+            const uint4 b = *reinterpret_cast<const uint4*>(xb);
+            const uint4 bb = MT > 1 ? *reinterpret_cast<const uint4*>(xb + 8 * 4 * 16) : b;
+#define BL_W(R) (i == 0 ? buf[R].x : i == 1 ? buf[R].y : i == 2 ? buf[R].z : buf[R].w)
+            gemv_step<MT>(acc, BL_W(0), BL_W(1), BL_W(2), BL_W(3), b, bb, mul2, mul16);
+#undef BL_W
+        }
+    };
+
     for (int kw = k_begin; kw < k_end; kw += kWindow) {
         const int kw_end = min(k_end, kw + kWindow);
-        const int nch = (kw_end - kw + kChunk - 1) / kChunk;
+        const int nfull = (kw_end - kw) / kChunk;        // chunks of 256 codes
+        const int tail = (kw_end - kw) - nfull * kChunk;  // 0, 64, 128 or 192 codes
+        const int nch = nfull + (tail ? 1 : 0);
+        const int64_t kb = kw / 4;  // packed byte offset of the window in each row
 
-        // weights of chunk c of this window for this thread: 64 codes of each of its 4 rows
-        auto load_chunk = [&](uint4 (&buf)[4], int c) {
-            const int k = kw + c * kChunk + 64 * t;
-            const bool ok = c < nch && k < kw_end;
+        // weights of full chunk c of this window: 64 codes of each of this thread's 4 rows
+        auto load_full = [&](uint4 (&buf)[4], int c) {
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                buf[r] = (ok && wok[r]) ? ldg_stream_v4(wrow[r] + (k >> 2)) : make_uint4(0, 0, 0, 0);
-        };
-        auto compute_chunk = [&](const uint4 (&buf)[4], int c) {
-            if (c >= nch) return;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t e0[4], e1[4], o0[4], o1[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const uint32_t w = i == 0 ? buf[r].x : i == 1 ? buf[r].y : i == 2 ? buf[r].z : buf[r].w;
-                    unpack16_evenodd(w, e0[r], e1[r], o0[r], o1[r]);
-                }
-#pragma unroll
-                for (int j = 0; j < MT; ++j) {
-                    const uint4 b = *reinterpret_cast<const uint4*>(
-                        xs + ((((c * 4 + i) * MP) + 8 * j + g) * 4 + t) * 16);
-#pragma unroll
-                    for (int tile = 0; tile < 2; ++tile) {
-                        mma_m16n8k32_s8(acc[tile][j], e0[2 * tile], e0[2 * tile + 1], o0[2 * tile],
-                                        o0[2 * tile + 1], b.x, b.y);
-                        mma_m16n8k32_s8(acc[tile][j], e1[2 * tile], e1[2 * tile + 1], o1[2 * tile],
-                                        o1[2 * tile + 1], b.z, b.w);
-                    }
-                }
-            }
+            for (int r = 0; r < 4; ++r) buf[r] = ldg_stream_v4(wrow[r] + kb + c * (kChunk / 4));
         };
 
         uint4 bufA[4], bufB[4], bufC[4];
-        load_chunk(bufA, 0);
-        load_chunk(bufB, 1);
+        if (nfull > 0) load_full(bufA, 0);
+        if (nfull > 1) load_full(bufB, 1);
 
         // stage this window's activations, permuted to match the even/odd unpack
         __syncthreads();
@@ -154,13 +265,24 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(GemvArgs a) {
         }
         __syncthreads();
 
-        for (int c = 0; c < nch; c += 3) {
-            load_chunk(bufC, c + 2);
+        // full chunks: loads two chunks ahead, no per-load predicates
+        for (int c = 0; c < nfull; c += 3) {
+            if (c + 2 < nfull) load_full(bufC, c + 2);
             compute_chunk(bufA, c);
-            load_chunk(bufA, c + 3);
+            if (c + 1 >= nfull) break;
+            if (c + 3 < nfull) load_full(bufA, c + 3);
             compute_chunk(bufB, c + 1);
-            load_chunk(bufB, c + 4);
+            if (c + 2 >= nfull) break;
+            if (c + 4 < nfull) load_full(bufB, c + 4);
             compute_chunk(bufC, c + 2);
+        }
+        if (tail) {
+            // last partial chunk: thread t holds codes [64 t, 64 t + 64) of it
+            const bool ok = 64 * t < tail;
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                bufA[r] = ok ? ldg_stream_v4(wrow[r] + kb + nfull * (kChunk / 4)) : make_uint4(0, 0, 0, 0);
+            compute_chunk(bufA, nfull);
         }
     }
 
@@ -287,15 +409,30 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
     const int64_t row_blocks = (N + kGvRows - 1) / kGvRows;
     const int MT = M <= 8 ? 1 : 2;
     const int64_t token_blocks = (M + 8 * MT - 1) / (8 * MT);
-    // K slices: enough blocks for ~2 per SM, at least one chunk per slice, at most 8.
+    // K slices (the cluster size S <= 8, at least one chunk per slice): pick the S whose
+    // block count fills the resident slots (2 blocks per SM) in the most even waves,
+    // preferring more blocks among near ties.
     const int64_t kchunks = (K + kChunk - 1) / kChunk;
-    int64_t S = (2 * sms + row_blocks * token_blocks - 1) / (row_blocks * token_blocks);
-    if (S < 1) S = 1;
-    if (S > kMaxCluster) S = kMaxCluster;
-    if (S > kchunks) S = kchunks;
+    const int64_t slots = 2 * static_cast<int64_t>(sms);
+    int64_t S = 1;
+    double best = -1.0;
+    for (int64_t cand = 1; cand <= kMaxCluster && cand <= kchunks; ++cand) {
+        const int64_t kc = ((K + cand - 1) / cand + kChunk - 1) / kChunk * kChunk;
+        if ((K + kc - 1) / kc != cand) continue;  // that split leaves an empty slice
+        const int64_t blocks = row_blocks * token_blocks * cand;
+        const int64_t waves = (blocks + slots - 1) / slots;
+        const double eff = static_cast<double>(blocks) / static_cast<double>(waves * slots);
+        if (eff > best + 0.02) {
+            best = eff;
+            S = cand;
+        } else if (eff > best - 0.02 && waves == 1) {
+            S = cand;  // a single, fuller wave with more, shorter blocks
+            best = eff > best ? eff : best;
+        }
+    }
     int64_t Kc = ((K + S - 1) / S + kChunk - 1) / kChunk * kChunk;
     S = (K + Kc - 1) / Kc;
-    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind};
+    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind, 1u << 30, 1u << 16};
     if (MT == 1) return launch_gemv_mt<1>(a, static_cast<int>(S), row_blocks, token_blocks, stream);
     return launch_gemv_mt<2>(a, static_cast<int>(S), row_blocks, token_blocks, stream);
 }
@@ -303,7 +440,7 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                                 int kind, cudaStream_t stream) {
-    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind};
+    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16};
     const int64_t total = M * N;
     gemv_generic_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(a);
     return cudaGetLastError();

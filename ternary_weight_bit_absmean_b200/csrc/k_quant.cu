@@ -10,8 +10,9 @@
 // by their absmax to signed 8 bits with no zero point.
 //
 // Bit-exactness: every float step is the IEEE operation the definition names --
-// __fdiv_rn for W / gamma and 127 / absmax, __fmul_rn for x * s, __float2int_rn
-// (round half to even) for round(); nothing here is compiled with fast-math.
+// __fdiv_rn for W / gamma and 127 / absmax, __fmul_rn for x * s, and a round half to
+// even for round() (__float2int_rn for the weights, an exact add of 1.5 * 2^23 for the
+// activations); nothing here is compiled with fast-math.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -113,10 +114,22 @@ __device__ __forceinline__ uint32_t encode_byte_code(uint32_t b, bool& bad) {
     return 0u;
 }
 
+// Four int8 codes (one per byte of w) -> one packed byte.  For valid bytes (0x00, 0x01,
+// 0xFF) the "-1" flag is the sign bit and the "+1" flag the low bit without the sign;
+// the flags of byte j sit at bits 8j and 8j+1 of x, and one multiply by
+// 2^24 + 2^18 + 2^12 + 2^6 moves them to bits 24+2j (the other partial products land
+// in disjoint fields below bit 24 or above bit 31, so nothing carries).  A word whose
+// flags do not re-expand to itself holds an invalid code; it takes the per-byte path,
+// which writes invalid codes as 00.
 __device__ __forceinline__ uint32_t pack_word_codes(uint32_t w, bool& bad) {
-    return encode_byte_code(w & 0xFFu, bad) | (encode_byte_code((w >> 8) & 0xFFu, bad) << 2) |
-           (encode_byte_code((w >> 16) & 0xFFu, bad) << 4) |
-           (encode_byte_code(w >> 24, bad) << 6);
+    const uint32_t minus = (w >> 7) & 0x01010101u;
+    const uint32_t plus = w & ~(w >> 7) & 0x01010101u;
+    if ((plus | (minus * 0xFFu)) != w) {
+        return encode_byte_code(w & 0xFFu, bad) | (encode_byte_code((w >> 8) & 0xFFu, bad) << 2) |
+               (encode_byte_code((w >> 16) & 0xFFu, bad) << 4) | (encode_byte_code(w >> 24, bad) << 6);
+    }
+    const uint32_t x = plus | (minus << 1);
+    return (x * 0x01041040u) >> 24;
 }
 
 __global__ void __launch_bounds__(256) pack_codes_kernel(const uint4* __restrict__ codes16,
@@ -124,38 +137,54 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint4* __restrict
                                                          uint8_t* __restrict__ packed,
                                                          int32_t* __restrict__ err) {
     bool bad = false;
-    const int64_t ngroups = numel / 16;
+    const int64_t ngroups = numel / 16;  // 16 codes -> one 32-bit word
     uint32_t* packed32 = reinterpret_cast<uint32_t*>(packed);
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < ngroups;
-         i += stride) {
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    // four groups per thread per step, all loads issued before any is used
+    int64_t i = tid;
+    for (; i + 3 * nthreads < ngroups; i += 4 * nthreads) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(codes16 + i + u * nthreads);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            packed32[i + u * nthreads] = pack_word_codes(v[u].x, bad) | (pack_word_codes(v[u].y, bad) << 8) |
+                                         (pack_word_codes(v[u].z, bad) << 16) | (pack_word_codes(v[u].w, bad) << 24);
+    }
+    for (; i < ngroups; i += nthreads) {
         const uint4 v = __ldg(codes16 + i);
         packed32[i] = pack_word_codes(v.x, bad) | (pack_word_codes(v.y, bad) << 8) |
                       (pack_word_codes(v.z, bad) << 16) | (pack_word_codes(v.w, bad) << 24);
     }
     const uint32_t* codes4 = reinterpret_cast<const uint32_t*>(codes16);
-    for (int64_t j = ngroups * 4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-         j < numel / 4; j += stride)
+    for (int64_t j = ngroups * 4 + tid; j < numel / 4; j += nthreads)
         packed[j] = static_cast<uint8_t>(pack_word_codes(__ldg(codes4 + j), bad));
     if (bad && err != nullptr) atomicOr(err, kErrBitBadCode);
 }
 
 // --------------------------------------------------- activation quantisation --
-// bf16 pairs -> int8: x * s rounded half to even, clipped to [-128, 127].
-__device__ __forceinline__ uint32_t quant_pair(uint32_t w, float s) {
-    const float lo = __uint_as_float(w << 16);
-    const float hi = __uint_as_float(w & 0xFFFF0000u);
-    int ql = __float2int_rn(__fmul_rn(lo, s));
-    int qh = __float2int_rn(__fmul_rn(hi, s));
-    ql = max(-128, min(127, ql));
-    qh = max(-128, min(127, qh));
-    return (static_cast<uint32_t>(ql) & 0xFFu) | ((static_cast<uint32_t>(qh) & 0xFFu) << 8);
+// round-half-even(x * s) as an int8 bit pattern in the low byte of the result.
+// t = fl(x * s) satisfies |t| <= 127 (1 + 2^-23): s = fl(127 / max(a, eps)) with
+// |x| <= a, or |x| <= a < eps.  Adding 1.5 * 2^23 to such a t rounds it to the nearest
+// integer, ties to even, in one IEEE add, leaving that integer in the low mantissa
+// bits; rint(t) is within [-127, 127], so the clip to [-128, 127] is never active.
+__device__ __forceinline__ uint32_t q8_bits(float x, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(x, s), 12582912.0f));
 }
 
+// 8 bf16 (one 16-byte vector) -> 8 int8 (8 bytes).
 __device__ __forceinline__ uint2 quant8(uint4 v, float s) {
+    uint32_t q[8];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        q[2 * i] = q8_bits(__uint_as_float(w[i] << 16), s);
+        q[2 * i + 1] = q8_bits(__uint_as_float(w[i] & 0xFFFF0000u), s);
+    }
     uint2 r;
-    r.x = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
-    r.y = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+    r.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+    r.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
     return r;
 }
 
@@ -171,58 +200,68 @@ __device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
 
 // One group of G threads per token row; each thread keeps up to NV 16-byte vectors of
 // its row in registers between the absmax pass and the quantise pass (longer rows are
-// re-read for the remainder).  Needs K % 8 == 0.
-template <int G>
+// re-read for the remainder).  Short rows (G = 32) give each warp R rows, whose loads
+// are all issued before the first reduction.  Needs K % 8 == 0.
+template <int G, int R>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
                          uint2* __restrict__ xq, float* __restrict__ s_out) {
     constexpr int CTA = G > 256 ? G : 256;
-    constexpr int RPC = CTA / G;   // rows per block
-    constexpr int WPG = G / 32;    // warps per row group
-    constexpr int NV = 8;
+    constexpr int RPC = CTA / G * R;  // rows per block
+    constexpr int WPG = G / 32;       // warps per row group
+    constexpr int NV = (R > 1) ? 4 : 8;
+    static_assert(R == 1 || G == 32, "several rows per group only for warp groups");
     __shared__ uint32_t red[CTA / 32];
 
     const int sub = threadIdx.x / G;
     const int j = threadIdx.x % G;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + sub;
     const int nvec = K / 8;
-    const bool active = row < M;
-    const uint4* xr = X + (active ? row : 0) * nvec;
+    const int64_t row_base = static_cast<int64_t>(blockIdx.x) * RPC + static_cast<int64_t>(sub) * R;
 
-    uint4 v[NV];
-    uint32_t m2 = 0;
+    uint4 v[R][NV];
+    uint32_t m2[R];
 #pragma unroll
-    for (int u = 0; u < NV; ++u) {
-        const int idx = j + u * G;
-        if (active && idx < nvec) {
-            v[u] = __ldg(xr + idx);
-            m2 = absmax_vec(m2, v[u]);
-        } else {
-            v[u] = make_uint4(0, 0, 0, 0);
+    for (int r = 0; r < R; ++r) {
+        const int64_t row = row_base + r;
+        const bool active = row < M;
+        const uint4* xr = X + (active ? row : 0) * nvec;
+        m2[r] = 0;
+#pragma unroll
+        for (int u = 0; u < NV; ++u) {
+            const int idx = j + u * G;
+            v[r][u] = (active && idx < nvec) ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
         }
     }
-    for (int idx = j + NV * G; active && idx < nvec; idx += G) m2 = absmax_vec(m2, __ldg(xr + idx));
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int64_t row = row_base + r;
+        const bool active = row < M;
+        const uint4* xr = X + (active ? row : 0) * nvec;
+#pragma unroll
+        for (int u = 0; u < NV; ++u) m2[r] = absmax_vec(m2[r], v[r][u]);
+        for (int idx = j + NV * G; active && idx < nvec; idx += G) m2[r] = absmax_vec(m2[r], __ldg(xr + idx));
 
-    uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
-    for (int off = 16; off > 0; off >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
-    if constexpr (WPG > 1) {
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
-        __syncthreads();
-        am = 0;
+        uint32_t am = max(m2[r] & 0xFFFFu, m2[r] >> 16);
+        for (int off = 16; off > 0; off >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
+        if constexpr (WPG > 1) {
+            if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+            __syncthreads();
+            am = 0;
 #pragma unroll
-        for (int w = 0; w < WPG; ++w) am = max(am, red[sub * WPG + w]);
-    }
-    const float a = __uint_as_float(am << 16);
-    const float s = __fdiv_rn(127.0f, fmaxf(a, eps));
-    if (!active) return;
-    if (j == 0) s_out[row] = s;
-    uint2* qr = xq + row * nvec;
+            for (int w = 0; w < WPG; ++w) am = max(am, red[sub * WPG + w]);
+        }
+        const float a = __uint_as_float(am << 16);
+        const float s = __fdiv_rn(127.0f, fmaxf(a, eps));
+        if (!active) continue;
+        if (j == 0) s_out[row] = s;
+        uint2* qr = xq + row * nvec;
 #pragma unroll
-    for (int u = 0; u < NV; ++u) {
-        const int idx = j + u * G;
-        if (idx < nvec) qr[idx] = quant8(v[u], s);
+        for (int u = 0; u < NV; ++u) {
+            const int idx = j + u * G;
+            if (idx < nvec) qr[idx] = quant8(v[r][u], s);
+        }
+        for (int idx = j + NV * G; idx < nvec; idx += G) qr[idx] = quant8(__ldg(xr + idx), s);
     }
-    for (int idx = j + NV * G; idx < nvec; idx += G) qr[idx] = quant8(__ldg(xr + idx), s);
 }
 
 // Any K: one warp per row, scalar loads.
@@ -297,16 +336,18 @@ cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float e
     const uint4* X4 = reinterpret_cast<const uint4*>(X);
     uint2* q8 = reinterpret_cast<uint2*>(xq);
     const int Ki = static_cast<int>(K);
-    if (nvec <= 128) {
-        act_quant_vec_kernel<32><<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    if (nvec <= 32) {
+        act_quant_vec_kernel<32, 4><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+    } else if (nvec <= 128) {
+        act_quant_vec_kernel<32, 2><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
     } else if (nvec <= 256) {
-        act_quant_vec_kernel<64><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+        act_quant_vec_kernel<64, 1><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
     } else if (nvec <= 512) {
-        act_quant_vec_kernel<128><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+        act_quant_vec_kernel<128, 1><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
     } else if (nvec <= 1024) {
-        act_quant_vec_kernel<256><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
+        act_quant_vec_kernel<256, 1><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
     } else {
-        act_quant_vec_kernel<512><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, Ki, eps, q8, s);
+        act_quant_vec_kernel<512, 1><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, Ki, eps, q8, s);
     }
     return cudaGetLastError();
 }

@@ -102,7 +102,8 @@ def test_other_entry_points_validation(L):
     assert fwd(FAKE, FAKE, FAKE, FAKE, 4, 8, 1 << 25, FAKE, 0, None, None) == SHAPE
     assert fwd(FAKE, ODD, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, None) == MISALIGNED
     path = L.bitlinear_forward_path
-    assert path(FAKE, FAKE, FAKE, FAKE, 40, 8, 96, FAKE, 0, None, 2, None) == SHAPE  # tcgen05 needs K % 64
+    for p in (2, 3, 4):  # every tcgen05 variant needs K % 64 == 0
+        assert path(FAKE, FAKE, FAKE, FAKE, 40, 8, 96, FAKE, 0, None, p, None) == SHAPE
     assert path(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 9, None) == INVALID
     assert L.bitlinear_status_string(3) == b"BL_ERR_MISALIGNED"
 

@@ -216,9 +216,10 @@ TC_CASES = [(17, 128, 128), (32, 256, 256), (64, 512, 256), (100, 300, 192), (25
             (8192, 512, 256), (130, 640, 8192)]
 
 
+@pytest.mark.parametrize("path", [B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM], ids=["tc1sm", "tc2sm"])
 @pytest.mark.parametrize("M,N,K", TC_CASES)
-def test_forward_tc(M, N, K):
-    check_forward(M, N, K, B.BL_PATH_TC, seed=M * 3 + N + K)
+def test_forward_tc(M, N, K, path):
+    check_forward(M, N, K, path, seed=M * 3 + N + K)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 64, 100), (3, 33, 4), (20, 17, 36), (5, 7, 1000)])
@@ -228,11 +229,11 @@ def test_forward_generic_k(M, N, K):
 
 
 def test_forward_paths_agree_and_are_deterministic():
-    g_ref, packed_ref, xq_ref, s_ref = make_problem(48, 768, 2048, 11)
-    a = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_GEMV)
-    b = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_TC)
-    c = run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, B.BL_PATH_TC)
-    assert torch.equal(a, b) and torch.equal(b, c)
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(300, 768, 2048, 11)
+    outs = [run_forward(xq_ref, s_ref, packed_ref, g_ref, torch.int32, p)
+            for p in (B.BL_PATH_GEMV, B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM, B.BL_PATH_TC, B.BL_PATH_TC_2SM)]
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
 
 
 def test_forward_zero_weights_give_zero():
@@ -241,7 +242,7 @@ def test_forward_zero_weights_give_zero():
     s = torch.ones(M, device=DEV)
     packed = torch.zeros(N, K // 4, dtype=torch.uint8, device=DEV)
     gamma = torch.tensor([EPS], device=DEV)
-    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC):
+    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM):
         y = B.forward(xq, s, packed, gamma, torch.float32, path=path)
         sync()
         assert not y.any().item()
@@ -257,7 +258,7 @@ def test_forward_extreme_accumulators():
     s = torch.ones(M, device=DEV)
     gamma = torch.tensor([1.0], device=DEV)
     want = (xq.long().sum(1)[:, None] * torch.where(torch.arange(N, device=DEV) % 3 == 0, -1, 1)[None, :])
-    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC):
+    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM):
         acc = B.forward(xq, s, packed, gamma, torch.int32, path=path)
         sync()
         assert torch.equal(acc.long(), want)
