@@ -13,11 +13,14 @@ of one LLaMA-700M-shaped layer (hidden 1536, FFN 4096: q/k/v/o 1536x1536, up/gat
 divided by the device time of the whole step, in TOPS, summed over ranks (each rank
 runs its own step: weak scaling, no collective on the data path).
 
-Timing: the step is captured once in a CUDA graph with timing events around every
-library call; each timed replay is bracketed by events, L2 is flushed (256 MiB write)
-between replays outside the events, and K replays are bracketed by a barrier and a
-device synchronisation.  `e2e` repeats the step with its inputs copied from pinned
-host memory and its outputs copied back inside the timed region.
+Timing: the step is captured once as a CUDA graph.  Each timed replay is bracketed by
+device events; between replays, outside the events, L2 is flushed (256 MiB written and
+another 256 MiB read, so no dirty line is left behind); K replays are bracketed by a
+barrier and a device synchronisation and the time is the maximum over ranks.  A second
+copy of the graph with a timing event around every library call gives the per-call
+breakdown and the roofline of the dominant kernel from the same number of replays.
+`e2e` repeats the step with its inputs copied from pinned host memory and its outputs
+copied back inside the timed region.
 
 --impl reference runs the CPU oracle (plain C, one core) on a bounded sample of the
 same workload and reports the same metric.
@@ -56,6 +59,8 @@ def parse():
     p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2"], default="auto")
     p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
     p.add_argument("--iters", type=int, default=20)
+    p.add_argument("--xq-layout", choices=["evenodd", "rowmajor"], default="evenodd",
+                   help="storage order of the int8 activations between quantize_act and forward")
     return p.parse_args()
 
 
@@ -77,6 +82,43 @@ def workload():
 
 def fwd_ops(projs, Ms):
     return sum(2 * M * N * K for M in Ms for (_, N, K) in projs)
+
+
+def rank_seed(pi, M, rank):
+    """Activation seed of projection pi at M tokens on a rank: every rank runs its own
+    token batch (data parallel), the weights are the same on every rank."""
+    return pi + 97 * M + 7919 * rank
+
+
+def max_over_ranks(x, device=None):
+    """The largest value of x over all ranks (x itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def whole_job_tops(ops_per_step, steps, world, total_ms_max):
+    """Work of all ranks over the slowest rank's device time, in TOPS."""
+    return ops_per_step * steps * world / (total_ms_max * 1e-3) / 1e12
+
+
+class L2Flusher:
+    """Evicts the L2 between timed iterations: writes a buffer twice the L2 size, then
+    reads a second one so that the evicted lines are clean and no write-back of flush
+    data lands inside the next timed region."""
+
+    def __init__(self, device, nbytes=256 << 20):
+        import torch
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.r = torch.ones(nbytes // 4, dtype=torch.int32, device=device)
+
+    def flush(self):
+        self.w.fill_(1)
+        self.sink = self.r.max()
 
 
 # ----------------------------------------------------------------- clocks --
@@ -157,10 +199,11 @@ def run_ours(args):
     B.lib()
 
     projs, Ms, ofrac = workload()
+    XQ_LAYOUT = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
     # inputs: weights are the same model replica on every rank; tokens differ per rank
     W = [synth.weight(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
     C = [synth.codes(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
-    X = {(pi, M): synth.activations(M, K, seed=pi + 97 * M + 7919 * rank, outlier_frac=ofrac).to(dev)
+    X = {(pi, M): synth.activations(M, K, seed=rank_seed(pi, M, rank), outlier_frac=ofrac).to(dev)
          for M in Ms for pi, (_, N, K) in enumerate(projs)}
     gam = [torch.empty(1, dtype=torch.float32, device=dev) for _ in projs]
     pk = [torch.empty(N, K // 4, dtype=torch.uint8, device=dev) for (_, N, K) in projs]
@@ -169,7 +212,7 @@ def run_ours(args):
     xq = {(pi, M): torch.empty(M, K, dtype=torch.int8, device=dev) for M in Ms for pi, (_, N, K) in enumerate(projs)}
     sc = {(pi, M): torch.empty(M, dtype=torch.float32, device=dev) for M in Ms for pi, _ in enumerate(projs)}
     Y = {(pi, M): torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in Ms for pi, (_, N, K) in enumerate(projs)}
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flusher = L2Flusher(dev)
 
     # (label, callable) list in step order; labels name the hot-path row
     calls = []
@@ -179,8 +222,10 @@ def run_ours(args):
         calls.append((("a3", pi, 0), lambda pi=pi: B.bitlinear_pack(C[pi], pk2[pi])))
     for M in sorted(Ms, reverse=True):
         for pi, _ in enumerate(projs):
-            calls.append((("a4", pi, M), lambda pi=pi, M=M: B.bitlinear_quantize_act(X[pi, M], EPS, xq[pi, M], sc[pi, M])))
-            calls.append((("fwd", pi, M), lambda pi=pi, M=M: B.bitlinear_forward(xq[pi, M], sc[pi, M], pk[pi], gam[pi], Y[pi, M])))
+            calls.append((("a4", pi, M), lambda pi=pi, M=M: B.bitlinear_quantize_act(
+                X[pi, M], EPS, xq[pi, M], sc[pi, M], layout=XQ_LAYOUT)))
+            calls.append((("fwd", pi, M), lambda pi=pi, M=M: B.bitlinear_forward(
+                xq[pi, M], sc[pi, M], pk[pi], gam[pi], Y[pi, M], layout=XQ_LAYOUT)))
     launches_per_call = {"a1a2": 2, "a3": 1, "a4": 1, "fwd": 1}
     launches_per_step = sum(launches_per_call[lab[0]] for lab, _ in calls)
 
@@ -191,28 +236,41 @@ def run_ours(args):
                 fn()
     torch.cuda.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-          for _ in calls]
-    ev_step = (torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+    # the step as a CUDA graph; a second copy carries a timing event around every call
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        ev_step[0].record()
+        for _, fn in calls:
+            fn()
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in calls]
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
         for (lab, fn), (e0, e1) in zip(calls, ev):
             e0.record()
             fn()
             e1.record()
-        ev_step[1].record()
     torch.cuda.synchronize()
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def one_step():
         with torch.cuda.stream(stream):
-            flush.fill_(1)
+            flusher.flush()
+            e_a.record()
             graph.replay()
+            e_b.record()
         torch.cuda.synchronize()
-        return ev_step[0].elapsed_time(ev_step[1]), [e0.elapsed_time(e1) for e0, e1 in ev]
+        return e_a.elapsed_time(e_b)
+
+    def one_instrumented_step():
+        with torch.cuda.stream(stream):
+            flusher.flush()
+            graph_ev.replay()
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
 
     for _ in range(max(3, args.warmup)):
         one_step()
+        one_instrumented_step()
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -220,21 +278,17 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms, call_ms = [], [0.0] * len(calls)
-    for _ in range(args.steps):
-        t, per = one_step()
-        step_ms.append(t)
-        call_ms = [a + b for a, b in zip(call_ms, per)]
+    step_ms = [one_step() for _ in range(args.steps)]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    # per-call device times from the same number of instrumented replays of the step
+    call_ms = [0.0] * len(calls)
+    for _ in range(args.steps):
+        call_ms = [a + b for a, b in zip(call_ms, one_instrumented_step())]
     call_ms = [c / args.steps for c in call_ms]
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = t.item()
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> pinned host
     h_W = [w.cpu().pin_memory() for w in W]
@@ -244,10 +298,9 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in h_W + h_C + list(h_X.values()))
     d2h = sum(t.numel() * t.element_size() for t in h_Y.values())
     e2e_ms = []
-    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(args.e2e_steps + 1):
         with torch.cuda.stream(stream):
-            flush.fill_(1)
+            flusher.flush()
             e_a.record()
             for d, h in zip(W, h_W):
                 d.copy_(h, non_blocking=True)
@@ -262,15 +315,11 @@ def run_ours(args):
         torch.cuda.synchronize()
         if i > 0:
             e2e_ms.append(e_a.elapsed_time(e_b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = t.item()
+    e2e_total = max_over_ranks(sum(e2e_ms), dev)
 
     ops_step = fwd_ops(projs, Ms)
-    value = ops_step * args.steps * world / (total_ms * 1e-3) / 1e12
-    e2e_value = ops_step * len(e2e_ms) * world / (e2e_total * 1e-3) / 1e12 if e2e_ms else None
+    value = whole_job_tops(ops_step, args.steps, world, total_ms)
+    e2e_value = whole_job_tops(ops_step, len(e2e_ms), world, e2e_total) if e2e_ms else None
 
     # ---- per-row breakdown and the dominant kernel's roofline
     pk_bytes = {pi: N * K // 4 for pi, (_, N, K) in enumerate(projs)}
@@ -313,10 +362,10 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
         "data": "synthetic (seeded N(0,0.02) fp32 weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
         "config": {"workload": "llama700m BitLinear set: q/k/v/o 1536x1536, up/gate 1536->4096, down 4096->1536",
-                   "M": Ms, "out_dtype": "bf16", "eps": EPS,
+                   "M": Ms, "out_dtype": "bf16", "eps": EPS, "xq_layout": args.xq_layout,
                    "stages": "a1+a2 quantize_weights x7, a3 pack x7, a4 quantize_act x28, a5/a6 forward x28",
-                   "l2": "flushed between steps (256 MiB write outside the timed events)",
-                   "timing": "CUDA graph replay, device events, sum over steps, max over ranks",
+                   "l2": "flushed between steps outside the timed events (256 MiB written, then another 256 MiB read so no dirty line is left)",
+                   "timing": "CUDA graph replay of the step bracketed by device events, summed over steps, max over ranks; per-call breakdown and roofline from the same number of replays of an instrumented copy of the graph",
                    "parallelism": "dp%d (independent token batches per GPU, replicated weights)" % world},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(e2e_value, 4) if e2e_value is not None else None, "unit": "TOPS",
@@ -330,6 +379,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(projs, Ms, ofrac, tokens=48)
     graph.reset()
+    graph_ev.reset()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -414,7 +464,7 @@ def run_single(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     M, N, K = args.M, args.N, args.K
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flusher = L2Flusher(dev)
     P = peaks()
     if args.single == "forward":
         xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
@@ -428,14 +478,16 @@ def run_single(args):
         out = torch.empty(M, N, dtype=odt, device=dev)
         path = {"auto": B.BL_PATH_AUTO, "gemv": B.BL_PATH_GEMV, "tc": B.BL_PATH_TC, "tc1": B.BL_PATH_TC_1SM,
                 "tc2": B.BL_PATH_TC_2SM}[args.path]
-        fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path)
+        lay = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
+        fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=lay)
         ops = 2 * M * N * K
         nbytes = N * K // 4 + M * K + 4 * M + M * N * out.element_size()
     elif args.single == "quantize_act":
         X = torch.randn(M, K, device=dev).to(torch.bfloat16)
         xq = torch.empty(M, K, dtype=torch.int8, device=dev)
         s = torch.empty(M, device=dev)
-        fn = lambda: B.bitlinear_quantize_act(X, EPS, xq, s)
+        lay = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
+        fn = lambda: B.bitlinear_quantize_act(X, EPS, xq, s, layout=lay)
         ops, nbytes = 0, 3 * M * K + 4 * M
     elif args.single == "quantize_weights":
         W = torch.randn(N, K, device=dev) * 0.02
@@ -455,7 +507,7 @@ def run_single(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ts = []
     for _ in range(args.iters):
-        flush.fill_(1)
+        flusher.flush()
         e0.record()
         fn()
         e1.record()
@@ -463,6 +515,7 @@ def run_single(args):
         ts.append(e0.elapsed_time(e1))
     t = statistics.median(ts) * 1e-3
     rec = {"single": args.single, "M": M, "N": N, "K": K, "path": args.path, "out_dtype": args.out_dtype,
+           "xq_layout": args.xq_layout,
            "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
            "gbs": round(nbytes / t / 1e9, 1), "hbm_frac": round(nbytes / t / 1e9 / P["hbm_gbs"], 4),
            "weight_gbs": round((N * K // 4) / t / 1e9, 1) if args.single == "forward" else None}

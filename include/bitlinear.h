@@ -85,6 +85,19 @@ typedef enum {
     BL_PATH_TC_2SM = 4  /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
 } bl_path;
 
+/* Storage order of x_q within each row.
+ *   BL_XQ_ROWMAJOR     element k at byte k (the plain [M, K] int8 matrix).
+ *   BL_XQ_K16_EVENODD  K % 16 == 0; inside every group of 16 consecutive elements
+ *                      (k = 16q + e) the bytes hold the elements in the order
+ *                      e = 0,2,4,6, 8,10,12,14, 1,3,5,7, 9,11,13,15 (element e sits at
+ *                      byte 16q + 8(e%2) + 4(e/8) + (e%8)/2).  The values are the same;
+ *                      this order matches the cheaper unpack of the packed weights, so
+ *                      the forward runs faster on it. */
+typedef enum {
+    BL_XQ_ROWMAJOR = 0,
+    BL_XQ_K16_EVENODD = 1
+} bl_xq_layout;
+
 /* Bytes of device workspace bitlinear_quantize_weights needs for an [N, K] matrix
  * (fp64 partial sums of |W|).  Depends on N*K only; 0 for a non-positive size. */
 BL_API size_t bitlinear_workspace_size(int64_t N, int64_t K);
@@ -132,6 +145,12 @@ BL_API bl_status bitlinear_pack(const int8_t *codes, int64_t N, int64_t K, uint8
 BL_API bl_status bitlinear_quantize_act(const uint16_t *X, int64_t M, int64_t K, float eps,
                                  int8_t *xq_out, float *s_out, void *stream);
 
+/* bitlinear_quantize_act writing x_q in the given layout (see bl_xq_layout).
+ * BL_XQ_K16_EVENODD needs K % 16 == 0 (else BL_ERR_UNSUPPORTED_SHAPE). */
+BL_API bl_status bitlinear_quantize_act_layout(const uint16_t *X, int64_t M, int64_t K, float eps,
+                                               int8_t *xq_out, float *s_out, bl_xq_layout layout,
+                                               void *stream);
+
 /* [BIN] + [STE] + [CH2] the BitLinear forward from quantised operands:
  *   acc[m, n] = sum_k x_q[m, k] * c[n, k]   (exact, int32)
  *   y[m, n]   = float(acc[m, n]) * (gamma / s[m])   (fp32: the quotient and the product
@@ -178,6 +197,13 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
 BL_API bl_status bitlinear_quantize_weights_noalloc(const float *W, int64_t N, int64_t K, float eps,
                                                     float *gamma_out, uint8_t *packed_out,
                                                     void *stream);
+
+/* bitlinear_forward_path reading x_q stored in the given layout (see bl_xq_layout);
+ * the result is the same for either layout. */
+BL_API bl_status bitlinear_forward_layout(const int8_t *xq, const float *s, const uint8_t *packed,
+                                          const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
+                                          bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,
+                                          bl_path path, void *stream);
 
 /* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
 BL_API int bitlinear_last_cuda_error(void);

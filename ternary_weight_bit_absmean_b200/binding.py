@@ -24,11 +24,13 @@ BL_OK = 0
 BL_OUT_F32, BL_OUT_BF16, BL_OUT_I32 = 0, 1, 2
 BL_PATH_AUTO, BL_PATH_GEMV, BL_PATH_TC, BL_PATH_TC_1SM, BL_PATH_TC_2SM = 0, 1, 2, 3, 4
 BL_ERRBIT_BAD_CODE, BL_ERRBIT_TIMEOUT = 0x1, 0x2
+BL_XQ_ROWMAJOR, BL_XQ_K16_EVENODD = 0, 1
 
 EXPORTED = [
     "bitlinear_workspace_size", "bitlinear_quantize_weights",
     "bitlinear_quantize_weights_with_scale", "bitlinear_pack", "bitlinear_quantize_act",
-    "bitlinear_forward", "bitlinear_forward_path", "bitlinear_last_cuda_error",
+    "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
+    "bitlinear_forward_layout", "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
 
@@ -70,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward.restype = S
         L.bitlinear_forward_path.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, P]
         L.bitlinear_forward_path.restype = S
+        L.bitlinear_quantize_act_layout.argtypes = [P, I64, I64, F, P, P, S, P]
+        L.bitlinear_quantize_act_layout.restype = S
+        L.bitlinear_forward_layout.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, S, P]
+        L.bitlinear_forward_layout.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
         L.bitlinear_last_cuda_error.restype = ctypes.c_int
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
@@ -132,17 +138,22 @@ def bitlinear_pack(codes, packed_out, err_word=None, stream=None):
         _opt(err_word, "err_word"), _stream(stream)), "bitlinear_pack")
 
 
-def bitlinear_quantize_act(X, eps, xq_out, s_out, stream=None):
+def bitlinear_quantize_act(X, eps, xq_out, s_out, stream=None, layout=BL_XQ_ROWMAJOR):
     M, K = X.shape
-    _check(lib().bitlinear_quantize_act(
-        _dev(X, torch.bfloat16, "X"), M, K, float(eps), _dev(xq_out, torch.int8, "xq_out", (M, K)),
-        _dev(s_out, torch.float32, "s_out", (M,)), _stream(stream)), "bitlinear_quantize_act")
+    args = (_dev(X, torch.bfloat16, "X"), M, K, float(eps), _dev(xq_out, torch.int8, "xq_out", (M, K)),
+            _dev(s_out, torch.float32, "s_out", (M,)))
+    if layout == BL_XQ_ROWMAJOR:
+        _check(lib().bitlinear_quantize_act(*args, _stream(stream)), "bitlinear_quantize_act")
+    else:
+        _check(lib().bitlinear_quantize_act_layout(*args, int(layout), _stream(stream)),
+               "bitlinear_quantize_act_layout")
 
 
 _OUT_DT = {BL_OUT_F32: torch.float32, BL_OUT_BF16: torch.bfloat16, BL_OUT_I32: torch.int32}
 
 
-def bitlinear_forward(xq, s, packed, gamma, out, err_word=None, stream=None, path=BL_PATH_AUTO):
+def bitlinear_forward(xq, s, packed, gamma, out, err_word=None, stream=None, path=BL_PATH_AUTO,
+                      layout=BL_XQ_ROWMAJOR):
     M, K = xq.shape
     N = packed.shape[0]
     kind = {v: k for k, v in _OUT_DT.items()}.get(out.dtype)
@@ -151,7 +162,10 @@ def bitlinear_forward(xq, s, packed, gamma, out, err_word=None, stream=None, pat
     args = (_dev(xq, torch.int8, "xq"), _dev(s, torch.float32, "s", (M,)),
             _dev(packed, torch.uint8, "packed", (N, K // 4)), _dev(gamma, torch.float32, "gamma", (1,)),
             M, N, K, _dev(out, out.dtype, "out", (M, N)), kind, _opt(err_word, "err_word"))
-    if path == BL_PATH_AUTO:
+    if layout != BL_XQ_ROWMAJOR:
+        _check(lib().bitlinear_forward_layout(*args, int(layout), int(path), _stream(stream)),
+               "bitlinear_forward_layout")
+    elif path == BL_PATH_AUTO:
         _check(lib().bitlinear_forward(*args, _stream(stream)), "bitlinear_forward")
     else:
         _check(lib().bitlinear_forward_path(*args, int(path), _stream(stream)), "bitlinear_forward_path")
@@ -169,17 +183,18 @@ def quantize_weights(W: torch.Tensor, eps: float = 1e-5, stream=None):
     return gamma, packed
 
 
-def quantize_act(X: torch.Tensor, eps: float = 1e-5, stream=None):
+def quantize_act(X: torch.Tensor, eps: float = 1e-5, stream=None, layout=BL_XQ_ROWMAJOR):
     """(x_q [M, K] int8, s [M] fp32) of a bf16 CUDA activation matrix."""
     M, K = X.shape
     xq = torch.empty(M, K, dtype=torch.int8, device=X.device)
     s = torch.empty(M, dtype=torch.float32, device=X.device)
-    bitlinear_quantize_act(X, eps, xq, s, stream)
+    bitlinear_quantize_act(X, eps, xq, s, stream, layout)
     return xq, s
 
 
-def forward(xq, s, packed, gamma, out_dtype=torch.float32, stream=None, path=BL_PATH_AUTO, err_word=None):
+def forward(xq, s, packed, gamma, out_dtype=torch.float32, stream=None, path=BL_PATH_AUTO, err_word=None,
+            layout=BL_XQ_ROWMAJOR):
     """y [M, N] of the BitLinear forward from quantised operands."""
     out = torch.empty(xq.shape[0], packed.shape[0], dtype=out_dtype, device=xq.device)
-    bitlinear_forward(xq, s, packed, gamma, out, err_word, stream, path)
+    bitlinear_forward(xq, s, packed, gamma, out, err_word, stream, path, layout)
     return out

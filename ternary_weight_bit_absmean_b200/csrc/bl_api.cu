@@ -87,19 +87,26 @@ bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, uint8_t* pac
     return cuda_status(e);
 }
 
-bl_status bitlinear_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
-                                 float* s_out, void* stream) {
+bl_status bitlinear_quantize_act_layout(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
+                                        float* s_out, bl_xq_layout layout, void* stream) {
     if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
     if (M <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (layout != BL_XQ_ROWMAJOR && layout != BL_XQ_K16_EVENODD) return BL_ERR_INVALID_ARG;
+    if (layout == BL_XQ_K16_EVENODD && (K % 16 != 0 || K > (int64_t(1) << 30))) return BL_ERR_UNSUPPORTED_SHAPE;
     if (M > (int64_t(1) << 40) / K) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(X) || !aligned16(xq_out) || !aligned16(s_out)) return BL_ERR_MISALIGNED;
-    cudaError_t e = bl::launch_quantize_act(X, M, K, eps, xq_out, s_out, as_stream(stream));
+    cudaError_t e = bl::launch_quantize_act(X, M, K, eps, xq_out, s_out, static_cast<int>(layout), as_stream(stream));
     return cuda_status(e);
 }
 
-bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                                 int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
-                                 int32_t* err_word, bl_path path, void* stream) {
+bl_status bitlinear_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
+                                 float* s_out, void* stream) {
+    return bitlinear_quantize_act_layout(X, M, K, eps, xq_out, s_out, BL_XQ_ROWMAJOR, stream);
+}
+
+bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                                   int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                   int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
     if (xq == nullptr || s == nullptr || packed == nullptr || gamma == nullptr || out == nullptr)
         return BL_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
@@ -108,7 +115,9 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t
     if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
         path != BL_PATH_TC_2SM)
         return BL_ERR_INVALID_ARG;
+    if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD) return BL_ERR_INVALID_ARG;
     if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (xq_layout == BL_XQ_K16_EVENODD && K % 16 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
     // |acc| <= 128 K must fit in int32; sizes must fit the kernels' 32-bit indexing.
     if (K > (int64_t(1) << 31) / 128 - 1) return BL_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
@@ -118,19 +127,28 @@ bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t
     if (tc && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
     if (path == BL_PATH_AUTO) path = (M <= 16 || !k64) ? BL_PATH_GEMV : BL_PATH_TC;
     const int kind = static_cast<int>(out_dtype);
+    const int lay = static_cast<int>(xq_layout);
+    cudaStream_t st = as_stream(stream);
     cudaError_t e;
     if (path == BL_PATH_TC) {
-        e = bl::launch_gemm_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+        e = bl::launch_gemm_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (path == BL_PATH_TC_1SM) {
-        e = bl::launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+        e = bl::launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (path == BL_PATH_TC_2SM) {
-        e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, as_stream(stream));
+        e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (k64 && M <= int64_t(65535) * 16) {
-        e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, as_stream(stream));
+        e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, lay, st);
     } else {
-        e = bl::launch_gemv_generic(xq, s, packed, gamma, M, N, K, out, kind, as_stream(stream));
+        e = bl::launch_gemv_generic(xq, s, packed, gamma, M, N, K, out, kind, lay, st);
     }
     return cuda_status(e);
+}
+
+bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                                 int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                 int32_t* err_word, bl_path path, void* stream) {
+    return bitlinear_forward_layout(xq, s, packed, gamma, M, N, K, out, out_dtype, err_word, BL_XQ_ROWMAJOR, path,
+                                    stream);
 }
 
 bl_status bitlinear_forward(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,

@@ -19,9 +19,12 @@ cudaError_t launch_ternarise_pack(const float* W, int64_t numel, const float* ga
 cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packed, int32_t* err,
                               cudaStream_t stream);
 
+// Layouts of x_q (mirror bl_xq_layout).
+enum XqLayout : int { kXqRowMajor = 0, kXqEvenOdd16 = 1 };
+
 // Per-token absmax int8 activation quantisation.
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
-                                float* s, cudaStream_t stream);
+                                float* s, int layout, cudaStream_t stream);
 
 // Output kinds (mirror bl_dtype).
 enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
@@ -29,23 +32,23 @@ enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
 // Decode GEMV: register unpack + mma.sync, any M (token groups of 16), K % 64 == 0.
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
                         const float* gamma, int64_t M, int64_t N, int64_t K, void* out, int kind,
-                        cudaStream_t stream);
+                        int layout, cudaStream_t stream);
 // Plain fallback for K % 64 != 0 (one output per thread).
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
-                                int kind, cudaStream_t stream);
+                                int kind, int layout, cudaStream_t stream);
 
 // Tiled tcgen05 kind::i8 paths (K % 64 == 0): launch_gemm_tc picks between the
 // single-SM kernel (tc1) and the CTA-pair kernel (tc2).
 cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed,
                            const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
-                           int kind, int32_t* err, cudaStream_t stream);
+                           int kind, int32_t* err, int layout, cudaStream_t stream);
 cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
-                            int kind, int32_t* err, cudaStream_t stream);
+                            int kind, int32_t* err, int layout, cudaStream_t stream);
 cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
-                            int kind, int32_t* err, cudaStream_t stream);
+                            int kind, int32_t* err, int layout, cudaStream_t stream);
 
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);

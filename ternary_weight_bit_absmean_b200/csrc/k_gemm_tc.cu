@@ -98,7 +98,7 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int BT>
+template <int BT, bool EO>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
                    const TcArgs a) {
@@ -253,8 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t words[4] = {p0.x, p0.y, p0.z, p0.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    // 16 codes -> 16 int8 in the order of the x_q layout: natural, or the
+                    // even/odd k16 order (codes 0,2,4,6 | 8,..,14 | 1,3,5,7 | 9,..,15)
                     uint4 u;
-                    unpack16_natural(words[c], u.x, u.y, u.z, u.w);
+                    if constexpr (EO)
+                        unpack16_evenodd(words[c], u.x, u.y, u.z, u.w);
+                    else
+                        unpack16_natural(words[c], u.x, u.y, u.z, u.w);
                     const uint32_t chunk = static_cast<uint32_t>(4 * half + c);
                     *reinterpret_cast<uint4*>(ap + ((chunk ^ sw) << 4)) = u;
                 }
@@ -353,7 +358,7 @@ bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64
 
 namespace {
 
-template <int BT>
+template <int BT, bool EO>
 cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms, cudaStream_t stream) {
     using C = TcCfg<BT>;
     CUtensorMap tx, tp;
@@ -365,13 +370,13 @@ cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT, EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     const int grid = a.num_tiles < sms ? a.num_tiles : sms;
-    gemm_tc_kernel<BT><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
+    gemm_tc_kernel<BT, EO><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
     return cudaGetLastError();
 }
 
@@ -398,7 +403,7 @@ static int tc1_tile(int64_t M, int64_t N, int sms, int64_t* cost) {
 }
 
 cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
                             cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -409,11 +414,12 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
              0, out, kind, err};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
+    const bool eo = layout == kXqEvenOdd16;
     switch (bt) {
-        case 32: return launch_bt<32>(xq, packed, a, sms, stream);
-        case 64: return launch_bt<64>(xq, packed, a, sms, stream);
-        case 128: return launch_bt<128>(xq, packed, a, sms, stream);
-        default: return launch_bt<256>(xq, packed, a, sms, stream);
+        case 32: return eo ? launch_bt<32, true>(xq, packed, a, sms, stream) : launch_bt<32, false>(xq, packed, a, sms, stream);
+        case 64: return eo ? launch_bt<64, true>(xq, packed, a, sms, stream) : launch_bt<64, false>(xq, packed, a, sms, stream);
+        case 128: return eo ? launch_bt<128, true>(xq, packed, a, sms, stream) : launch_bt<128, false>(xq, packed, a, sms, stream);
+        default: return eo ? launch_bt<256, true>(xq, packed, a, sms, stream) : launch_bt<256, false>(xq, packed, a, sms, stream);
     }
 }
 
@@ -421,7 +427,7 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
 // it is preferred unless its coarser 256 x 256 tiles leave more waves than the
 // single-SM kernel's.
 cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                           int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                           int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
                            cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -432,8 +438,8 @@ cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* pack
     const int64_t pairs = sms / 2;
     const int64_t cost2 = (tiles2 + pairs - 1) / pairs * 512;
     if (M > 128 && cost2 <= cost1)
-        return launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
-    return launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
+        return launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err, layout, stream);
+    return launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err, layout, stream);
 }
 
 }  // namespace bl

@@ -121,6 +121,7 @@ __device__ __forceinline__ void store_row32(void* out, int kind, int64_t row_off
     }
 }
 
+template <bool EO>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
                     const Tc2Args a) {
@@ -283,8 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t words[2] = {p0.x, p0.y};
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
+                    // natural order, or the even/odd k16 order of the x_q layout
                     uint4 u;
-                    unpack16_natural(words[c], u.x, u.y, u.z, u.w);
+                    if constexpr (EO)
+                        unpack16_evenodd(words[c], u.x, u.y, u.z, u.w);
+                    else
+                        unpack16_natural(words[c], u.x, u.y, u.z, u.w);
                     const uint32_t chunk = static_cast<uint32_t>(2 * part + c);
                     *reinterpret_cast<uint4*>(bp + ((chunk ^ sw) << 4)) = u;
                 }
@@ -355,28 +360,18 @@ int gemm_tc2_clusters(int64_t M, int64_t N, int sms) {
     return static_cast<int>(tiles < pairs ? tiles : pairs);
 }
 
-cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
-                            cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    CUtensorMap tx, tp;
-    if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, kTok, true) ||
-        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kBK / 4, kFeat,
-                           false))
-        return cudaErrorInvalidValue;
+template <bool EO>
+static cudaError_t launch_tc2_eo(const CUtensorMap& tx, const CUtensorMap& tp, const Tc2Args& a, int clusters,
+                                 cudaStream_t stream) {
     static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
-    Tc2Args a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-              static_cast<int>((N + 255) / 256), static_cast<int>(((N + 255) / 256) * ((M + 255) / 256)),
-              out, kind, err};
-    const int clusters = gemm_tc2_clusters(M, N, sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -389,7 +384,26 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, tx, tp, a);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<EO>, tx, tp, a);
+}
+
+cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
+                            cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    CUtensorMap tx, tp;
+    if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, kTok, true) ||
+        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kBK / 4, kFeat,
+                           false))
+        return cudaErrorInvalidValue;
+    Tc2Args a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+              static_cast<int>((N + 255) / 256), static_cast<int>(((N + 255) / 256) * ((M + 255) / 256)),
+              out, kind, err};
+    const int clusters = gemm_tc2_clusters(M, N, sms);
+    return layout == kXqEvenOdd16 ? launch_tc2_eo<true>(tx, tp, a, clusters, stream)
+                                  : launch_tc2_eo<false>(tx, tp, a, clusters, stream);
 }
 
 }  // namespace bl

@@ -51,6 +51,7 @@ struct GemvArgs {
     void* out;
     int kind;
     uint32_t mul2, mul16;  // 2^30 and 2^16: right shifts by 2 and 16 as high-half multiplies
+    int eo;                // x_q in the even/odd k16 layout
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -187,7 +188,7 @@ __device__ __forceinline__ void gemv_step(int (&acc)[2][MT][4], uint32_t w0, uin
     }
 }
 
-template <int MT>
+template <int MT, bool EO>
 __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
     constexpr int MP = 8 * MT;  // tokens per block (padded)
     extern __shared__ __align__(16) uint8_t smem[];
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
         if (nfull > 0) load_full(bufA, 0);
         if (nfull > 1) load_full(bufB, 1);
 
-        // stage this window's activations, permuted to match the even/odd unpack
+        // stage this window's activations in the order of the even/odd unpack
         __syncthreads();
         const int groups = nch * 16;  // 16-byte groups per token row in the window
         for (int idx = threadIdx.x; idx < groups * MP; idx += kGvThreads) {
@@ -260,8 +261,10 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
             if (tok < a.M && k < kw_end)
                 v = __ldg(reinterpret_cast<const uint4*>(a.xq + tok * a.K + k));
             const int c = q >> 4, tt = (q >> 2) & 3, i = q & 3;
+            // words wanted per 16-group: {0,2,4,6}, {1,3,5,7}, {8,..,14}, {9,..,15}; the
+            // even/odd k16 layout already holds them, as words 0, 2, 1, 3
             *reinterpret_cast<uint4*>(xs + ((((c * 4 + i) * MP) + m) * 4 + tt) * 16) =
-                permute16_evenodd(v);
+                EO ? make_uint4(v.x, v.z, v.y, v.w) : permute16_evenodd(v);
         }
         __syncthreads();
 
@@ -355,7 +358,10 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t c = (b >> (2 * i)) & 3u;
-            const int xv = x[4 * j + i];
+            const int64_t k = 4 * j + i;
+            // position of element k: itself, or its slot in the even/odd k16 layout
+            const int64_t pos = a.eo ? ((k & ~int64_t(15)) | ((k & 1) * 8 + ((k >> 3) & 1) * 4 + ((k & 7) >> 1))) : k;
+            const int xv = x[pos];
             acc += c == 1u ? xv : (c == 2u ? -xv : 0);
         }
     }
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
     store_y(a.out, a.kind, idx, acc, fac);
 }
 
-template <int MT>
+template <int MT, bool EO>
 cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_blocks,
                            cudaStream_t stream) {
     constexpr int MP = 8 * MT;
@@ -375,7 +381,7 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MT, EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kWindow * MP + MP * kGvRows * static_cast<int>(sizeof(int)));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
@@ -395,13 +401,13 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, a);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<MT, EO>, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                        int64_t M, int64_t N, int64_t K, void* out, int kind,
+                        int64_t M, int64_t N, int64_t K, void* out, int kind, int layout,
                         cudaStream_t stream) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -432,15 +438,21 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
     }
     int64_t Kc = ((K + S - 1) / S + kChunk - 1) / kChunk * kChunk;
     S = (K + Kc - 1) / Kc;
-    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind, 1u << 30, 1u << 16};
-    if (MT == 1) return launch_gemv_mt<1>(a, static_cast<int>(S), row_blocks, token_blocks, stream);
-    return launch_gemv_mt<2>(a, static_cast<int>(S), row_blocks, token_blocks, stream);
+    const bool eo = layout == kXqEvenOdd16;
+    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind, 1u << 30, 1u << 16,
+               eo ? 1 : 0};
+    const int Si = static_cast<int>(S);
+    if (MT == 1) return eo ? launch_gemv_mt<1, true>(a, Si, row_blocks, token_blocks, stream)
+                           : launch_gemv_mt<1, false>(a, Si, row_blocks, token_blocks, stream);
+    return eo ? launch_gemv_mt<2, true>(a, Si, row_blocks, token_blocks, stream)
+              : launch_gemv_mt<2, false>(a, Si, row_blocks, token_blocks, stream);
 }
 
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
-                                int kind, cudaStream_t stream) {
-    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16};
+                                int kind, int layout, cudaStream_t stream) {
+    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16,
+               layout == kXqEvenOdd16 ? 1 : 0};
     const int64_t total = M * N;
     gemv_generic_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(a);
     return cudaGetLastError();

@@ -173,7 +173,7 @@ __device__ __forceinline__ uint32_t q8_bits(float x, float s) {
     return __float_as_uint(__fadd_rn(__fmul_rn(x, s), 12582912.0f));
 }
 
-// 8 bf16 (one 16-byte vector) -> 8 int8 (8 bytes).
+// 8 bf16 (one 16-byte vector) -> 8 int8 (8 bytes), in order.
 __device__ __forceinline__ uint2 quant8(uint4 v, float s) {
     uint32_t q[8];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -188,6 +188,22 @@ __device__ __forceinline__ uint2 quant8(uint4 v, float s) {
     return r;
 }
 
+// 16 bf16 (two 16-byte vectors) -> 16 int8 in the even/odd k16 layout: the group's
+// elements 0,2,4,6 | 8,10,12,14 | 1,3,5,7 | 9,11,13,15.
+__device__ __forceinline__ uint4 quant16_evenodd(uint4 a, uint4 b, float s) {
+    uint32_t q[16];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        q[2 * i] = q8_bits(__uint_as_float(w[i] << 16), s);
+        q[2 * i + 1] = q8_bits(__uint_as_float(w[i] & 0xFFFF0000u), s);
+    }
+    auto pack4 = [&](int e0, int e1, int e2, int e3) {
+        return __byte_perm(__byte_perm(q[e0], q[e1], 0x0040), __byte_perm(q[e2], q[e3], 0x0040), 0x5410);
+    };
+    return make_uint4(pack4(0, 2, 4, 6), pack4(8, 10, 12, 14), pack4(1, 3, 5, 7), pack4(9, 11, 13, 15));
+}
+
 // |x| of two bf16 at once as unsigned 16-bit lanes; for finite values the integer
 // order of |x| bit patterns is the float order.
 __device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
@@ -198,48 +214,82 @@ __device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
     return m;
 }
 
-// One group of G threads per token row; each thread keeps up to NV 16-byte vectors of
-// its row in registers between the absmax pass and the quantise pass (longer rows are
-// re-read for the remainder).  Short rows (G = 32) give each warp R rows, whose loads
-// are all issued before the first reduction.  Needs K % 8 == 0.
-template <int G, int R>
+// A unit is U 16-byte vectors of one row: U = 1 (8 elements, row-major output) or U = 2
+// (16 elements, even/odd k16 output).
+template <int U>
+struct Unit {
+    uint4 v[U];
+};
+
+template <int U>
+__device__ __forceinline__ Unit<U> load_unit(const uint4* xr, int idx) {
+    Unit<U> u;
+#pragma unroll
+    for (int i = 0; i < U; ++i) u.v[i] = __ldg(xr + U * idx + i);
+    return u;
+}
+
+template <int U>
+__device__ __forceinline__ void store_unit(uint8_t* qrow, int idx, const Unit<U>& u, float s) {
+    if constexpr (U == 1)
+        reinterpret_cast<uint2*>(qrow)[idx] = quant8(u.v[0], s);
+    else
+        reinterpret_cast<uint4*>(qrow)[idx] = quant16_evenodd(u.v[0], u.v[1], s);
+}
+
+// One group of G threads per token row; each thread keeps up to NV units of its row in
+// registers between the absmax pass and the quantise pass (longer rows are re-read for
+// the remainder).  Short rows (G = 32) give each warp R rows, whose loads are all issued
+// before the first reduction.  Needs K % (8 U) == 0.
+template <int G, int R, int U>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
-                         uint2* __restrict__ xq, float* __restrict__ s_out) {
+                         uint8_t* __restrict__ xq, float* __restrict__ s_out) {
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G * R;  // rows per block
     constexpr int WPG = G / 32;       // warps per row group
-    constexpr int NV = (R > 1) ? 4 : 8;
+    constexpr int NV = ((R > 1) ? 4 : 8) / U;
     static_assert(R == 1 || G == 32, "several rows per group only for warp groups");
     __shared__ uint32_t red[CTA / 32];
 
     const int sub = threadIdx.x / G;
     const int j = threadIdx.x % G;
-    const int nvec = K / 8;
+    const int nunit = K / (8 * U);
     const int64_t row_base = static_cast<int64_t>(blockIdx.x) * RPC + static_cast<int64_t>(sub) * R;
 
-    uint4 v[R][NV];
+    Unit<U> v[R][NV];
     uint32_t m2[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int64_t row = row_base + r;
         const bool active = row < M;
-        const uint4* xr = X + (active ? row : 0) * nvec;
+        const uint4* xr = X + (active ? row : 0) * (K / 8);
         m2[r] = 0;
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
             const int idx = j + u * G;
-            v[r][u] = (active && idx < nvec) ? __ldg(xr + idx) : make_uint4(0, 0, 0, 0);
+            if (active && idx < nunit) {
+                v[r][u] = load_unit<U>(xr, idx);
+            } else {
+#pragma unroll
+                for (int i = 0; i < U; ++i) v[r][u].v[i] = make_uint4(0, 0, 0, 0);
+            }
         }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int64_t row = row_base + r;
         const bool active = row < M;
-        const uint4* xr = X + (active ? row : 0) * nvec;
+        const uint4* xr = X + (active ? row : 0) * (K / 8);
 #pragma unroll
-        for (int u = 0; u < NV; ++u) m2[r] = absmax_vec(m2[r], v[r][u]);
-        for (int idx = j + NV * G; active && idx < nvec; idx += G) m2[r] = absmax_vec(m2[r], __ldg(xr + idx));
+        for (int u = 0; u < NV; ++u)
+#pragma unroll
+            for (int i = 0; i < U; ++i) m2[r] = absmax_vec(m2[r], v[r][u].v[i]);
+        for (int idx = j + NV * G; active && idx < nunit; idx += G) {
+            const Unit<U> t = load_unit<U>(xr, idx);
+#pragma unroll
+            for (int i = 0; i < U; ++i) m2[r] = absmax_vec(m2[r], t.v[i]);
+        }
 
         uint32_t am = max(m2[r] & 0xFFFFu, m2[r] >> 16);
         for (int off = 16; off > 0; off >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, off));
@@ -254,13 +304,13 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
         const float s = __fdiv_rn(127.0f, fmaxf(a, eps));
         if (!active) continue;
         if (j == 0) s_out[row] = s;
-        uint2* qr = xq + row * nvec;
+        uint8_t* qrow = xq + row * K;
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
             const int idx = j + u * G;
-            if (idx < nvec) qr[idx] = quant8(v[r][u], s);
+            if (idx < nunit) store_unit<U>(qrow, idx, v[r][u], s);
         }
-        for (int idx = j + NV * G; idx < nvec; idx += G) qr[idx] = quant8(__ldg(xr + idx), s);
+        for (int idx = j + NV * G; idx < nunit; idx += G) store_unit<U>(qrow, idx, load_unit<U>(xr, idx), s);
     }
 }
 
@@ -326,29 +376,37 @@ cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packe
     return cudaGetLastError();
 }
 
+template <int U>
+static void launch_act_vec(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s, cudaStream_t stream) {
+    const int nvec = K / 8;
+    if (nvec <= 32) {
+        act_quant_vec_kernel<32, 4, U><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+    } else if (nvec <= 128) {
+        act_quant_vec_kernel<32, 2, U><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+    } else if (nvec <= 256) {
+        act_quant_vec_kernel<64, 1, U><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+    } else if (nvec <= 512) {
+        act_quant_vec_kernel<128, 1, U><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+    } else if (nvec <= 1024) {
+        act_quant_vec_kernel<256, 1, U><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+    } else {
+        act_quant_vec_kernel<512, 1, U><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, K, eps, xq, s);
+    }
+}
+
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
-                                float* s, cudaStream_t stream) {
+                                float* s, int layout, cudaStream_t stream) {
+    uint8_t* q = reinterpret_cast<uint8_t*>(xq);
+    const uint4* X4 = reinterpret_cast<const uint4*>(X);
+    if (layout == kXqEvenOdd16) {  // K % 16 == 0 checked by the caller
+        launch_act_vec<2>(X4, M, static_cast<int>(K), eps, q, s, stream);
+        return cudaGetLastError();
+    }
     if (K % 8 != 0 || K > (int64_t(1) << 30)) {
         act_quant_scalar_kernel<<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X, M, K, eps, xq, s);
         return cudaGetLastError();
     }
-    const int nvec = static_cast<int>(K / 8);
-    const uint4* X4 = reinterpret_cast<const uint4*>(X);
-    uint2* q8 = reinterpret_cast<uint2*>(xq);
-    const int Ki = static_cast<int>(K);
-    if (nvec <= 32) {
-        act_quant_vec_kernel<32, 4><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    } else if (nvec <= 128) {
-        act_quant_vec_kernel<32, 2><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    } else if (nvec <= 256) {
-        act_quant_vec_kernel<64, 1><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    } else if (nvec <= 512) {
-        act_quant_vec_kernel<128, 1><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    } else if (nvec <= 1024) {
-        act_quant_vec_kernel<256, 1><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    } else {
-        act_quant_vec_kernel<512, 1><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, Ki, eps, q8, s);
-    }
+    launch_act_vec<1>(X4, M, static_cast<int>(K), eps, q, s, stream);
     return cudaGetLastError();
 }
 

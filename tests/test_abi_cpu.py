@@ -106,6 +106,12 @@ def test_other_entry_points_validation(L):
         assert path(FAKE, FAKE, FAKE, FAKE, 40, 8, 96, FAKE, 0, None, p, None) == SHAPE
     assert path(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 9, None) == INVALID
     assert L.bitlinear_status_string(3) == b"BL_ERR_MISALIGNED"
+    lay = L.bitlinear_forward_layout
+    assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 72, FAKE, 0, None, 1, 0, None) == SHAPE   # even/odd needs K % 16
+    assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 5, 0, None) == INVALID
+    qa = L.bitlinear_quantize_act_layout
+    assert qa(FAKE, 4, 24, 1e-5, FAKE, FAKE, 1, None) == SHAPE
+    assert qa(FAKE, 4, 32, 1e-5, FAKE, FAKE, 2, None) == INVALID
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

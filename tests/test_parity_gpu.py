@@ -300,3 +300,60 @@ def test_workload_sizes(name):
             y = B.forward(xq, s, pk, gamma, torch.float32).cpu().numpy()
             assert np.array_equal(acc[rows], acc_ref), (name, pname, M)
             assert_float_close(y[rows], y_ref, "%s %s M=%d" % (name, pname, M))
+
+
+# ------------------------------------------------ x_q in the even/odd k16 layout --
+
+def evenodd_positions(K):
+    """Byte position of every element k in the even/odd k16 layout, built from the
+    layout's definition: inside each group of 16 the element order is
+    0,2,4,6, 8,10,12,14, 1,3,5,7, 9,11,13,15."""
+    order = [0, 2, 4, 6, 8, 10, 12, 14, 1, 3, 5, 7, 9, 11, 13, 15]
+    pos = np.empty(K, dtype=np.int64)
+    for q in range(K // 16):
+        for p, e in enumerate(order):
+            pos[16 * q + e] = 16 * q + p
+    return pos
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (5, 1536), (33, 4096), (4096, 1536), (3, 28672), (64, 208)])
+def test_quantize_act_evenodd_layout(M, K):
+    X = synth.activations(M, K, seed=M + 11 * K)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    xq = guarded_empty((M, K), torch.int8)
+    s = guarded_empty((M,), torch.float32)
+    B.bitlinear_quantize_act(X.to(DEV), EPS, xq, s, layout=B.BL_XQ_K16_EVENODD)
+    sync()
+    check_guard(xq)
+    check_guard(s)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    got = xq.cpu().numpy()
+    assert np.array_equal(got[:, evenodd_positions(K)], xq_ref)
+
+
+EO_CASES = [(1, 300, 256, B.BL_PATH_GEMV), (16, 4096, 1536, B.BL_PATH_GEMV), (9, 640, 4160, B.BL_PATH_GEMV),
+            (40, 200, 256, B.BL_PATH_GEMV), (5, 64, 208, B.BL_PATH_AUTO), (100, 300, 192, B.BL_PATH_TC_1SM),
+            (513, 4096, 1536, B.BL_PATH_TC_1SM), (300, 200, 320, B.BL_PATH_TC_2SM),
+            (1000, 1536, 4096, B.BL_PATH_TC_2SM), (4096, 1536, 1536, B.BL_PATH_TC)]
+
+
+@pytest.mark.parametrize("M,N,K,path", EO_CASES)
+def test_forward_evenodd_layout(M, N, K, path):
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=M + N + 7 * K, zero_row=True)
+    acc_ref = oracle.forward(xq_ref, s_ref, packed_ref, g_ref, K, oracle.OUT_I32)
+    y_ref = oracle.dequant(acc_ref, s_ref, g_ref)
+    xq_eo = np.empty_like(xq_ref)
+    xq_eo[:, evenodd_positions(K)] = xq_ref
+    xq = torch.from_numpy(xq_eo).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    for dt in (torch.int32, torch.float32):
+        out = guarded_empty((M, N), dt)
+        B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=B.BL_XQ_K16_EVENODD)
+        sync()
+        check_guard(out)
+        if dt == torch.int32:
+            assert np.array_equal(out.cpu().numpy(), acc_ref)
+        else:
+            assert_float_close(out.cpu().numpy(), y_ref, "evenodd fp32")
