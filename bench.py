@@ -59,7 +59,9 @@ def parse():
     p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2"], default="auto")
     p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
     p.add_argument("--iters", type=int, default=20)
-    p.add_argument("--xq-layout", choices=["evenodd", "rowmajor"], default="evenodd",
+    p.add_argument("--sweep", choices=["llama3b", "llama70b", "grid"], default=None,
+                   help="time the forward over a family of shapes (one JSON line per shape)")
+    p.add_argument("--xq-layout", choices=["stride4", "evenodd", "rowmajor"], default="stride4",
                    help="storage order of the int8 activations between quantize_act and forward")
     return p.parse_args()
 
@@ -82,6 +84,10 @@ def workload():
 
 def fwd_ops(projs, Ms):
     return sum(2 * M * N * K for M in Ms for (_, N, K) in projs)
+
+
+def xq_layout_of(B, name):
+    return {"rowmajor": B.BL_XQ_ROWMAJOR, "evenodd": B.BL_XQ_K16_EVENODD, "stride4": B.BL_XQ_K16_STRIDE4}[name]
 
 
 def rank_seed(pi, M, rank):
@@ -199,7 +205,7 @@ def run_ours(args):
     B.lib()
 
     projs, Ms, ofrac = workload()
-    XQ_LAYOUT = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
+    XQ_LAYOUT = xq_layout_of(B, args.xq_layout)
     # inputs: weights are the same model replica on every rank; tokens differ per rank
     W = [synth.weight(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
     C = [synth.codes(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
@@ -478,7 +484,7 @@ def run_single(args):
         out = torch.empty(M, N, dtype=odt, device=dev)
         path = {"auto": B.BL_PATH_AUTO, "gemv": B.BL_PATH_GEMV, "tc": B.BL_PATH_TC, "tc1": B.BL_PATH_TC_1SM,
                 "tc2": B.BL_PATH_TC_2SM}[args.path]
-        lay = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
+        lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=lay)
         ops = 2 * M * N * K
         nbytes = N * K // 4 + M * K + 4 * M + M * N * out.element_size()
@@ -486,7 +492,7 @@ def run_single(args):
         X = torch.randn(M, K, device=dev).to(torch.bfloat16)
         xq = torch.empty(M, K, dtype=torch.int8, device=dev)
         s = torch.empty(M, device=dev)
-        lay = B.BL_XQ_K16_EVENODD if args.xq_layout == "evenodd" else B.BL_XQ_ROWMAJOR
+        lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_quantize_act(X, EPS, xq, s, layout=lay)
         ops, nbytes = 0, 3 * M * K + 4 * M
     elif args.single == "quantize_weights":
@@ -501,18 +507,7 @@ def run_single(args):
         packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
         fn = lambda: B.bitlinear_pack(c, packed)
         ops, nbytes = 0, N * K + N * K // 4
-    for _ in range(3):
-        fn()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ts = []
-    for _ in range(args.iters):
-        flusher.flush()
-        e0.record()
-        fn()
-        e1.record()
-        torch.cuda.synchronize()
-        ts.append(e0.elapsed_time(e1))
+    ts = time_calls(fn, flusher, args.iters)
     t = statistics.median(ts) * 1e-3
     rec = {"single": args.single, "M": M, "N": N, "K": K, "path": args.path, "out_dtype": args.out_dtype,
            "xq_layout": args.xq_layout,
@@ -525,9 +520,90 @@ def run_single(args):
     print(json.dumps(rec), flush=True)
 
 
+def time_calls(fn, flusher, iters):
+    """Milliseconds of each of `iters` calls of fn, CUDA events on the current stream,
+    L2 flushed before each call (outside the events), after 3 untimed calls."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(iters):
+        flusher.flush()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return ts
+
+
+def sweep_shapes(name):
+    """(M, N, K, tag) of a sweep: the projections of one LLaMA-3B- or LLaMA-70B-shaped
+    layer at their token counts, or the K, N grid of square and rectangular GEMMs."""
+    from ternary_weight_bit_absmean_b200 import synth
+    if name == "grid":
+        return [(M, N, K, "grid") for K in synth.SWEEP_KN for N in synth.SWEEP_KN for M in synth.SWEEP_M]
+    spec = synth.WORKLOADS[name]
+    seen, out = set(), []
+    for pname, N, K in spec["proj"]:
+        for M in spec["M"]:
+            if (M, N, K) not in seen:
+                seen.add((M, N, K))
+                out.append((M, N, K, pname))
+    return out
+
+
+def run_sweep(args):
+    """The forward (automatic dispatch, bf16 y) on every shape of a sweep, each timed
+    alone with L2 flushed: one JSON line per shape with TOPS, weight GB/s and the
+    fraction of the roofline of its regime (HBM for M <= 16, int8 tensor otherwise)."""
+    import torch
+
+    from ternary_weight_bit_absmean_b200 import binding as B
+    from ternary_weight_bit_absmean_b200 import build_lib, synth
+
+    build_lib.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flusher = L2Flusher(dev)
+    P = peaks()
+    lay = xq_layout_of(B, args.xq_layout)
+    packed_of = {}
+    for M, N, K, tag in sweep_shapes(args.sweep):
+        X = synth.activations(M, K, seed=M + K, outlier_frac=0.01).to(dev)
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        s = torch.empty(M, device=dev)
+        B.bitlinear_quantize_act(X, EPS, xq, s, layout=lay)
+        if (N, K) not in packed_of:
+            packed_of.clear()
+            c = synth.codes(N, K, seed=N + K).to(dev)
+            packed_of[N, K] = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+            B.bitlinear_pack(c, packed_of[N, K])
+            del c
+        packed = packed_of[N, K]
+        gamma = torch.tensor([0.02], device=dev)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ts = time_calls(lambda: B.bitlinear_forward(xq, s, packed, gamma, out, layout=lay), flusher, args.iters)
+        t = statistics.median(ts) * 1e-3
+        ops = 2 * M * N * K
+        nbytes = N * K // 4 + M * K + 4 * M + 2 * M * N
+        rec = {"sweep": args.sweep, "tag": tag, "M": M, "N": N, "K": K, "xq_layout": args.xq_layout,
+               "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
+               "tops": round(ops / t / 1e12, 2), "weight_gbs": round((N * K // 4) / t / 1e9, 1),
+               "hbm_frac": round(nbytes / t / 1e9 / P["hbm_gbs"], 4),
+               "int8_frac": round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4),
+               "regime": "hbm" if M <= 16 else "tensor"}
+        print(json.dumps(rec), flush=True)
+        del X, xq, s, out
+
+
 def main():
     args = parse()
-    if args.single:
+    if args.sweep:
+        run_sweep(args)
+    elif args.single:
         run_single(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -91,11 +91,17 @@ typedef enum {
  *                      (k = 16q + e) the bytes hold the elements in the order
  *                      e = 0,2,4,6, 8,10,12,14, 1,3,5,7, 9,11,13,15 (element e sits at
  *                      byte 16q + 8(e%2) + 4(e/8) + (e%8)/2).  The values are the same;
- *                      this order matches the cheaper unpack of the packed weights, so
- *                      the forward runs faster on it. */
+ *                      this order matches a cheaper unpack of the packed weights, so
+ *                      the forward runs faster on it.
+ *   BL_XQ_K16_STRIDE4  K % 16 == 0; inside every group of 16 consecutive elements the
+ *                      bytes hold e = 0,4,8,12, 1,5,9,13, 2,6,10,14, 3,7,11,15 (element e
+ *                      sits at byte 16q + 4(e%4) + e/4).  This order matches the unpack
+ *                      with the fewest integer instructions, which the fastest decode
+ *                      and prefill kernels use. */
 typedef enum {
     BL_XQ_ROWMAJOR = 0,
-    BL_XQ_K16_EVENODD = 1
+    BL_XQ_K16_EVENODD = 1,
+    BL_XQ_K16_STRIDE4 = 2
 } bl_xq_layout;
 
 /* Bytes of device workspace bitlinear_quantize_weights needs for an [N, K] matrix
@@ -146,7 +152,7 @@ BL_API bl_status bitlinear_quantize_act(const uint16_t *X, int64_t M, int64_t K,
                                  int8_t *xq_out, float *s_out, void *stream);
 
 /* bitlinear_quantize_act writing x_q in the given layout (see bl_xq_layout).
- * BL_XQ_K16_EVENODD needs K % 16 == 0 (else BL_ERR_UNSUPPORTED_SHAPE). */
+ * The k16 layouts need K % 16 == 0 and K <= 2^30 (else BL_ERR_UNSUPPORTED_SHAPE). */
 BL_API bl_status bitlinear_quantize_act_layout(const uint16_t *X, int64_t M, int64_t K, float eps,
                                                int8_t *xq_out, float *s_out, bl_xq_layout layout,
                                                void *stream);
@@ -199,7 +205,9 @@ BL_API bl_status bitlinear_quantize_weights_noalloc(const float *W, int64_t N, i
                                                     void *stream);
 
 /* bitlinear_forward_path reading x_q stored in the given layout (see bl_xq_layout);
- * the result is the same for either layout. */
+ * the result is the same for every layout.  The k16 layouts need K % 16 == 0.  With
+ * BL_XQ_K16_STRIDE4 the tensor-core paths need K <= 2^17 (BL_PATH_AUTO runs the GEMV
+ * above that; a forced BL_PATH_TC* returns BL_ERR_UNSUPPORTED_SHAPE). */
 BL_API bl_status bitlinear_forward_layout(const int8_t *xq, const float *s, const uint8_t *packed,
                                           const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
                                           bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,

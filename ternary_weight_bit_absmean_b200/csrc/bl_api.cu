@@ -91,8 +91,9 @@ bl_status bitlinear_quantize_act_layout(const uint16_t* X, int64_t M, int64_t K,
                                         float* s_out, bl_xq_layout layout, void* stream) {
     if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
     if (M <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
-    if (layout != BL_XQ_ROWMAJOR && layout != BL_XQ_K16_EVENODD) return BL_ERR_INVALID_ARG;
-    if (layout == BL_XQ_K16_EVENODD && (K % 16 != 0 || K > (int64_t(1) << 30))) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (layout != BL_XQ_ROWMAJOR && layout != BL_XQ_K16_EVENODD && layout != BL_XQ_K16_STRIDE4)
+        return BL_ERR_INVALID_ARG;
+    if (layout != BL_XQ_ROWMAJOR && (K % 16 != 0 || K > (int64_t(1) << 30))) return BL_ERR_UNSUPPORTED_SHAPE;
     if (M > (int64_t(1) << 40) / K) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(X) || !aligned16(xq_out) || !aligned16(s_out)) return BL_ERR_MISALIGNED;
     cudaError_t e = bl::launch_quantize_act(X, M, K, eps, xq_out, s_out, static_cast<int>(layout), as_stream(stream));
@@ -115,9 +116,10 @@ bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8
     if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
         path != BL_PATH_TC_2SM)
         return BL_ERR_INVALID_ARG;
-    if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD) return BL_ERR_INVALID_ARG;
+    if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD && xq_layout != BL_XQ_K16_STRIDE4)
+        return BL_ERR_INVALID_ARG;
     if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
-    if (xq_layout == BL_XQ_K16_EVENODD && K % 16 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (xq_layout != BL_XQ_ROWMAJOR && K % 16 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
     // |acc| <= 128 K must fit in int32; sizes must fit the kernels' 32-bit indexing.
     if (K > (int64_t(1) << 31) / 128 - 1) return BL_ERR_UNSUPPORTED_SHAPE;
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
@@ -125,7 +127,10 @@ bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8
     const bool k64 = (K % 64) == 0;
     const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM;
     if (tc && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
-    if (path == BL_PATH_AUTO) path = (M <= 16 || !k64) ? BL_PATH_GEMV : BL_PATH_TC;
+    // the tensor-core kernels expand stride-4 codes as 64 * code: 64 * 128 * K must fit
+    const bool s4_big = xq_layout == BL_XQ_K16_STRIDE4 && K > (int64_t(1) << 17);
+    if (tc && s4_big) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (path == BL_PATH_AUTO) path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : BL_PATH_TC;
     const int kind = static_cast<int>(out_dtype);
     const int lay = static_cast<int>(xq_layout);
     cudaStream_t st = as_stream(stream);
@@ -137,7 +142,7 @@ bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8
     } else if (path == BL_PATH_TC_2SM) {
         e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (k64 && M <= int64_t(65535) * 16) {
-        e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, lay, st);
+        e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else {
         e = bl::launch_gemv_generic(xq, s, packed, gamma, M, N, K, out, kind, lay, st);
     }

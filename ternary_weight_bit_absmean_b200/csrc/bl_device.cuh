@@ -109,6 +109,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// 4-D tiled bulk tensor load global -> shared::cta (c0 innermost).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (the tensor core reads its operands through it).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -357,6 +367,46 @@ __device__ __forceinline__ void unpack16_evenodd_fma(uint32_t p, uint32_t mul2, 
     e1 = __byte_perm(kCodeTable, 0u, __umulhi(sa, mul16));
     o0 = __byte_perm(kCodeTable, 0u, sb);
     o1 = __byte_perm(kCodeTable, 0u, __umulhi(sb, mul16));
+}
+
+// Runtime multipliers of the stride-4 unpack: passed in as values so that the shifts
+// stay multiplies (FMA pipe) and leave the integer ALU pipe to the logic ops.
+struct S4Mul {
+    uint32_t hi1;                // 2^31: a right shift by 1 as a high-half multiply
+    uint32_t two, m4, m16, m64;  // left shifts by 1, 2, 4, 6
+};
+__host__ __device__ constexpr S4Mul s4_mul() { return S4Mul{1u << 31, 2u, 4u, 16u, 64u}; }
+
+// PTX of the stride-4 unpack of one packed word W (16 codes) into O0..O3, with scratch
+// registers ta, tx, ty, tv, tt; HI1, TWO, M4, M16, M64 name the operands holding the
+// S4Mul values.  The fields are first rewritten as 2-bit two's complement (00 -> 00,
+// 01 -> 01, 10 -> 11, the unused 11 -> 00): low bit l ^ h, high bit h & ~l, from two
+// 3-input logic ops and one multiply-add; output word i is then the word shifted left by
+// 6 - 2i and masked to bits 6..7 of every byte.  Byte j of Oi is 64 * code(4j + i).
+#define BL_S4_UNPACK(W, O0, O1, O2, O3, HI1, TWO, M4, M16, M64)                     \
+    "mul.hi.u32 ta, " W ", " HI1 ";\n\t"                                           \
+    "lop3.b32 tx, " W ", ta, 0x55555555, 0x28;\n\t" /* (w ^ (w >> 1)) & 0x55.. */  \
+    "lop3.b32 ty, ta, " W ", 0x55555555, 0x20;\n\t" /* (w >> 1) & ~w & 0x55.. */   \
+    "mad.lo.u32 tv, ty, " TWO ", tx;\n\t"                                          \
+    "and.b32 " O3 ", tv, 0xC0C0C0C0;\n\t"                                          \
+    "mul.lo.u32 tt, tv, " M4 ";\n\t"                                               \
+    "and.b32 " O2 ", tt, 0xC0C0C0C0;\n\t"                                          \
+    "mul.lo.u32 tt, tv, " M16 ";\n\t"                                              \
+    "and.b32 " O1 ", tt, 0xC0C0C0C0;\n\t"                                          \
+    "mul.lo.u32 tt, tv, " M64 ";\n\t"                                              \
+    "and.b32 " O0 ", tt, 0xC0C0C0C0;\n\t"
+
+// Unpack 16 codes into 16 int8 equal to 64 * code, in stride-4 order: o0 = codes
+// {0,4,8,12}, o1 = {1,5,9,13}, o2 = {2,6,10,14}, o3 = {3,7,11,15}.  Matched against
+// activations in the same order, the integer dot products come out 64 times the true
+// ones (exact while they fit in int32), and an arithmetic shift right by 6 restores them.
+__device__ __forceinline__ void unpack16_stride4_x64(uint32_t p, const S4Mul& k, uint32_t& o0, uint32_t& o1,
+                                                     uint32_t& o2, uint32_t& o3) {
+    asm("{\n\t.reg .b32 ta, tx, ty, tv, tt;\n\t"
+        BL_S4_UNPACK("%4", "%0", "%1", "%2", "%3", "%5", "%6", "%7", "%8", "%9")
+        "}\n"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(p), "r"(k.hi1), "r"(k.two), "r"(k.m4), "r"(k.m16), "r"(k.m64));
 }
 
 // The matching permutation of 16 activation bytes (v = bytes 0..15 little-endian):

@@ -20,7 +20,7 @@ cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packe
                               cudaStream_t stream);
 
 // Layouts of x_q (mirror bl_xq_layout).
-enum XqLayout : int { kXqRowMajor = 0, kXqEvenOdd16 = 1 };
+enum XqLayout : int { kXqRowMajor = 0, kXqEvenOdd16 = 1, kXqStride4K16 = 2 };
 
 // Per-token absmax int8 activation quantisation.
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
@@ -30,9 +30,15 @@ cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float e
 enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
 
 // Decode GEMV: register unpack + mma.sync, any M (token groups of 16), K % 64 == 0.
+// With x_q in the stride-4 k16 layout and a shape gemv_tma_applicable accepts, it runs
+// the persistent TMA-fed kernel (k_gemv_tma.cu).
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
                         const float* gamma, int64_t M, int64_t N, int64_t K, void* out, int kind,
-                        int layout, cudaStream_t stream);
+                        int32_t* err, int layout, cudaStream_t stream);
+bool gemv_tma_applicable(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
+                            cudaStream_t stream);
 // Plain fallback for K % 64 != 0 (one output per thread).
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,

@@ -75,6 +75,7 @@ struct TcArgs {
     void* out;
     int kind;
     int32_t* err;
+    S4Mul mul;
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -98,7 +99,7 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-template <int BT, bool EO>
+template <int BT, int LAY>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
                    const TcArgs a) {
@@ -253,11 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t words[4] = {p0.x, p0.y, p0.z, p0.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    // 16 codes -> 16 int8 in the order of the x_q layout: natural, or the
-                    // even/odd k16 order (codes 0,2,4,6 | 8,..,14 | 1,3,5,7 | 9,..,15)
+                    // 16 codes -> 16 int8 in the order of the x_q layout: natural, the
+                    // even/odd k16 order (codes 0,2,4,6 | 8,..,14 | 1,3,5,7 | 9,..,15) or
+                    // the stride-4 k16 order (0,4,8,12 | 1,5,9,13 | ..), the last as
+                    // 64 * code
                     uint4 u;
-                    if constexpr (EO)
+                    if constexpr (LAY == kXqEvenOdd16)
                         unpack16_evenodd(words[c], u.x, u.y, u.z, u.w);
+                    else if constexpr (LAY == kXqStride4K16)
+                        unpack16_stride4_x64(words[c], a.mul, u.x, u.y, u.z, u.w);
                     else
                         unpack16_natural(words[c], u.x, u.y, u.z, u.w);
                     const uint32_t chunk = static_cast<uint32_t>(4 * half + c);
@@ -274,6 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // -------------------------------------------------------------- epilogue --
+        // the stride-4 unpack feeds 64 * code: its sums are exact multiples of 64
+        constexpr int kAccShift = LAY == kXqStride4K16 ? 6 : 0;
         const int q = warp & 3;                   // TMEM lane quarter this warp may access
         const int first = 32 * ((warp - kWarpEpi) >> 2);  // this warp's first column chunk
         const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
@@ -304,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float fj = __shfl_sync(0xffffffffu, fac, j);
                     const int tok = t0 + c0 + j;
                     if (tok < a.M && row_ok)
-                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row, static_cast<int>(r[j]), fj);
+                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
+                                static_cast<int>(r[j]) >> kAccShift, fj);
                 }
             }
             tc_fence_before();
@@ -356,9 +364,30 @@ bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// uint8 tensor map of any rank (<= 5): dims[0] is the contiguous dimension, strides[i]
+// the byte stride of dims[i + 1].  The strides need not grow with i, so a box can gather
+// a permutation of the tensor's dimensions into shared memory.
+bool encode_tmap_u8(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
+                    const uint32_t* box, bool swizzle128) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
+    if (fn == nullptr || rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t b[5], estr[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        estr[i] = 1;
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), d, st, b,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
-template <int BT, bool EO>
+template <int BT, int LAY>
 cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms, cudaStream_t stream) {
     using C = TcCfg<BT>;
     CUtensorMap tx, tp;
@@ -370,17 +399,28 @@ cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT, EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     const int grid = a.num_tiles < sms ? a.num_tiles : sms;
-    gemm_tc_kernel<BT, EO><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
+    gemm_tc_kernel<BT, LAY><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+template <int LAY>
+static cudaError_t launch_bt_layout(int bt, const int8_t* xq, const uint8_t* packed, const TcArgs& a, int sms,
+                                   cudaStream_t stream) {
+    switch (bt) {
+        case 32: return launch_bt<32, LAY>(xq, packed, a, sms, stream);
+        case 64: return launch_bt<64, LAY>(xq, packed, a, sms, stream);
+        case 128: return launch_bt<128, LAY>(xq, packed, a, sms, stream);
+        default: return launch_bt<256, LAY>(xq, packed, a, sms, stream);
+    }
+}
 
 // Token tile of the single-SM kernel and its cost (cycles of the busiest SM, up to a
 // constant): a 128-byte K stage costs ~2 BT cycles of MMA at peak but never less than a
@@ -412,14 +452,12 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     int64_t cost = 0;
     const int bt = tc1_tile(M, N, sms, &cost);
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
-             0, out, kind, err};
+             0, out, kind, err, s4_mul()};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
-    const bool eo = layout == kXqEvenOdd16;
-    switch (bt) {
-        case 32: return eo ? launch_bt<32, true>(xq, packed, a, sms, stream) : launch_bt<32, false>(xq, packed, a, sms, stream);
-        case 64: return eo ? launch_bt<64, true>(xq, packed, a, sms, stream) : launch_bt<64, false>(xq, packed, a, sms, stream);
-        case 128: return eo ? launch_bt<128, true>(xq, packed, a, sms, stream) : launch_bt<128, false>(xq, packed, a, sms, stream);
-        default: return eo ? launch_bt<256, true>(xq, packed, a, sms, stream) : launch_bt<256, false>(xq, packed, a, sms, stream);
+    switch (layout) {
+        case kXqEvenOdd16: return launch_bt_layout<kXqEvenOdd16>(bt, xq, packed, a, sms, stream);
+        case kXqStride4K16: return launch_bt_layout<kXqStride4K16>(bt, xq, packed, a, sms, stream);
+        default: return launch_bt_layout<kXqRowMajor>(bt, xq, packed, a, sms, stream);
     }
 }
 

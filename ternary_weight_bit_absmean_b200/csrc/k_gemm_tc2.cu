@@ -62,6 +62,7 @@ struct Tc2Args {
     void* out;
     int kind;
     int32_t* err;
+    S4Mul mul;
 };
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -121,7 +122,7 @@ __device__ __forceinline__ void store_row32(void* out, int kind, int64_t row_off
     }
 }
 
-template <bool EO>
+template <int LAY>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
                     const Tc2Args a) {
@@ -284,10 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t words[2] = {p0.x, p0.y};
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    // natural order, or the even/odd k16 order of the x_q layout
+                    // natural order, or the even/odd or stride-4 k16 order of the x_q
+                    // layout (the last as 64 * code)
                     uint4 u;
-                    if constexpr (EO)
+                    if constexpr (LAY == kXqEvenOdd16)
                         unpack16_evenodd(words[c], u.x, u.y, u.z, u.w);
+                    else if constexpr (LAY == kXqStride4K16)
+                        unpack16_stride4_x64(words[c], a.mul, u.x, u.y, u.z, u.w);
                     else
                         unpack16_natural(words[c], u.x, u.y, u.z, u.w);
                     const uint32_t chunk = static_cast<uint32_t>(2 * part + c);
@@ -327,6 +331,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        static_cast<uint32_t>(buf * 2 * kFeat + c0),
                                    r);
                 tmem_ld_wait();
+                if constexpr (LAY == kXqStride4K16) {
+                    // the stride-4 unpack feeds 64 * code: the sums are exact multiples of 64
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) >> 6);
+                }
                 if (tok_ok && n0 + c0 < a.N) store_row32(a.out, a.kind, row_off, n0 + c0, a.N, r, fac, vec_ok);
             }
             tc_fence_before();
@@ -360,14 +369,14 @@ int gemm_tc2_clusters(int64_t M, int64_t N, int sms) {
     return static_cast<int>(tiles < pairs ? tiles : pairs);
 }
 
-template <bool EO>
-static cudaError_t launch_tc2_eo(const CUtensorMap& tx, const CUtensorMap& tp, const Tc2Args& a, int clusters,
+template <int LAY>
+static cudaError_t launch_tc2_layout(const CUtensorMap& tx, const CUtensorMap& tp, const Tc2Args& a, int clusters,
                                  cudaStream_t stream) {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
@@ -384,7 +393,7 @@ static cudaError_t launch_tc2_eo(const CUtensorMap& tx, const CUtensorMap& tp, c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<EO>, tx, tp, a);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<LAY>, tx, tp, a);
 }
 
 cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
@@ -400,10 +409,13 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
         return cudaErrorInvalidValue;
     Tc2Args a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
               static_cast<int>((N + 255) / 256), static_cast<int>(((N + 255) / 256) * ((M + 255) / 256)),
-              out, kind, err};
+              out, kind, err, s4_mul()};
     const int clusters = gemm_tc2_clusters(M, N, sms);
-    return layout == kXqEvenOdd16 ? launch_tc2_eo<true>(tx, tp, a, clusters, stream)
-                                  : launch_tc2_eo<false>(tx, tp, a, clusters, stream);
+    switch (layout) {
+        case kXqEvenOdd16: return launch_tc2_layout<kXqEvenOdd16>(tx, tp, a, clusters, stream);
+        case kXqStride4K16: return launch_tc2_layout<kXqStride4K16>(tx, tp, a, clusters, stream);
+        default: return launch_tc2_layout<kXqRowMajor>(tx, tp, a, clusters, stream);
+    }
 }
 
 }  // namespace bl

@@ -51,7 +51,7 @@ struct GemvArgs {
     void* out;
     int kind;
     uint32_t mul2, mul16;  // 2^30 and 2^16: right shifts by 2 and 16 as high-half multiplies
-    int eo;                // x_q in the even/odd k16 layout
+    int layout;            // XqLayout of x_q
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -188,7 +188,7 @@ __device__ __forceinline__ void gemv_step(int (&acc)[2][MT][4], uint32_t w0, uin
     }
 }
 
-template <int MT, bool EO>
+template <int MT, int LAY>
 __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
     constexpr int MP = 8 * MT;  // tokens per block (padded)
     extern __shared__ __align__(16) uint8_t smem[];
@@ -262,9 +262,18 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
                 v = __ldg(reinterpret_cast<const uint4*>(a.xq + tok * a.K + k));
             const int c = q >> 4, tt = (q >> 2) & 3, i = q & 3;
             // words wanted per 16-group: {0,2,4,6}, {1,3,5,7}, {8,..,14}, {9,..,15}; the
-            // even/odd k16 layout already holds them, as words 0, 2, 1, 3
-            *reinterpret_cast<uint4*>(xs + ((((c * 4 + i) * MP) + m) * 4 + tt) * 16) =
-                EO ? make_uint4(v.x, v.z, v.y, v.w) : permute16_evenodd(v);
+            // even/odd k16 layout already holds them, as words 0, 2, 1, 3; the stride-4
+            // layout holds {0,4,8,12}, {1,5,9,13}, {2,6,10,14}, {3,7,11,15}
+            uint4 o;
+            if constexpr (LAY == kXqEvenOdd16) {
+                o = make_uint4(v.x, v.z, v.y, v.w);
+            } else if constexpr (LAY == kXqStride4K16) {
+                o = make_uint4(__byte_perm(v.x, v.z, 0x5140), __byte_perm(v.y, v.w, 0x5140),
+                               __byte_perm(v.x, v.z, 0x7362), __byte_perm(v.y, v.w, 0x7362));
+            } else {
+                o = permute16_evenodd(v);
+            }
+            *reinterpret_cast<uint4*>(xs + ((((c * 4 + i) * MP) + m) * 4 + tt) * 16) = o;
         }
         __syncthreads();
 
@@ -359,8 +368,12 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
         for (int i = 0; i < 4; ++i) {
             const uint32_t c = (b >> (2 * i)) & 3u;
             const int64_t k = 4 * j + i;
-            // position of element k: itself, or its slot in the even/odd k16 layout
-            const int64_t pos = a.eo ? ((k & ~int64_t(15)) | ((k & 1) * 8 + ((k >> 3) & 1) * 4 + ((k & 7) >> 1))) : k;
+            // position of element k: itself, or its slot in a k16 layout
+            int64_t pos = k;
+            if (a.layout == kXqEvenOdd16)
+                pos = (k & ~int64_t(15)) | ((k & 1) * 8 + ((k >> 3) & 1) * 4 + ((k & 7) >> 1));
+            else if (a.layout == kXqStride4K16)
+                pos = (k & ~int64_t(15)) | ((k & 3) * 4 + ((k & 15) >> 2));
             const int xv = x[pos];
             acc += c == 1u ? xv : (c == 2u ? -xv : 0);
         }
@@ -369,7 +382,7 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
     store_y(a.out, a.kind, idx, acc, fac);
 }
 
-template <int MT, bool EO>
+template <int MT, int LAY>
 cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_blocks,
                            cudaStream_t stream) {
     constexpr int MP = 8 * MT;
@@ -381,7 +394,7 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MT, EO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kWindow * MP + MP * kGvRows * static_cast<int>(sizeof(int)));
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
@@ -401,14 +414,16 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<MT, EO>, a);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<MT, LAY>, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                        int64_t M, int64_t N, int64_t K, void* out, int kind, int layout,
+                        int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
                         cudaStream_t stream) {
+    if (layout == kXqStride4K16 && gemv_tma_applicable(M, N, K))
+        return launch_gemv_tma(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -438,21 +453,24 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
     }
     int64_t Kc = ((K + S - 1) / S + kChunk - 1) / kChunk * kChunk;
     S = (K + Kc - 1) / Kc;
-    const bool eo = layout == kXqEvenOdd16;
     GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind, 1u << 30, 1u << 16,
-               eo ? 1 : 0};
+               layout};
     const int Si = static_cast<int>(S);
-    if (MT == 1) return eo ? launch_gemv_mt<1, true>(a, Si, row_blocks, token_blocks, stream)
-                           : launch_gemv_mt<1, false>(a, Si, row_blocks, token_blocks, stream);
-    return eo ? launch_gemv_mt<2, true>(a, Si, row_blocks, token_blocks, stream)
-              : launch_gemv_mt<2, false>(a, Si, row_blocks, token_blocks, stream);
+    if (MT == 1) {
+        if (layout == kXqEvenOdd16) return launch_gemv_mt<1, kXqEvenOdd16>(a, Si, row_blocks, token_blocks, stream);
+        if (layout == kXqStride4K16) return launch_gemv_mt<1, kXqStride4K16>(a, Si, row_blocks, token_blocks, stream);
+        return launch_gemv_mt<1, kXqRowMajor>(a, Si, row_blocks, token_blocks, stream);
+    }
+    if (layout == kXqEvenOdd16) return launch_gemv_mt<2, kXqEvenOdd16>(a, Si, row_blocks, token_blocks, stream);
+    if (layout == kXqStride4K16) return launch_gemv_mt<2, kXqStride4K16>(a, Si, row_blocks, token_blocks, stream);
+    return launch_gemv_mt<2, kXqRowMajor>(a, Si, row_blocks, token_blocks, stream);
 }
 
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                                 int kind, int layout, cudaStream_t stream) {
     GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16,
-               layout == kXqEvenOdd16 ? 1 : 0};
+               layout};
     const int64_t total = M * N;
     gemv_generic_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(a);
     return cudaGetLastError();

@@ -204,6 +204,22 @@ __device__ __forceinline__ uint4 quant16_evenodd(uint4 a, uint4 b, float s) {
     return make_uint4(pack4(0, 2, 4, 6), pack4(8, 10, 12, 14), pack4(1, 3, 5, 7), pack4(9, 11, 13, 15));
 }
 
+// 16 bf16 -> 16 int8 in the stride-4 k16 layout: word i of the group holds the
+// elements i, i+4, i+8, i+12.
+__device__ __forceinline__ uint4 quant16_stride4(uint4 a, uint4 b, float s) {
+    uint32_t q[16];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        q[2 * i] = q8_bits(__uint_as_float(w[i] << 16), s);
+        q[2 * i + 1] = q8_bits(__uint_as_float(w[i] & 0xFFFF0000u), s);
+    }
+    auto pack4 = [&](int e0, int e1, int e2, int e3) {
+        return __byte_perm(__byte_perm(q[e0], q[e1], 0x0040), __byte_perm(q[e2], q[e3], 0x0040), 0x5410);
+    };
+    return make_uint4(pack4(0, 4, 8, 12), pack4(1, 5, 9, 13), pack4(2, 6, 10, 14), pack4(3, 7, 11, 15));
+}
+
 // |x| of two bf16 at once as unsigned 16-bit lanes; for finite values the integer
 // order of |x| bit patterns is the float order.
 __device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
@@ -214,8 +230,12 @@ __device__ __forceinline__ uint32_t absmax_vec(uint32_t m, uint4 v) {
     return m;
 }
 
-// A unit is U 16-byte vectors of one row: U = 1 (8 elements, row-major output) or U = 2
-// (16 elements, even/odd k16 output).
+// A unit is the U 16-byte input vectors of one row that make one output store.  The
+// output layout L (XqLayout) fixes U: 1 (8 elements, row-major) or 2 (16 elements, the
+// even/odd or stride-4 k16 orders).
+template <int L>
+constexpr int kUnitVecs = L == kXqRowMajor ? 1 : 2;
+
 template <int U>
 struct Unit {
     uint4 v[U];
@@ -229,22 +249,25 @@ __device__ __forceinline__ Unit<U> load_unit(const uint4* xr, int idx) {
     return u;
 }
 
-template <int U>
+template <int L, int U>
 __device__ __forceinline__ void store_unit(uint8_t* qrow, int idx, const Unit<U>& u, float s) {
-    if constexpr (U == 1)
+    if constexpr (L == kXqRowMajor)
         reinterpret_cast<uint2*>(qrow)[idx] = quant8(u.v[0], s);
-    else
+    else if constexpr (L == kXqEvenOdd16)
         reinterpret_cast<uint4*>(qrow)[idx] = quant16_evenodd(u.v[0], u.v[1], s);
+    else
+        reinterpret_cast<uint4*>(qrow)[idx] = quant16_stride4(u.v[0], u.v[1], s);
 }
 
 // One group of G threads per token row; each thread keeps up to NV units of its row in
 // registers between the absmax pass and the quantise pass (longer rows are re-read for
 // the remainder).  Short rows (G = 32) give each warp R rows, whose loads are all issued
 // before the first reduction.  Needs K % (8 U) == 0.
-template <int G, int R, int U>
+template <int G, int R, int L>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
                          uint8_t* __restrict__ xq, float* __restrict__ s_out) {
+    constexpr int U = kUnitVecs<L>;
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G * R;  // rows per block
     constexpr int WPG = G / 32;       // warps per row group
@@ -308,9 +331,9 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
 #pragma unroll
         for (int u = 0; u < NV; ++u) {
             const int idx = j + u * G;
-            if (idx < nunit) store_unit<U>(qrow, idx, v[r][u], s);
+            if (idx < nunit) store_unit<L>(qrow, idx, v[r][u], s);
         }
-        for (int idx = j + NV * G; idx < nunit; idx += G) store_unit<U>(qrow, idx, load_unit<U>(xr, idx), s);
+        for (int idx = j + NV * G; idx < nunit; idx += G) store_unit<L>(qrow, idx, load_unit<U>(xr, idx), s);
     }
 }
 
@@ -376,21 +399,21 @@ cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packe
     return cudaGetLastError();
 }
 
-template <int U>
+template <int L>
 static void launch_act_vec(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s, cudaStream_t stream) {
     const int nvec = K / 8;
     if (nvec <= 32) {
-        act_quant_vec_kernel<32, 4, U><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<32, 4, L><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
     } else if (nvec <= 128) {
-        act_quant_vec_kernel<32, 2, U><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<32, 2, L><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
     } else if (nvec <= 256) {
-        act_quant_vec_kernel<64, 1, U><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<64, 1, L><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
     } else if (nvec <= 512) {
-        act_quant_vec_kernel<128, 1, U><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<128, 1, L><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
     } else if (nvec <= 1024) {
-        act_quant_vec_kernel<256, 1, U><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<256, 1, L><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
     } else {
-        act_quant_vec_kernel<512, 1, U><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, K, eps, xq, s);
+        act_quant_vec_kernel<512, 1, L><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, K, eps, xq, s);
     }
 }
 
@@ -398,15 +421,20 @@ cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float e
                                 float* s, int layout, cudaStream_t stream) {
     uint8_t* q = reinterpret_cast<uint8_t*>(xq);
     const uint4* X4 = reinterpret_cast<const uint4*>(X);
-    if (layout == kXqEvenOdd16) {  // K % 16 == 0 checked by the caller
-        launch_act_vec<2>(X4, M, static_cast<int>(K), eps, q, s, stream);
+    // K % 16 == 0 for the k16 layouts is checked by the caller
+    if (layout == kXqEvenOdd16) {
+        launch_act_vec<kXqEvenOdd16>(X4, M, static_cast<int>(K), eps, q, s, stream);
+        return cudaGetLastError();
+    }
+    if (layout == kXqStride4K16) {
+        launch_act_vec<kXqStride4K16>(X4, M, static_cast<int>(K), eps, q, s, stream);
         return cudaGetLastError();
     }
     if (K % 8 != 0 || K > (int64_t(1) << 30)) {
         act_quant_scalar_kernel<<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X, M, K, eps, xq, s);
         return cudaGetLastError();
     }
-    launch_act_vec<1>(X4, M, static_cast<int>(K), eps, q, s, stream);
+    launch_act_vec<kXqRowMajor>(X4, M, static_cast<int>(K), eps, q, s, stream);
     return cudaGetLastError();
 }
 

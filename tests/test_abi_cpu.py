@@ -107,11 +107,17 @@ def test_other_entry_points_validation(L):
     assert path(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 9, None) == INVALID
     assert L.bitlinear_status_string(3) == b"BL_ERR_MISALIGNED"
     lay = L.bitlinear_forward_layout
-    assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 72, FAKE, 0, None, 1, 0, None) == SHAPE   # even/odd needs K % 16
+    for k16 in (1, 2):  # the k16 layouts need K % 16 == 0
+        assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 72, FAKE, 0, None, k16, 0, None) == SHAPE
     assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 5, 0, None) == INVALID
+    assert lay(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 3, 0, None) == INVALID
+    # stride-4 x_q on a forced tensor-core path needs K <= 2^17
+    for p in (2, 3, 4):
+        assert lay(FAKE, FAKE, FAKE, FAKE, 40, 8, (1 << 17) + 64, FAKE, 0, None, 2, p, None) == SHAPE
     qa = L.bitlinear_quantize_act_layout
     assert qa(FAKE, 4, 24, 1e-5, FAKE, FAKE, 1, None) == SHAPE
-    assert qa(FAKE, 4, 32, 1e-5, FAKE, FAKE, 2, None) == INVALID
+    assert qa(FAKE, 4, 24, 1e-5, FAKE, FAKE, 2, None) == SHAPE
+    assert qa(FAKE, 4, 32, 1e-5, FAKE, FAKE, 3, None) == INVALID
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

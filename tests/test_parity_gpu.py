@@ -269,8 +269,8 @@ def test_forward_extreme_accumulators():
 @pytest.mark.parametrize("name", ["toy", "llama700m", "llama3b", "llama70b"])
 def test_workload_sizes(name):
     """Every projection of each workload at its decode and prefill token counts, in the
-    configuration the benchmark times (automatic dispatch); large problems are checked
-    on sampled token rows plus the linearity property over all rows."""
+    configuration the benchmark times (automatic dispatch, x_q in the stride-4 k16
+    layout) and with row-major x_q; large problems are checked on sampled token rows."""
     spec = synth.WORKLOADS[name]
     projs = spec["proj"]
     if name == "llama70b":
@@ -288,21 +288,37 @@ def test_workload_sizes(name):
             X = synth.activations(M, K, seed=pi + 100 * M, outlier_frac=spec["outlier_frac"])
             xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
             xq, s = B.quantize_act(X.to(DEV), EPS)
+            xq4, s4 = B.quantize_act(X.to(DEV), EPS, layout=B.BL_XQ_K16_STRIDE4)
             sync()
             assert np.array_equal(xq.cpu().numpy(), xq_ref) and np.array_equal(s.cpu().numpy(), s_ref)
+            assert np.array_equal(xq4.cpu().numpy()[:, stride4_positions(K)], xq_ref)
+            assert np.array_equal(s4.cpu().numpy(), s_ref)
             rows = np.arange(M) if M * N * K <= 4e9 else np.unique(
                 np.r_[0, M - 1, np.random.default_rng(M).integers(0, M, 6)])
             acc_ref = oracle.forward(xq_ref[rows], s_ref[rows], packed_ref, g_ref, K, oracle.OUT_I32)
             y_ref = oracle.dequant(acc_ref, s_ref[rows], g_ref)
             gamma = torch.tensor([g_ref], device=DEV)
             pk = torch.from_numpy(packed_ref).to(DEV)
-            acc = B.forward(xq, s, pk, gamma, torch.int32).cpu().numpy()
-            y = B.forward(xq, s, pk, gamma, torch.float32).cpu().numpy()
-            assert np.array_equal(acc[rows], acc_ref), (name, pname, M)
-            assert_float_close(y[rows], y_ref, "%s %s M=%d" % (name, pname, M))
+            for lay, xl, sl in ((B.BL_XQ_ROWMAJOR, xq, s), (B.BL_XQ_K16_STRIDE4, xq4, s4)):
+                acc = B.forward(xl, sl, pk, gamma, torch.int32, layout=lay).cpu().numpy()
+                y = B.forward(xl, sl, pk, gamma, torch.float32, layout=lay).cpu().numpy()
+                assert np.array_equal(acc[rows], acc_ref), (name, pname, M, lay)
+                assert_float_close(y[rows], y_ref, "%s %s M=%d layout %d" % (name, pname, M, lay))
 
 
-# ------------------------------------------------ x_q in the even/odd k16 layout --
+# ------------------------------------------------ x_q in the k16 layouts --
+
+def stride4_positions(K):
+    """Byte position of every element k in the stride-4 k16 layout, built from the
+    layout's definition: inside each group of 16 the element order is
+    0,4,8,12, 1,5,9,13, 2,6,10,14, 3,7,11,15."""
+    order = [0, 4, 8, 12, 1, 5, 9, 13, 2, 6, 10, 14, 3, 7, 11, 15]
+    pos = np.empty(K, dtype=np.int64)
+    for q in range(K // 16):
+        for p, e in enumerate(order):
+            pos[16 * q + e] = 16 * q + p
+    return pos
+
 
 def evenodd_positions(K):
     """Byte position of every element k in the even/odd k16 layout, built from the
@@ -357,3 +373,124 @@ def test_forward_evenodd_layout(M, N, K, path):
             assert np.array_equal(out.cpu().numpy(), acc_ref)
         else:
             assert_float_close(out.cpu().numpy(), y_ref, "evenodd fp32")
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (5, 1536), (33, 4096), (4096, 1536), (3, 28672), (64, 208)])
+def test_quantize_act_stride4_layout(M, K):
+    X = synth.activations(M, K, seed=M + 13 * K)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    xq = guarded_empty((M, K), torch.int8)
+    s = guarded_empty((M,), torch.float32)
+    B.bitlinear_quantize_act(X.to(DEV), EPS, xq, s, layout=B.BL_XQ_K16_STRIDE4)
+    sync()
+    check_guard(xq)
+    check_guard(s)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(xq.cpu().numpy()[:, stride4_positions(K)], xq_ref)
+
+
+def run_layout_forward(xq_ref, s_ref, packed_ref, g_ref, layout, positions, path, dtypes, rows=None):
+    M, K = xq_ref.shape
+    N = packed_ref.shape[0]
+    sel = np.arange(M) if rows is None else np.asarray(rows)
+    acc_ref = oracle.forward(xq_ref[sel], s_ref[sel], packed_ref, g_ref, K, oracle.OUT_I32)
+    y_ref = oracle.dequant(acc_ref, s_ref[sel], g_ref)
+    xl = np.empty_like(xq_ref)
+    xl[:, positions] = xq_ref
+    xq = torch.from_numpy(xl).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    for dt in dtypes:
+        out = guarded_empty((M, N), dt)
+        err = torch.zeros(1, dtype=torch.int32, device=DEV)
+        B.bitlinear_forward(xq, s, packed, gamma, out, err, path=path, layout=layout)
+        sync()
+        check_guard(out)
+        assert err.item() == 0
+        if dt == torch.int32:
+            assert np.array_equal(out.cpu().numpy()[sel], acc_ref), "int32 accumulators differ"
+        elif dt == torch.float32:
+            assert_float_close(out.cpu().numpy()[sel], y_ref, "fp32 y")
+        else:
+            yb = out.view(torch.int16).cpu().numpy().view(np.uint16)[sel]
+            assert_bf16_match(yb, y_ref, oracle.f32_to_bf16(y_ref), "bf16 y")
+
+
+# (M, N, K, path): the persistent TMA decode kernel takes M <= 16 with at least one
+# 16-row tile per SM; N picks how many tiles each SM owns (1, 2, 4, 13, 18, 32) and so
+# how warps share tile pairs; K covers partial 512-code units and ragged 128-code tails
+S4_CASES = [(1, 2368, 128, B.BL_PATH_GEMV), (1, 4096, 1536, B.BL_PATH_GEMV), (16, 8192, 640, B.BL_PATH_GEMV),
+            (8, 28672, 1536, B.BL_PATH_GEMV), (9, 3001, 3200, B.BL_PATH_GEMV), (2, 40000, 1024, B.BL_PATH_GEMV),
+            (16, 75000, 256, B.BL_PATH_GEMV), (3, 9000, 8192, B.BL_PATH_AUTO), (1, 300, 256, B.BL_PATH_GEMV),
+            (40, 200, 256, B.BL_PATH_GEMV), (5, 64, 208, B.BL_PATH_AUTO), (100, 300, 192, B.BL_PATH_TC_1SM),
+            (513, 4096, 1536, B.BL_PATH_TC_1SM), (300, 200, 320, B.BL_PATH_TC_2SM),
+            (1000, 1536, 4096, B.BL_PATH_TC_2SM), (4096, 1536, 1536, B.BL_PATH_TC), (17, 128, 128, B.BL_PATH_TC_1SM)]
+
+
+@pytest.mark.parametrize("M,N,K,path", S4_CASES)
+def test_forward_stride4_layout(M, N, K, path):
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=M + N + 5 * K, zero_row=True)
+    run_layout_forward(xq_ref, s_ref, packed_ref, g_ref, B.BL_XQ_K16_STRIDE4, stride4_positions(K), path,
+                       (torch.int32, torch.float32, torch.bfloat16))
+
+
+@pytest.mark.parametrize("layout", [B.BL_XQ_ROWMAJOR, B.BL_XQ_K16_EVENODD, B.BL_XQ_K16_STRIDE4],
+                         ids=["rowmajor", "evenodd", "stride4"])
+@pytest.mark.parametrize("M,N,K,path", [(1, 2400, 1024, B.BL_PATH_GEMV), (16, 512, 512, B.BL_PATH_GEMV),
+                                        (200, 384, 512, B.BL_PATH_TC_1SM), (300, 512, 512, B.BL_PATH_TC_2SM)])
+def test_forward_reads_code_11_as_zero(M, N, K, path, layout):
+    """Packed bytes drawn uniformly from 0..255 hold the unused code 11 in a quarter of
+    the fields; every kernel must read it as 0, as the oracle does."""
+    rng = np.random.default_rng(M + N + K + layout)
+    packed_ref = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    xq_ref = rng.integers(-128, 128, size=(M, K), dtype=np.int8)
+    s_ref = rng.uniform(0.5, 2.0, size=M).astype(np.float32)
+    pos = {B.BL_XQ_ROWMAJOR: np.arange(K), B.BL_XQ_K16_EVENODD: evenodd_positions(K),
+           B.BL_XQ_K16_STRIDE4: stride4_positions(K)}[layout]
+    run_layout_forward(xq_ref, s_ref, packed_ref, np.float32(0.03), layout, pos, path, (torch.int32,))
+
+
+def test_forward_stride4_extreme_accumulators_and_k_limit():
+    """The stride-4 kernels sum 64 * code: at K = 2^17 with |x_q| = 128 and every code -1
+    the scaled sums reach 2^30 and must still be exact; above 2^17 the tensor-core paths
+    refuse the shape and the automatic dispatch runs the unscaled GEMV."""
+    N = 2400
+    for M, K, path in ((1, 1 << 17, B.BL_PATH_GEMV), (16, 1 << 15, B.BL_PATH_GEMV), (200, 1 << 17, B.BL_PATH_TC_1SM),
+                       (300, 1 << 17, B.BL_PATH_TC_2SM), (16, (1 << 17) + 128, B.BL_PATH_AUTO)):
+        xq = torch.full((M, K), -128, dtype=torch.int8, device=DEV)
+        xq[1::2] = 127
+        packed = torch.full((N, K // 4), 0xAA, dtype=torch.uint8, device=DEV)  # all -1
+        packed[::5] = 0x55                                                     # all +1
+        s = torch.ones(M, device=DEV)
+        gamma = torch.tensor([1.0], device=DEV)
+        # the layout only permutes x_q inside each 16-group; a row of equal bytes is unchanged
+        want = (xq.long().sum(1)[:, None] * torch.where(torch.arange(N, device=DEV) % 5 == 0, 1, -1)[None, :])
+        acc = B.forward(xq, s, packed, gamma, torch.int32, path=path, layout=B.BL_XQ_K16_STRIDE4)
+        sync()
+        assert torch.equal(acc.long(), want), (M, K, path)
+    xq = torch.zeros((200, (1 << 17) + 128), dtype=torch.int8, device=DEV)
+    packed = torch.zeros((256, xq.shape[1] // 4), dtype=torch.uint8, device=DEV)
+    with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):
+        B.forward(xq, torch.ones(200, device=DEV), packed, torch.ones(1, device=DEV), torch.int32,
+                  path=B.BL_PATH_TC, layout=B.BL_XQ_K16_STRIDE4)
+
+
+def test_forward_all_paths_and_layouts_agree():
+    M, N, K = 16, 4800, 2048
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, 21)
+    xq = torch.from_numpy(xq_ref).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    outs = []
+    for layout, pos in ((B.BL_XQ_ROWMAJOR, np.arange(K)), (B.BL_XQ_K16_EVENODD, evenodd_positions(K)),
+                        (B.BL_XQ_K16_STRIDE4, stride4_positions(K))):
+        xl = np.empty_like(xq_ref)
+        xl[:, pos] = xq_ref
+        xd = torch.from_numpy(xl).to(DEV)
+        for path in (B.BL_PATH_GEMV, B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM):
+            outs.append(B.forward(xd, s, packed, gamma, torch.int32, path=path, layout=layout))
+    sync()
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
