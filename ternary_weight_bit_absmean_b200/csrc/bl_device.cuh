@@ -92,6 +92,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// ------------------------------------------------ programmatic dependent launch --
+
+// Every kernel of the library is launched with programmatic stream serialisation
+// allowed, so that its launch and prologue can overlap the tail of the previous kernel
+// on the stream.  It calls this before its first access to global memory: wait until
+// the previous kernel has completed and its writes are visible (a no-op when there is
+// none), then let the next kernel on the stream launch.
+__device__ __forceinline__ void pdl_wait_then_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -59,4 +59,33 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);
 
+// Launch `kernel` on `stream` with programmatic stream serialisation allowed (the kernel
+// calls pdl_wait_then_release() before touching global memory) and, when cluster.x > 0,
+// a thread-block cluster of that shape.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       dim3 cluster, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster.x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster.x;
+        attr[n].val.clusterDim.y = cluster.y;
+        attr[n].val.clusterDim.z = cluster.z;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+constexpr unsigned kNoCluster = 0;
+
 }  // namespace bl

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmap_x);
         tma_prefetch_desc(&tmap_p);
     }
+    pdl_wait_then_release();
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
@@ -405,8 +406,8 @@ cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
     const int grid = a.num_tiles < sms ? a.num_tiles : sms;
-    gemm_tc_kernel<BT, LAY><<<grid, kThreads, C::kSmemBytes, stream>>>(tx, tp, a);
-    return cudaGetLastError();
+    return launch_pdl(gemm_tc_kernel<BT, LAY>, dim3(grid), dim3(kThreads), C::kSmemBytes, stream, dim3(kNoCluster),
+                      tx, tp, a);
 }
 
 }  // namespace

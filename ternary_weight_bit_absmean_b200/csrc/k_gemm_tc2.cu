@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmap_x);
         tma_prefetch_desc(&tmap_p);
     }
+    pdl_wait_then_release();
     if (warp == kWarpMma) {
         tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish_pair();
@@ -381,19 +382,8 @@ static cudaError_t launch_tc2_layout(const CUtensorMap& tx, const CUtensorMap& t
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<LAY>, tx, tp, a);
+    return launch_pdl(gemm_tc2_kernel<LAY>, dim3(static_cast<unsigned>(2 * clusters)), dim3(kThreads), kSmemBytes,
+                      stream, dim3(2, 1, 1), tx, tp, a);
 }
 
 cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,

@@ -190,6 +190,7 @@ __device__ __forceinline__ void gemv_step(int (&acc)[2][MT][4], uint32_t w0, uin
 
 template <int MT, int LAY>
 __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
+    pdl_wait_then_release();
     constexpr int MP = 8 * MT;  // tokens per block (padded)
     extern __shared__ __align__(16) uint8_t smem[];
     // xs: for window chunk c, word i (0..3), token m, thread-in-group t: 16 permuted bytes
@@ -355,6 +356,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
 
 // One output per thread, any K % 4 == 0 (rows of packed bytes need not be aligned).
 __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
+    pdl_wait_then_release();
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= a.M * a.N) return;
     const int64_t m = idx / a.N, n = idx % a.N;
@@ -399,22 +401,9 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[dev] = true;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(S),
-                       static_cast<unsigned>(token_blocks));
-    cfg.blockDim = dim3(kGvThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    if (S > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 1;
-        attr[0].val.clusterDim.y = S;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    }
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<MT, LAY>, a);
+    return launch_pdl(gemv_kernel<MT, LAY>,
+                      dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(S), static_cast<unsigned>(token_blocks)),
+                      dim3(kGvThreads), smem, stream, S > 1 ? dim3(1, S, 1) : dim3(kNoCluster), a);
 }
 
 }  // namespace
@@ -472,8 +461,8 @@ cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t*
     GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16,
                layout};
     const int64_t total = M * N;
-    gemv_generic_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(gemv_generic_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, stream,
+                      dim3(kNoCluster), a);
 }
 
 }  // namespace bl

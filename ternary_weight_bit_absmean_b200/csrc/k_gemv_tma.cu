@@ -18,12 +18,12 @@
 // the whole of K.  The block's warps are grouped per pair of tiles; when a block has
 // few tiles, several warps share a pair, each taking part of every stage's K range, and
 // they add their partial sums through shared memory at the end.  A producer lane
-// streams, per stage and per 512 codes of K, one 128-byte-swizzled TMA box of 16 rows x
-// 128 bytes per tile and one box of the activations.  The activation box gathers a 4-D
-// view of x_q (bytes of a 16-group, 128-byte blocks along K, tokens, 16-groups of a
-// block) so that shared memory holds [16-group][token][block][16 bytes]; the warps'
-// fragment reads of both operands are then free of bank conflicts.  K tails and rows
-// past N read the TMA's zero fill.  Every wait is bounded.
+// streams the weights, per stage and per 1024 codes of K, as one TMA box of 16 rows x
+// 256 bytes per tile (256 contiguous bytes per row keep the DRAM reads long; 128-byte
+// boxes measured a third slower).  The activations, a few kilobytes per stage shared by
+// every warp, are read by the warps themselves through L1, issued before each wait for
+// the weights.  K tails and rows past N read the TMA's zero fill.  Every wait is
+// bounded.
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cuda.h>
@@ -34,8 +34,6 @@
 
 namespace bl {
 
-bool encode_tmap_u8(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-                    const uint32_t* box, bool swizzle128);
 bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                        uint32_t box_outer, bool swizzle128);
 
@@ -43,20 +41,22 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kUnitCodes = 512;       // K codes per TMA box: 128 packed bytes per row
-constexpr int kTileBytes = 16 * 128;  // one 16-row weight box
+constexpr int kUnitCodes = 1024;      // K codes per weight box: 256 packed bytes per row
+constexpr int kTileBytes = 16 * 256;  // one 16-row weight box
 constexpr int kMaxTilesPerBlock = 2 * kConsumerWarps;
+constexpr int kMaxPairs = kMaxTilesPerBlock / 2;
 constexpr int64_t kMaxK = int64_t(1) << 17;  // keeps 64 * 128 * K below 2^31
 constexpr int kSmemLimit = 227 * 1024;
 
 struct GtArgs {
+    const int8_t* xq;
     const float* s;
     const float* gamma;
     int M, N, K;
     int ntiles;      // 16-row tiles in N
     int nstages;     // shared-memory stages
     int tile_slots;  // tiles per unit buffer (even, >= the most tiles any block owns)
-    int units;       // 512-code units per stage
+    int units;       // 1024-code units per stage
     int wpp;         // warps per tile pair (a power of two)
     void* out;
     int kind;
@@ -135,16 +135,22 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// Shared memory (1024-byte aligned): per stage, [unit][tile slot][16 rows x 128 B]
-// weights then [unit][16-group of a block (8)][token (MP)][block (4)][16 B] activations;
-// after the stages the full and empty barriers, the abort flag and the buffer through
-// which warps that share a tile pair add their partial sums.
+// Shared memory (1024-byte aligned): per stage and per 1024-code unit, the weight boxes
+// [tile slot][16 rows][256 B]; after the stages one full barrier per (stage, tile pair),
+// one empty barrier per stage, and the abort flag.  A stage streams every tile of the
+// block at the same K offset (long, regular DRAM reads), but each pair of tiles has its
+// own full barrier, so a warp starts on its tiles as soon as their boxes land.  Warps
+// that share a tile pair add their partial sums through the stage memory once every
+// stage has been consumed.
+//
+// Quarter c of a unit (256 codes) gives thread t of a quad weight piece P = 4c + t of its
+// rows (16-groups 4P + i, i = 0..3).  Those weight reads, 256 bytes apart per row, are
+// 2-way bank conflicted.  The thread reads the matching 16 activation bytes of its
+// tokens straight from global memory (the stride-4 layout keeps a 16-group contiguous):
+// every warp of the block reads the same few kilobytes per stage, which stay in L1.
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                    const GtArgs a) {
-    constexpr int MP = 8 * MT;
-    constexpr int kXUnit = MP * kUnitCodes;  // activation bytes per unit
+    gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const GtArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -152,33 +158,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = raw + pad;
     const int ST = a.nstages, U = a.units, R = a.wpp;
     const uint32_t w_unit = static_cast<uint32_t>(a.tile_slots) * kTileBytes;
-    const uint32_t w_stage = static_cast<uint32_t>(U) * w_unit;
-    const uint32_t stage_bytes = w_stage + static_cast<uint32_t>(U) * kXUnit;
+    const uint32_t stage_bytes = static_cast<uint32_t>(U) * w_unit;
     const uint32_t off_bar = static_cast<uint32_t>(ST) * stage_bytes;
     const uint32_t sBar = base + off_bar;
-    auto full = [&](int s) { return sBar + 8u * s; };
-    auto empty = [&](int s) { return sBar + 8u * (ST + s); };
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + off_bar + 16 * ST);
-    int* red = reinterpret_cast<int*>(gbase + off_bar + 16 * ST + 16);
+    auto full = [&](int s, int pr) { return sBar + 8u * (s * kMaxPairs + pr); };
+    auto empty = [&](int s) { return sBar + 8u * (ST * kMaxPairs + s); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + off_bar + 8 * ST * (kMaxPairs + 1));
+    int* red = reinterpret_cast<int*>(gbase);  // aliases the stages once they are all consumed
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * a.ntiles) / gridDim.x);
     const int t_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * a.ntiles) / gridDim.x);
     const int nt = t_end - t_begin;
     const int npairs = (nt + 1) / 2;
-    const int kunits = a.K / kUnitCodes + (a.K % kUnitCodes ? 1 : 0);  // 512-code units in K
+    const int kunits = (a.K + kUnitCodes - 1) / kUnitCodes;  // 1024-code units in K
     const int nstep = (kunits + U - 1) / U;
 
     if (threadIdx.x == 0) {
+        // only the warps that own a tile pair consume (and release) stages: a warp with no
+        // pair must not arrive, or its arrivals would run ahead into later phases and
+        // release a stage that a slower pair is still reading
         for (int s = 0; s < ST; ++s) {
-            mbar_init(full(s), 1);
-            mbar_init(empty(s), kConsumerWarps);
+            for (int pr = 0; pr < npairs; ++pr) mbar_init(full(s, pr), 1);
+            mbar_init(empty(s), npairs * R);
         }
         *abort_flag = 0;
         mbar_fence_init();
         tma_prefetch_desc(&tmap_w);
-        tma_prefetch_desc(&tmap_x);
     }
+    pdl_wait_then_release();
     __syncthreads();
 
     if (warp == kConsumerWarps) {
@@ -194,16 +202,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 // units past the end of K are neither loaded nor read
-                const int uk = kunits - kt * U < U ? kunits - kt * U : U;
-                mbar_arrive_expect_tx(full(stage),
-                                      static_cast<uint32_t>(uk) * (static_cast<uint32_t>(nt) * kTileBytes + kXUnit));
+                const int u0 = kt * U;
+                const int uk = kunits - u0 < U ? kunits - u0 : U;
                 const uint32_t sw = base + stage * stage_bytes;
-                for (int u = 0; u < uk; ++u) {
-                    const int unit = kt * U + u;
-                    for (int t = 0; t < nt; ++t)
-                        tma_load_2d(sw + u * w_unit + t * kTileBytes, &tmap_w, full(stage), unit * 128,
-                                    16 * (t_begin + t));
-                    tma_load_4d(sw + w_stage + u * kXUnit, &tmap_x, full(stage), 0, 4 * unit, 0, 0);
+                for (int pr = 0; pr < npairs; ++pr) {
+                    const int tn = nt - 2 * pr < 2 ? nt - 2 * pr : 2;
+                    mbar_arrive_expect_tx(full(stage, pr), static_cast<uint32_t>(uk * tn) * kTileBytes);
+                    for (int u = 0; u < uk; ++u)
+                        for (int t = 2 * pr; t < 2 * pr + tn; ++t)
+                            tma_load_2d(sw + u * w_unit + t * kTileBytes, &tmap_w, full(stage, pr), (u0 + u) * 256,
+                                        16 * (t_begin + t));
                 }
                 ++issued;
                 if (++stage == ST) {
@@ -215,9 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // let every issued copy land before the block exits
                 for (int s = 0; s < ST; ++s) {
                     const long long fills = (issued - s + ST - 1) / ST;
-                    if (fills > 0) {
+                    for (int pr = 0; fills > 0 && pr < npairs; ++pr) {
                         const unsigned long long t0 = globaltimer_ns();
-                        while (!mbar_try_wait(full(s), static_cast<uint32_t>((fills - 1) & 1)) &&
+                        while (!mbar_try_wait(full(s, pr), static_cast<uint32_t>((fills - 1) & 1)) &&
                                globaltimer_ns() - t0 < 200000000ull) {
                         }
                     }
@@ -229,6 +237,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = lane >> 2, t = lane & 3;
         const int pair = warp / R, part = warp % R;
         const bool active = pair < npairs;
+        // the unpack's multipliers, held in registers for the whole loop
+        S4Mul mul;
+        asm volatile("mov.b32 %0, %5;\n\tmov.b32 %1, %6;\n\tmov.b32 %2, %7;\n\tmov.b32 %3, %8;\n\tmov.b32 %4, %9;"
+                     : "=r"(mul.hi1), "=r"(mul.two), "=r"(mul.m4), "=r"(mul.m16), "=r"(mul.m64)
+                     : "r"(a.mul.hi1), "r"(a.mul.two), "r"(a.mul.m4), "r"(a.mul.m16), "r"(a.mul.m64));
         int acc[2][MT][4];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -236,55 +249,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < MT; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][j][e] = 0;
-        // byte offsets in a unit's weight buffer of this thread's rows, per half h of the
-        // unit: rows g and g + 8 of the pair's two tiles; 16-byte piece 2t + h of a
-        // 128-byte row sits at slot (2t + h) ^ g (the 128-byte swizzle)
-        uint32_t woff[2][4];
+        // byte offsets in a unit's weight buffer of rows g and g + 8 of the pair's tiles,
+        // at this thread's piece of quarter 0
+        const uint32_t tb = static_cast<uint32_t>(2 * pair) * kTileBytes + 16u * t;
+        const uint32_t woff[4] = {tb + g * 256u, tb + (g + 8) * 256u, tb + kTileBytes + g * 256u,
+                                  tb + kTileBytes + (g + 8) * 256u};
+        // this thread's activation rows (tokens g and g + 8; padding tokens read as zero)
+        const int8_t* xrow0 = a.xq + static_cast<int64_t>(g < a.M ? g : 0) * a.K + 64 * t;
+        const int8_t* xrow1 = a.xq + static_cast<int64_t>(g + 8 < a.M ? g + 8 : 0) * a.K + 64 * t;
+        const bool ok0 = g < a.M, ok1 = MT > 1 && g + 8 < a.M;
+        // the activations of quarter c (global 256-code index q) for this thread
+        auto load_x = [&](int q, uint4 (&b)[4], uint4 (&bb)[4]) {
+            const int k0 = q * 256;  // + 64 t + 16 i inside the row
+            // K % 128 == 0: this thread's 64 codes are all inside K or all past it
+            const bool in = k0 + 64 * t < a.K;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t ps = static_cast<uint32_t>(((2 * t + h) ^ g) << 4);
-            woff[h][0] = (2 * pair) * kTileBytes + g * 128 + ps;
-            woff[h][1] = (2 * pair) * kTileBytes + (g + 8) * 128 + ps;
-            woff[h][2] = (2 * pair + 1) * kTileBytes + g * 128 + ps;
-            woff[h][3] = (2 * pair + 1) * kTileBytes + (g + 8) * 128 + ps;
-        }
-        // the activations of 16-group 4h + i of block t for token g sit at
-        // ((4h + i) * MP + g) * 64 + t * 16; token g + 8 is 512 bytes further
-        const uint32_t xoff = static_cast<uint32_t>((g * 4 + t) * 16);
+            for (int i = 0; i < 4; ++i) {
+                b[i] = (ok0 && in) ? __ldg(reinterpret_cast<const uint4*>(xrow0 + k0 + 16 * i)) : make_uint4(0, 0, 0, 0);
+                if constexpr (MT > 1)
+                    bb[i] = (ok1 && in) ? __ldg(reinterpret_cast<const uint4*>(xrow1 + k0 + 16 * i))
+                                        : make_uint4(0, 0, 0, 0);
+                else
+                    bb[i] = b[i];
+            }
+        };
         int stage = 0;
         uint32_t phase = 0;
         for (int kt = 0; kt < nstep; ++kt) {
-            if (!mbar_wait_bounded(full(stage), phase, abort_flag)) break;
+            const int uk = kunits - kt * U < U ? kunits - kt * U : U;
+            // the first quarter's activations are requested before the wait for the weights
+            uint4 b[4], bb[4];
+            if (active && part < 4 * uk) load_x(4 * kt * U + part, b, bb);
+            if (active && !mbar_wait_bounded(full(stage, pair), phase, abort_flag)) break;
             if (active) {
                 const uint8_t* sw = gbase + stage * stage_bytes;
-                const int uk = kunits - kt * U < U ? kunits - kt * U : U;
-                for (int c = part; c < 2 * uk; c += R) {
-                    const int u = c >> 1, h = c & 1;
-                    const uint8_t* wu = sw + u * w_unit;
-                    const uint8_t* xu = sw + w_stage + u * kXUnit + h * (4 * MP * 64) + xoff;
+                for (int c = part; c < 4 * uk; c += R) {
+                    if (c != part) load_x(4 * kt * U + c, b, bb);
+                    const uint8_t* wq = sw + (c >> 2) * w_unit + (c & 3) * 64;
                     uint4 w[4];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        w[r] = *reinterpret_cast<const uint4*>(wu + (h ? woff[1][r] : woff[0][r]));
+                    for (int r = 0; r < 4; ++r) w[r] = *reinterpret_cast<const uint4*>(wq + woff[r]);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 b = *reinterpret_cast<const uint4*>(xu + i * (MP * 64));
-                        uint4 bb = b;
-                        if constexpr (MT > 1) bb = *reinterpret_cast<const uint4*>(xu + i * (MP * 64) + 8 * 64);
+                    for (int i = 0; i < 4; ++i)
                         s4_step<MT>(acc, word_of(w[0], i), word_of(w[1], i), word_of(w[2], i), word_of(w[3], i),
-                                    b, bb, a.mul);
-                    }
+                                    b[i], bb[i], mul);
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty(stage));
+            if (active && lane == 0) mbar_arrive(empty(stage));
             if (++stage == ST) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
-        // warps that share a pair add their partial sums into the pair's first warp
+        // warps that share a pair add their partial sums into the pair's first warp, in
+        // the stage memory: every consumer has left the loop, and every issued copy was
+        // waited for, before the first write
         if (R > 1) {
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
 #pragma unroll
             for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -354,22 +376,21 @@ bool plan_gemv_tma(int64_t M, int64_t N, int64_t K, int sms, GtPlan* p) {
     int wpp = 1;
     while (2 * wpp * npairs <= kConsumerWarps) wpp *= 2;
     const int kunits = static_cast<int>((K + kUnitCodes - 1) / kUnitCodes);
-    int units = wpp / 2 > 1 ? wpp / 2 : 1;
+    int units = wpp / 4 > 1 ? wpp / 4 : 1;  // a unit gives four warps a quarter each
     if (units > kunits) units = kunits;
     const size_t red = static_cast<size_t>(kConsumerWarps) * 32 * 8 * MT * sizeof(int);
-    const size_t fixed = 1024 + 16 + red + 64;
+    const size_t fixed = 1024 + 16 + 64;
     for (;;) {
-        const size_t stage =
-            static_cast<size_t>(units) * (static_cast<size_t>(slots) * kTileBytes + 8 * MT * kUnitCodes);
-        int stages = static_cast<int>((kSmemLimit - fixed) / (stage + 16));
+        const size_t stage = static_cast<size_t>(units) * static_cast<size_t>(slots) * kTileBytes;
+        int stages = static_cast<int>((kSmemLimit - fixed) / (stage + 8 * (kMaxPairs + 1)));
         if (stages > 8) stages = 8;
-        if (stages >= 2) {
+        if (stages >= 2 && static_cast<size_t>(stages) * stage >= red) {
             p->grid = sms;
             p->tile_slots = slots;
             p->units = units;
             p->wpp = wpp;
             p->stages = stages;
-            p->smem = fixed + static_cast<size_t>(stages) * (stage + 16);
+            p->smem = fixed + static_cast<size_t>(stages) * (stage + 8 * (kMaxPairs + 1));
             return true;
         }
         if (units == 1) return false;
@@ -399,18 +420,11 @@ cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* pac
     GtPlan p;
     if (!plan_gemv_tma(M, N, K, sm_count(), &p)) return cudaErrorInvalidValue;
     const int MT = M <= 8 ? 1 : 2;
-    const int MP = 8 * MT;
-    CUtensorMap tw, tx;
-    // activations viewed as (16 bytes, 128-byte blocks along K, tokens, 16-groups of a
-    // block); the box takes 4 blocks (512 codes) of MP tokens
-    const uint64_t xdims[4] = {16, static_cast<uint64_t>(K / 128), static_cast<uint64_t>(M), 8};
-    const uint64_t xstrides[3] = {128, static_cast<uint64_t>(K), 16};
-    const uint32_t xbox[4] = {16, 4, static_cast<uint32_t>(MP), 8};
-    if (!encode_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), 128, 16, true) ||
-        !encode_tmap_u8(&tx, xq, 4, xdims, xstrides, xbox, false))
+    CUtensorMap tw;
+    if (!encode_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), 256, 16, false))
         return cudaErrorInvalidValue;
     const int64_t ntiles = (N + 15) / 16;
-    GtArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(ntiles),
+    GtArgs a{xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(ntiles),
              p.stages, p.tile_slots, p.units, p.wpp, out, kind, err, s4_mul()};
     static bool attr_done[2][64] = {};
     const int mi = MT - 1;
@@ -422,11 +436,8 @@ cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* pac
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_done[mi][dev] = true;
     }
-    if (MT == 1)
-        gemv_tma_kernel<1><<<p.grid, kThreads, p.smem, stream>>>(tw, tx, a);
-    else
-        gemv_tma_kernel<2><<<p.grid, kThreads, p.smem, stream>>>(tw, tx, a);
-    return cudaGetLastError();
+    if (MT == 1) return launch_pdl(gemv_tma_kernel<1>, dim3(p.grid), dim3(kThreads), p.smem, stream, dim3(kNoCluster), tw, a);
+    return launch_pdl(gemv_tma_kernel<2>, dim3(p.grid), dim3(kThreads), p.smem, stream, dim3(kNoCluster), tw, a);
 }
 
 }  // namespace bl

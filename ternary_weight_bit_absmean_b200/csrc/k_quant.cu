@@ -42,6 +42,7 @@ __device__ __forceinline__ uint32_t pack4_codes(float4 w, float gamma) {
 __global__ void __launch_bounds__(kAbsThreads) absmean_partials_kernel(const float4* __restrict__ W4,
                                                                       int64_t n4,
                                                                       double* __restrict__ partials) {
+    pdl_wait_then_release();
     double acc = 0.0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kAbsThreads;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * kAbsThreads + threadIdx.x; i < n4;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(256) ternarise_pack_kernel(
     const float4* __restrict__ W4, int64_t numel, const float* __restrict__ gamma_in,
     const double* __restrict__ partials, int nparts, float eps, float* __restrict__ gamma_out,
     uint8_t* __restrict__ packed) {
+    pdl_wait_then_release();
     __shared__ float s_gamma;
     if (threadIdx.x < 32) {
         float g;
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const uint4* __restrict
                                                          int64_t numel,
                                                          uint8_t* __restrict__ packed,
                                                          int32_t* __restrict__ err) {
+    pdl_wait_then_release();
     bool bad = false;
     const int64_t ngroups = numel / 16;  // 16 codes -> one 32-bit word
     uint32_t* packed32 = reinterpret_cast<uint32_t*>(packed);
@@ -267,6 +270,7 @@ template <int G, int R, int L>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
                          uint8_t* __restrict__ xq, float* __restrict__ s_out) {
+    pdl_wait_then_release();
     constexpr int U = kUnitVecs<L>;
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G * R;  // rows per block
@@ -342,6 +346,7 @@ __global__ void __launch_bounds__(256) act_quant_scalar_kernel(const uint16_t* _
                                                               int64_t M, int64_t K, float eps,
                                                               int8_t* __restrict__ xq,
                                                               float* __restrict__ s_out) {
+    pdl_wait_then_release();
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= M) return;
@@ -376,45 +381,43 @@ int absmean_num_partials(int64_t numel) {
 
 cudaError_t launch_absmean_partials(const float* W, int64_t numel, double* partials, int nparts,
                                     cudaStream_t stream) {
-    absmean_partials_kernel<<<nparts, kAbsThreads, 0, stream>>>(
-        reinterpret_cast<const float4*>(W), numel / 4, partials);
-    return cudaGetLastError();
+    return launch_pdl(absmean_partials_kernel, dim3(nparts), dim3(kAbsThreads), 0, stream, dim3(kNoCluster),
+                      reinterpret_cast<const float4*>(W), numel / 4, partials);
 }
 
 cudaError_t launch_ternarise_pack(const float* W, int64_t numel, const float* gamma_in,
                                   const double* partials, int nparts, float eps,
                                   float* gamma_out, uint8_t* packed, cudaStream_t stream) {
     const int grid = grid_for(numel / 16, 256 * 4, 148 * 16);
-    ternarise_pack_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), numel,
-                                                     gamma_in, partials, nparts, eps, gamma_out,
-                                                     packed);
-    return cudaGetLastError();
+    return launch_pdl(ternarise_pack_kernel, dim3(grid), dim3(256), 0, stream, dim3(kNoCluster),
+                      reinterpret_cast<const float4*>(W), numel, gamma_in, partials, nparts, eps, gamma_out, packed);
 }
 
 cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packed, int32_t* err,
                               cudaStream_t stream) {
     const int grid = grid_for(numel / 16, 256 * 4, 148 * 16);
-    pack_codes_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(codes), numel,
-                                                packed, err);
-    return cudaGetLastError();
+    return launch_pdl(pack_codes_kernel, dim3(grid), dim3(256), 0, stream, dim3(kNoCluster),
+                      reinterpret_cast<const uint4*>(codes), numel, packed, err);
+}
+
+template <int G, int R, int L>
+static cudaError_t launch_act_g(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s,
+                                cudaStream_t stream) {
+    constexpr int CTA = G > 256 ? G : 256;
+    return launch_pdl(act_quant_vec_kernel<G, R, L>, dim3(grid_for(M, CTA / G * R, 1 << 30)), dim3(CTA), 0, stream,
+                      dim3(kNoCluster), X4, M, K, eps, xq, s);
 }
 
 template <int L>
-static void launch_act_vec(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s, cudaStream_t stream) {
+static cudaError_t launch_act_vec(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s,
+                                  cudaStream_t stream) {
     const int nvec = K / 8;
-    if (nvec <= 32) {
-        act_quant_vec_kernel<32, 4, L><<<grid_for(M, 32, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
-    } else if (nvec <= 128) {
-        act_quant_vec_kernel<32, 2, L><<<grid_for(M, 16, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
-    } else if (nvec <= 256) {
-        act_quant_vec_kernel<64, 1, L><<<grid_for(M, 4, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
-    } else if (nvec <= 512) {
-        act_quant_vec_kernel<128, 1, L><<<grid_for(M, 2, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
-    } else if (nvec <= 1024) {
-        act_quant_vec_kernel<256, 1, L><<<grid_for(M, 1, 1 << 30), 256, 0, stream>>>(X4, M, K, eps, xq, s);
-    } else {
-        act_quant_vec_kernel<512, 1, L><<<grid_for(M, 1, 1 << 30), 512, 0, stream>>>(X4, M, K, eps, xq, s);
-    }
+    if (nvec <= 32) return launch_act_g<32, 4, L>(X4, M, K, eps, xq, s, stream);
+    if (nvec <= 128) return launch_act_g<32, 2, L>(X4, M, K, eps, xq, s, stream);
+    if (nvec <= 256) return launch_act_g<64, 1, L>(X4, M, K, eps, xq, s, stream);
+    if (nvec <= 512) return launch_act_g<128, 1, L>(X4, M, K, eps, xq, s, stream);
+    if (nvec <= 1024) return launch_act_g<256, 1, L>(X4, M, K, eps, xq, s, stream);
+    return launch_act_g<512, 1, L>(X4, M, K, eps, xq, s, stream);
 }
 
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
@@ -422,20 +425,12 @@ cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float e
     uint8_t* q = reinterpret_cast<uint8_t*>(xq);
     const uint4* X4 = reinterpret_cast<const uint4*>(X);
     // K % 16 == 0 for the k16 layouts is checked by the caller
-    if (layout == kXqEvenOdd16) {
-        launch_act_vec<kXqEvenOdd16>(X4, M, static_cast<int>(K), eps, q, s, stream);
-        return cudaGetLastError();
-    }
-    if (layout == kXqStride4K16) {
-        launch_act_vec<kXqStride4K16>(X4, M, static_cast<int>(K), eps, q, s, stream);
-        return cudaGetLastError();
-    }
-    if (K % 8 != 0 || K > (int64_t(1) << 30)) {
-        act_quant_scalar_kernel<<<grid_for(M, 8, 1 << 30), 256, 0, stream>>>(X, M, K, eps, xq, s);
-        return cudaGetLastError();
-    }
-    launch_act_vec<kXqRowMajor>(X4, M, static_cast<int>(K), eps, q, s, stream);
-    return cudaGetLastError();
+    if (layout == kXqEvenOdd16) return launch_act_vec<kXqEvenOdd16>(X4, M, static_cast<int>(K), eps, q, s, stream);
+    if (layout == kXqStride4K16) return launch_act_vec<kXqStride4K16>(X4, M, static_cast<int>(K), eps, q, s, stream);
+    if (K % 8 != 0 || K > (int64_t(1) << 30))
+        return launch_pdl(act_quant_scalar_kernel, dim3(grid_for(M, 8, 1 << 30)), dim3(256), 0, stream,
+                          dim3(kNoCluster), X, M, K, eps, xq, s);
+    return launch_act_vec<kXqRowMajor>(X4, M, static_cast<int>(K), eps, q, s, stream);
 }
 
 }  // namespace bl

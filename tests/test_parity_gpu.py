@@ -494,3 +494,23 @@ def test_forward_all_paths_and_layouts_agree():
     sync()
     for o in outs[1:]:
         assert torch.equal(outs[0], o)
+
+
+@pytest.mark.parametrize("M", [16, 8])
+def test_forward_stride4_wide_layer_repeated(M):
+    """The LLaMA-70B up projection (28672 x 8192) on the persistent decode kernel, where
+    blocks own 12 or 13 tiles and some warps own no tile pair: repeated launches, each
+    right after an activation-quantisation launch, must all match the oracle (a warp
+    that released stages it did not read once let a stage be refilled under a slower
+    pair)."""
+    N, K = 28672, 8192
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=M + 3)
+    acc_ref = oracle.forward(xq_ref, s_ref, packed_ref, g_ref, K, oracle.OUT_I32)
+    X = synth.activations(M, K, seed=M + 3, outlier_frac=0.01, outlier_scale=20.0).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    for _ in range(6):
+        xq, s = B.quantize_act(X, EPS, layout=B.BL_XQ_K16_STRIDE4)
+        acc = B.forward(xq, s, packed, gamma, torch.int32, path=B.BL_PATH_GEMV, layout=B.BL_XQ_K16_STRIDE4)
+        sync()
+        assert np.array_equal(acc.cpu().numpy(), acc_ref)
