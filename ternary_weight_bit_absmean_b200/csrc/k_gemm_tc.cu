@@ -51,16 +51,19 @@ constexpr int kExpWarps = kWarpEpi - kWarpExp;
 constexpr int kEpiWarps = 8;      // two per TMEM lane quarter, alternating 32-column chunks
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
 
+constexpr int pow2_at_least(int v) { return v <= 32 ? 32 : 2 * pow2_at_least((v + 1) / 2); }
+
 template <int BT>
 struct TcCfg {
-    static_assert(BT == 32 || BT == 64 || BT == 128 || BT == 256, "token tile");
+    // the epilogue reads the accumulator in 32-column chunks
+    static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
     static constexpr int kXBytes = BT * kBK;
     static constexpr int kABytes = kBN * kBK;
     static constexpr int kPBytes = kBN * (kBK / 4);
     static constexpr int kStageBytes = kXBytes + kABytes + kPBytes;
     static constexpr int kStagesRaw = (220 * 1024) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-    static constexpr int kTmemCols = 2 * BT;
+    static constexpr int kTmemCols = pow2_at_least(2 * BT);  // TMEM is allocated in powers of two
     static constexpr int kBarBytes = 8 * (3 * kStages + 5) + 16;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
     static_assert(kStages >= 2, "stages");
@@ -418,29 +421,39 @@ static cudaError_t launch_bt_layout(int bt, const int8_t* xq, const uint8_t* pac
     switch (bt) {
         case 32: return launch_bt<32, LAY>(xq, packed, a, sms, stream);
         case 64: return launch_bt<64, LAY>(xq, packed, a, sms, stream);
+        case 96: return launch_bt<96, LAY>(xq, packed, a, sms, stream);
         case 128: return launch_bt<128, LAY>(xq, packed, a, sms, stream);
+        case 160: return launch_bt<160, LAY>(xq, packed, a, sms, stream);
+        case 192: return launch_bt<192, LAY>(xq, packed, a, sms, stream);
+        case 224: return launch_bt<224, LAY>(xq, packed, a, sms, stream);
         default: return launch_bt<256, LAY>(xq, packed, a, sms, stream);
     }
 }
 
 // Token tile of the single-SM kernel and its cost (cycles of the busiest SM, up to a
-// constant): a 128-byte K stage costs ~2 BT cycles of MMA at peak but never less than a
-// fixed pipeline floor (TMA + expansion latency spread over the stages in flight).
-static int tc1_tile(int64_t M, int64_t N, int sms, int64_t* cost) {
+// constant).  A 128-byte K stage's MMAs take ~2.9 BT cycles at the int8 peak, but its
+// shared-memory traffic (the activation tile written by TMA and read by the MMA, the
+// expanded weights written and read, the packed codes) takes ~320 + 2 BT cycles at 128
+// bytes per cycle and dominates; the epilogue of a tile adds ~8 BT cycles that the next
+// tile's main loop does not hide (its outputs leave as 2-byte stores).  Among token
+// tiles in steps of 32, the one with the fewest waves x tile cycles wins (ties: the
+// smaller).
+static int tc1_tile(int64_t M, int64_t N, int64_t K, int sms, int64_t* cost) {
     const int64_t nN = (N + kBN - 1) / kBN;
-    const int64_t nK = 1;
-    auto c = [&](int b) {
+    const int64_t nK = (K + kBK - 1) / kBK;
+    int best = 32;
+    int64_t best_cost = -1;
+    for (int b = 32; b <= 256; b += 32) {
         const int64_t tiles = nN * ((M + b - 1) / b);
         const int64_t waves = (tiles + sms - 1) / sms;
-        const int64_t per_stage = 2 * b > 400 ? 2 * b : 400;
-        return waves * per_stage * nK;
-    };
-    int bt = 256;
-    if (M <= 32) bt = 32;
-    else if (M <= 64) bt = 64;
-    else bt = c(128) < c(256) ? 128 : 256;
-    *cost = c(bt);
-    return bt;
+        const int64_t c = waves * (nK * (320 + 2 * b) + 8 * b);
+        if (best_cost < 0 || c < best_cost) {
+            best_cost = c;
+            best = b;
+        }
+    }
+    *cost = best_cost;
+    return best;
 }
 
 cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
@@ -451,7 +464,7 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t nN = (N + kBN - 1) / kBN;
     int64_t cost = 0;
-    const int bt = tc1_tile(M, N, sms, &cost);
+    const int bt = tc1_tile(M, N, K, sms, &cost);
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
              0, out, kind, err, s4_mul()};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
@@ -462,9 +475,8 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     }
 }
 
-// The pair kernel moves half the activation bytes per SM and stores 16-byte vectors;
-// it is preferred unless its coarser 256 x 256 tiles leave more waves than the
-// single-SM kernel's.
+// The pair kernel moves half the activation bytes per SM and stores 16-byte vectors; the
+// two kernels are compared with the cost model of tc1_tile.
 cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                            int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
                            cudaStream_t stream) {
@@ -472,10 +484,13 @@ cudaError_t launch_gemm_tc(const int8_t* xq, const float* s, const uint8_t* pack
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int64_t cost1 = 0;
-    tc1_tile(M, N, sms, &cost1);
+    tc1_tile(M, N, K, sms, &cost1);
+    // a pair tile (256 x 256) costs ~918 cycles per stage in the same units, its vector-
+    // store epilogue hidden behind the next tile (fitted to the measured times of both
+    // kernels on ten prefill shapes, M = 512 to 8192)
     const int64_t tiles2 = ((N + 255) / 256) * ((M + 255) / 256);
     const int64_t pairs = sms / 2;
-    const int64_t cost2 = (tiles2 + pairs - 1) / pairs * 512;
+    const int64_t cost2 = (tiles2 + pairs - 1) / pairs * ((K + kBK - 1) / kBK) * 918;
     if (M > 128 && cost2 <= cost1)
         return launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err, layout, stream);
     return launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err, layout, stream);

@@ -213,7 +213,7 @@ def test_forward_gemv(M, N, K):
 
 TC_CASES = [(17, 128, 128), (32, 256, 256), (64, 512, 256), (100, 300, 192), (256, 128, 1536),
             (300, 200, 320), (512, 1536, 1536), (513, 4096, 1536), (1000, 1536, 4096),
-            (8192, 512, 256), (130, 640, 8192)]
+            (8192, 512, 256), (130, 640, 8192), (1792, 2304, 320), (1536, 2304, 192)]
 
 
 @pytest.mark.parametrize("path", [B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM], ids=["tc1sm", "tc2sm"])
