@@ -42,6 +42,8 @@ class Oracle:
         L.oracle_unpack.argtypes = [P, I, I, P]
         L.oracle_unpack.restype = None
         L.oracle_quantize_act.argtypes = [P, I, I, F, P, P]
+        L.oracle_norm_quantize_act.argtypes = [P, P, I, I, ctypes.c_int, F, F, P, P, P]
+        L.oracle_norm_quantize_act.restype = None
         L.oracle_quantize_act.restype = None
         L.oracle_int_matmul.argtypes = [P, P, I, I, I, P]
         L.oracle_int_matmul.restype = I
@@ -102,6 +104,22 @@ class Oracle:
         s = np.empty((M,), dtype=np.float32)
         self.L.oracle_quantize_act(p, M, K, eps, _vp(xq), _vp(s))
         return xq, s
+
+    def norm_quantize_act(self, X_bits, w, kind, norm_eps, eps):
+        """RMSNorm (kind 0) or LayerNorm (kind 1) then the int8 quantiser
+        (oracle_norm_quantize_act).  X_bits: uint16 bf16 bits [M, K]; w: fp32 [K] or None.
+        Returns (x_q, s, x_n)."""
+        X_bits, p = _c(X_bits, np.uint16)
+        M, K = X_bits.shape
+        wp = None
+        if w is not None:
+            w, wp = _c(np.asarray(w, dtype=np.float32).reshape(K), np.float32)
+        xq = np.empty((M, K), dtype=np.int8)
+        s = np.empty((M,), dtype=np.float32)
+        xn = np.empty((M, K), dtype=np.float32)
+        self.L.oracle_norm_quantize_act(p, wp, M, K, int(kind), float(norm_eps), float(eps), _vp(xq), _vp(s),
+                                        _vp(xn))
+        return xq, s, xn
 
     def int_matmul(self, xq, codes):
         """Exact int32 accumulators x_q . codes^T (oracle_int_matmul)."""
@@ -165,6 +183,7 @@ def pack(codes): return default().pack(codes)
 def unpack(packed, K): return default().unpack(packed, K)
 def quantize_weights(W, eps): return default().quantize_weights(W, eps)
 def quantize_act(X_bits, eps): return default().quantize_act(X_bits, eps)
+def norm_quantize_act(X_bits, w, kind, norm_eps, eps): return default().norm_quantize_act(X_bits, w, kind, norm_eps, eps)
 def int_matmul(xq, codes): return default().int_matmul(xq, codes)
 def dequant(acc, s, gamma): return default().dequant(acc, s, gamma)
 def f32_to_bf16(y): return default().f32_to_bf16(y)

@@ -40,6 +40,7 @@
  * Build: plain C99, no SIMD intrinsics, no -ffast-math, -ffp-contract=off.
  */
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #include <math.h>
 
@@ -152,6 +153,54 @@ void oracle_quantize_act(const uint16_t *X, int64_t M, int64_t K, float eps,
             xq[m * K + k] = (int8_t)q;
         }
     }
+}
+
+/* [BIN] Quant(LN(x)): the per-token normalisation in front of the activation
+ * quantiser ("LN = LayerNorm before quant"; [B158]: b1.58 adopts LLaMA-style components, the
+ * RMSNorm among them).  For each token:
+ *   kind 0 (RMSNorm):   mu = 0
+ *   kind 1 (LayerNorm): mu = (sum_k x_k) / K
+ *   v = (sum_k (x_k - mu)^2) / K;   r = 1 / sqrt(v + norm_eps);
+ *   x_n[k] = (x_k - mu) * r * w_k   (w = the per-channel norm weight, 1 when absent),
+ * every step in double precision, sums in index order, x_n rounded once to fp32.
+ * x_n then goes through the activation quantiser of oracle_quantize_act, in fp32:
+ *   a = max_k |x_n[k]|;  s = 127 / max(a, eps);  x_q = clip(round(x_n * s), -128, 127).
+ * xn_out (may be NULL) receives x_n. */
+void oracle_norm_quantize_act(const uint16_t *X, const float *w, int64_t M, int64_t K, int kind,
+                              float norm_eps, float eps, int8_t *xq, float *s_out, float *xn_out)
+{
+    int64_t m, k;
+    float *xn = (float *)malloc((size_t)K * sizeof(float));
+    if (xn == NULL) return;
+    for (m = 0; m < M; ++m) {
+        double mu = 0.0, v = 0.0;
+        if (kind == 1) {
+            for (k = 0; k < K; ++k) mu += (double)bf16_bits_to_float(X[m * K + k]);
+            mu = mu / (double)K;
+        }
+        for (k = 0; k < K; ++k) {
+            double d = (double)bf16_bits_to_float(X[m * K + k]) - mu;
+            v += d * d;
+        }
+        v = v / (double)K;
+        double r = 1.0 / sqrt(v + (double)norm_eps);
+        float a = 0.0f;
+        for (k = 0; k < K; ++k) {
+            double wk = (w != NULL) ? (double)w[k] : 1.0;
+            xn[k] = (float)(((double)bf16_bits_to_float(X[m * K + k]) - mu) * r * wk);
+            if (fabsf(xn[k]) > a) a = fabsf(xn[k]);
+        }
+        const float s = 127.0f / fmaxf(a, eps);
+        s_out[m] = s;
+        for (k = 0; k < K; ++k) {
+            float q = rintf(xn[k] * s);
+            if (q < -128.0f) q = -128.0f;
+            if (q > 127.0f) q = 127.0f;
+            xq[m * K + k] = (int8_t)q;
+            if (xn_out != NULL) xn_out[m * K + k] = xn[k];
+        }
+    }
+    free(xn);
 }
 
 /* --------------------------------------------------------------- forward -- */

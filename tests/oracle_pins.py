@@ -300,7 +300,84 @@ def pin_dequant_vs_float64(O):
     assert np.array_equal(yb, torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
 
 
+# ----------------------------------------------- normalisation + quantiser --
+
+def pin_hand_norm(O):
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "normact":
+            continue
+        x = _floats(r["x"])[None, :]
+        w = _floats(r["w"]) if "w" in r else None
+        xq, s, _ = O.norm_quantize_act(_bf16_bits(x), w, int(r["kind"]), float(r["norm_eps"]), EPS)
+        assert np.array_equal(xq[0].astype(np.int64), _ints(r["xq"])), (r, xq)
+        if "s" in r:
+            assert s[0] == np.float32(float(r["s"])), (r, s)
+        else:
+            assert abs(float(s[0]) / float(r["s_approx"]) - 1.0) < 1e-6, (r, s)
+        n += 1
+    assert n >= 3
+
+
+def _torch_norm_quant(xb, w, kind, norm_eps):
+    """The same two steps through torch's own norm routines (float64) and fp32 ops."""
+    import torch.nn.functional as F
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(torch.float64)
+    K = x.shape[1]
+    wt = None if w is None else torch.from_numpy(w).to(torch.float64)
+    if kind == 0:
+        xn = F.rms_norm(x, (K,), weight=wt, eps=norm_eps)
+    else:
+        xn = F.layer_norm(x, (K,), weight=wt, bias=None, eps=norm_eps)
+    xn = xn.to(torch.float32)
+    a = xn.abs().amax(dim=1)
+    s = torch.tensor(127.0, dtype=torch.float32) / torch.clamp(a, min=EPS)
+    q = torch.round(xn * s[:, None]).clamp(-128, 127)
+    return q.numpy().astype(np.int64), s.numpy(), (xn * s[:, None]).numpy()
+
+
+def pin_norm_vs_torch(O):
+    """torch's rms_norm / layer_norm in float64 then the quantiser in fp32: the scale
+    within 2^-22 (the two sums run in different orders), the codes equal except where
+    x_n s sits within 1e-3 of a rounding midpoint, and those are rare."""
+    rng = np.random.default_rng(7)
+    for kind in (0, 1):
+        for with_w in (False, True):
+            x = rng.standard_normal((64, 384)).astype(np.float32) * 3.0 + (0.7 if kind == 1 else 0.0)
+            x[:, :4] *= 20.0
+            xb = _bf16_bits(x)
+            w = (rng.uniform(0.5, 1.5, size=384).astype(np.float32) if with_w else None)
+            xq, s, _ = O.norm_quantize_act(xb, w, kind, 1e-5, EPS)
+            tq, ts, tv = _torch_norm_quant(xb, w, kind, 1e-5)
+            assert np.all(np.abs(s / ts - 1.0) < 2.0 ** -22), (kind, with_w)
+            frac = np.abs(tv - np.floor(tv) - 0.5)
+            differ = xq.astype(np.int64) != tq
+            assert np.all(frac[differ] < 1e-3), (kind, with_w)
+            assert differ.mean() < 1e-3
+
+
+def pin_norm_invariants(O):
+    """RMSNorm is exactly invariant to scaling a token by a power of two (no norm_eps);
+    a zero token normalises to zero and quantises to zero with s = 127 / eps."""
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((8, 64)).astype(np.float32)
+    xb1, xb2 = _bf16_bits(x), _bf16_bits(np.float32(4.0) * _bf16_to_f32(_bf16_bits(x)))
+    a = O.norm_quantize_act(xb1, None, 0, 0.0, EPS)
+    b = O.norm_quantize_act(xb2, None, 0, 0.0, EPS)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    z = np.zeros((2, 32), dtype=np.uint16)
+    for kind in (0, 1):
+        xq, s, xn = O.norm_quantize_act(z, None, kind, 1e-5, EPS)
+        assert not xq.any() and not xn.any()
+        assert np.all(s == np.float32(127.0) / np.float32(EPS))
+
+
+def _bf16_to_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
 ALL_PINS = [
+    pin_hand_norm, pin_norm_vs_torch, pin_norm_invariants,
     pin_hand_ternarise, pin_hand_absmean, pin_hand_act, pin_hand_pack, pin_hand_matmul,
     pin_gaussian_statistics, pin_constant_magnitude, pin_zero_weights, pin_zero_token,
     pin_code_alphabet_and_sign_symmetry, pin_act_range_and_symmetry,

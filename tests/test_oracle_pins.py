@@ -31,7 +31,7 @@ MUTANTS = [
     ("codes_swapped", "if (c == 1) return 1;\n    if (c == -1) return 2;",
      "if (c == 1) return 2;\n    if (c == -1) return 1;"),
     ("msb_first", "byte |= (unsigned)e << (2 * i);", "byte |= (unsigned)e << (6 - 2 * i);"),
-    ("qb_128", "float s = 127.0f / fmaxf(a, eps);", "float s = 128.0f / fmaxf(a, eps);"),
+    ("qb_128", "\n        float s = 127.0f / fmaxf(a, eps);", "\n        float s = 128.0f / fmaxf(a, eps);"),
     ("act_round_away", "float q = rintf(bf16_bits_to_float(X[m * K + k]) * s);",
      "float q = roundf(bf16_bits_to_float(X[m * K + k]) * s);"),
     ("act_no_abs", "float v = fabsf(bf16_bits_to_float(X[m * K + k]));",
@@ -45,6 +45,12 @@ MUTANTS = [
     ("bf16_truncate", "u += 0x7FFFu + lsb;", "u += 0u * lsb;"),
     ("unpack_wrong_shift", "unsigned c = (byte >> (2 * (k % 4))) & 3u;",
      "unsigned c = (byte >> (2 * (3 - k % 4))) & 3u;"),
+    ("layernorm_no_mean", "mu = mu / (double)K;", "mu = 0.0;"),
+    ("norm_variance_unbiased", "v = v / (double)K;", "v = v / (double)(K - 1);"),
+    ("norm_weight_ignored", "double wk = (w != NULL) ? (double)w[k] : 1.0;", "double wk = 1.0;"),
+    ("norm_eps_dropped", "double r = 1.0 / sqrt(v + (double)norm_eps);", "double r = 1.0 / sqrt(v);"),
+    ("norm_round_away", "float q = rintf(xn[k] * s);", "float q = roundf(xn[k] * s);"),
+    ("norm_qb_128", "const float s = 127.0f / fmaxf(a, eps);", "const float s = 128.0f / fmaxf(a, eps);"),
 ]
 
 
