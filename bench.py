@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2"], default="auto")
     p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
     p.add_argument("--iters", type=int, default=20)
+    p.add_argument("--step-streams", choices=["branches", "serial"], default="branches",
+                   help="capture the timed step with the projections as concurrent graph branches, or in one stream")
     p.add_argument("--sweep", choices=["llama3b", "llama70b", "grid"], default=None,
                    help="time the forward over a family of shapes (one JSON line per shape)")
     p.add_argument("--xq-layout", choices=["stride4", "evenodd", "rowmajor"], default="stride4",
@@ -242,11 +244,32 @@ def run_ours(args):
                 fn()
     torch.cuda.synchronize()
 
-    # the step as a CUDA graph; a second copy carries a timing event around every call
+    # the step as a CUDA graph.  The seven projections are independent, so by default each
+    # one's chain (weight quantisation, packing, then act quant + forward at every M, in
+    # that order) is captured on its own stream: seven concurrent graph branches, forked
+    # from and joined back to the capture stream.  A second, single-stream copy of the
+    # step carries a timing event around every call (per-call breakdown and roofline).
+    side = [torch.cuda.Stream(device=dev) for _ in projs]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        for _, fn in calls:
-            fn()
+        if args.step_streams == "serial":
+            for _, fn in calls:
+                fn()
+        else:
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            joins = []
+            for pi in range(len(projs)):
+                side[pi].wait_event(fork)
+                with torch.cuda.stream(side[pi]):
+                    for lab, fn in calls:
+                        if lab[1] == pi:
+                            fn()
+                    j = torch.cuda.Event()
+                    j.record(side[pi])
+                joins.append(j)
+            for j in joins:
+                stream.wait_event(j)
     ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
           for _ in calls]
     graph_ev = torch.cuda.CUDAGraph()
@@ -371,7 +394,9 @@ def run_ours(args):
                    "M": Ms, "out_dtype": "bf16", "eps": EPS, "xq_layout": args.xq_layout,
                    "stages": "a1+a2 quantize_weights x7, a3 pack x7, a4 quantize_act x28, a5/a6 forward x28",
                    "l2": "flushed between steps outside the timed events (256 MiB written, then another 256 MiB read so no dirty line is left)",
-                   "timing": "CUDA graph replay of the step bracketed by device events, summed over steps, max over ranks; per-call breakdown and roofline from the same number of replays of an instrumented copy of the graph",
+                   "timing": "CUDA graph replay of the step bracketed by device events, summed over steps, max over ranks; per-call breakdown and roofline from the same number of replays of an instrumented single-stream copy of the graph",
+                   "step_streams": ("the 7 projections as concurrent graph branches (each projection's calls in order)"
+                                    if args.step_streams == "branches" else "one stream, calls in order"),
                    "parallelism": "dp%d (independent token batches per GPU, replicated weights)" % world},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": round(e2e_value, 4) if e2e_value is not None else None, "unit": "TOPS",

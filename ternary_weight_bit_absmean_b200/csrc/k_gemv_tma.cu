@@ -254,21 +254,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tb = static_cast<uint32_t>(2 * pair) * kTileBytes + 16u * t;
         const uint32_t woff[4] = {tb + g * 256u, tb + (g + 8) * 256u, tb + kTileBytes + g * 256u,
                                   tb + kTileBytes + (g + 8) * 256u};
-        // this thread's activation rows (tokens g and g + 8; padding tokens read as zero)
+        // this thread's activation rows, tokens g and g + 8.  A padding token (>= M) reads
+        // token 0's row: it only feeds MMA columns whose outputs are never stored.  A
+        // 16-group past K reads the row's start: its weights are the TMA's zero fill.
+        // So every load is unconditional, on an in-bounds address.
         const int8_t* xrow0 = a.xq + static_cast<int64_t>(g < a.M ? g : 0) * a.K + 64 * t;
         const int8_t* xrow1 = a.xq + static_cast<int64_t>(g + 8 < a.M ? g + 8 : 0) * a.K + 64 * t;
-        const bool ok0 = g < a.M, ok1 = MT > 1 && g + 8 < a.M;
-        // the activations of quarter c (global 256-code index q) for this thread
+        // the activations of 256-code quarter q (global index) for this thread
         auto load_x = [&](int q, uint4 (&b)[4], uint4 (&bb)[4]) {
-            const int k0 = q * 256;  // + 64 t + 16 i inside the row
             // K % 128 == 0: this thread's 64 codes are all inside K or all past it
-            const bool in = k0 + 64 * t < a.K;
+            const int k0 = q * 256 + 64 * t < a.K ? q * 256 : 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                b[i] = (ok0 && in) ? __ldg(reinterpret_cast<const uint4*>(xrow0 + k0 + 16 * i)) : make_uint4(0, 0, 0, 0);
+                b[i] = __ldg(reinterpret_cast<const uint4*>(xrow0 + k0 + 16 * i));
                 if constexpr (MT > 1)
-                    bb[i] = (ok1 && in) ? __ldg(reinterpret_cast<const uint4*>(xrow1 + k0 + 16 * i))
-                                        : make_uint4(0, 0, 0, 0);
+                    bb[i] = __ldg(reinterpret_cast<const uint4*>(xrow1 + k0 + 16 * i));
                 else
                     bb[i] = b[i];
             }
@@ -277,14 +277,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t phase = 0;
         for (int kt = 0; kt < nstep; ++kt) {
             const int uk = kunits - kt * U < U ? kunits - kt * U : U;
-            // the first quarter's activations are requested before the wait for the weights
+            // the first quarter's activations are requested before the wait for the weights;
+            // with one token tile (registers to spare) each later quarter's are requested
+            // while the previous quarter computes
             uint4 b[4], bb[4];
             if (active && part < 4 * uk) load_x(4 * kt * U + part, b, bb);
             if (active && !mbar_wait_bounded(full(stage, pair), phase, abort_flag)) break;
             if (active) {
                 const uint8_t* sw = gbase + stage * stage_bytes;
                 for (int c = part; c < 4 * uk; c += R) {
-                    if (c != part) load_x(4 * kt * U + c, b, bb);
+                    uint4 nb[4], nbb[4];
+                    if constexpr (MT == 1) {
+                        if (c + R < 4 * uk) load_x(4 * kt * U + c + R, nb, nbb);
+                    } else {
+                        if (c != part) load_x(4 * kt * U + c, b, bb);
+                    }
                     const uint8_t* wq = sw + (c >> 2) * w_unit + (c & 3) * 64;
                     uint4 w[4];
 #pragma unroll
@@ -293,6 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 4; ++i)
                         s4_step<MT>(acc, word_of(w[0], i), word_of(w[1], i), word_of(w[2], i), word_of(w[3], i),
                                     b[i], bb[i], mul);
+                    if constexpr (MT == 1) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) b[i] = nb[i];
+                    }
                 }
             }
             __syncwarp();
