@@ -51,7 +51,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ref-tokens", type=int, default=4,
                    help="token rows per M in one reference-arm (oracle) step")
-    p.add_argument("--single", choices=["forward", "quantize_act", "quantize_weights", "pack"],
+    p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack"],
                    help="time one entry point on one shape instead of the step (kernel study, ncu)")
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
@@ -520,6 +520,14 @@ def run_single(args):
         lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_quantize_act(X, EPS, xq, s, layout=lay)
         ops, nbytes = 0, 3 * M * K + 4 * M
+    elif args.single == "norm_quantize_act":
+        X = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        nw = torch.rand(K, device=dev) + 0.5
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        s = torch.empty(M, device=dev)
+        lay = xq_layout_of(B, args.xq_layout)
+        fn = lambda: B.bitlinear_norm_quantize_act(X, nw, B.BL_NORM_RMS, 1e-5, EPS, xq, s, layout=lay)
+        ops, nbytes = 0, 3 * M * K + 4 * M + 4 * K
     elif args.single == "quantize_weights":
         W = torch.randn(N, K, device=dev) * 0.02
         gamma = torch.empty(1, device=dev)

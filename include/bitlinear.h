@@ -157,6 +157,37 @@ BL_API bl_status bitlinear_quantize_act_layout(const uint16_t *X, int64_t M, int
                                                int8_t *xq_out, float *s_out, bl_xq_layout layout,
                                                void *stream);
 
+/* Kind of the per-token normalisation in front of the quantiser. */
+typedef enum {
+    BL_NORM_RMS = 0,   /* RMSNorm: mu = 0 */
+    BL_NORM_LAYER = 1  /* LayerNorm without a bias: mu = mean of the token */
+} bl_norm_kind;
+
+/* [BIN] Quant(LN(x)): the normalisation in front of the activation quantiser, fused
+ * with it ("LN = LayerNorm before quant"; [B158]: the b1.58 models use the LLaMA-style
+ * RMSNorm).  Per token m:
+ *   mu = 0 (BL_NORM_RMS) or sum_k x_mk / K (BL_NORM_LAYER)
+ *   v = sum_k (x_mk - mu)^2 / K;   r = 1 / sqrt(v + norm_eps)
+ *   x_n = (x_mk - mu) * r * w_k    (w = norm_weight, or 1 when NULL)
+ * mu, v, r and the product in double precision, x_n rounded once to fp32; then the
+ * quantiser of bitlinear_quantize_act on x_n:
+ *   s_m = 127 / max(max_k |x_n|, eps);   x_q = clip(rint(x_n * s_m), -128, 127).
+ * The sums run in a parallel order; a sequential sum differs by ~1e-16 relative, which
+ * changes x_n only when it lies that close to an fp32 rounding boundary.
+ *   X           in  : bf16 [M, K] as raw uint16 bit patterns, device.  Finite values.
+ *   norm_weight in  : fp32 [K], device, or NULL.
+ *   norm_kind   in  : bl_norm_kind.
+ *   norm_eps    in  : >= 0, finite.
+ *   eps         in  : > 0, finite.
+ *   xq_out      out : int8 [M, K], device, in the given layout (see bl_xq_layout).
+ *   s_out       out : fp32 [M], device.
+ * K % 8 == 0 (K % 16 == 0 for the k16 layouts), K <= 2^30 (else
+ * BL_ERR_UNSUPPORTED_SHAPE).  Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE,
+ * BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_norm_quantize_act(const uint16_t *X, const float *norm_weight, int64_t M, int64_t K,
+                                             bl_norm_kind norm_kind, float norm_eps, float eps, int8_t *xq_out,
+                                             float *s_out, bl_xq_layout layout, void *stream);
+
 /* [BIN] + [STE] + [CH2] the BitLinear forward from quantised operands:
  *   acc[m, n] = sum_k x_q[m, k] * c[n, k]   (exact, int32)
  *   y[m, n]   = float(acc[m, n]) * (gamma / s[m])   (fp32: the quotient and the product

@@ -25,12 +25,13 @@ BL_OUT_F32, BL_OUT_BF16, BL_OUT_I32 = 0, 1, 2
 BL_PATH_AUTO, BL_PATH_GEMV, BL_PATH_TC, BL_PATH_TC_1SM, BL_PATH_TC_2SM = 0, 1, 2, 3, 4
 BL_ERRBIT_BAD_CODE, BL_ERRBIT_TIMEOUT = 0x1, 0x2
 BL_XQ_ROWMAJOR, BL_XQ_K16_EVENODD, BL_XQ_K16_STRIDE4 = 0, 1, 2
+BL_NORM_RMS, BL_NORM_LAYER = 0, 1
 
 EXPORTED = [
     "bitlinear_workspace_size", "bitlinear_quantize_weights",
     "bitlinear_quantize_weights_with_scale", "bitlinear_pack", "bitlinear_quantize_act",
     "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
-    "bitlinear_forward_layout", "bitlinear_last_cuda_error",
+    "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
 
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_quantize_act_layout.restype = S
         L.bitlinear_forward_layout.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, S, P]
         L.bitlinear_forward_layout.restype = S
+        L.bitlinear_norm_quantize_act.argtypes = [P, P, I64, I64, S, F, F, P, P, S, P]
+        L.bitlinear_norm_quantize_act.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
         L.bitlinear_last_cuda_error.restype = ctypes.c_int
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
@@ -149,6 +152,16 @@ def bitlinear_quantize_act(X, eps, xq_out, s_out, stream=None, layout=BL_XQ_ROWM
                "bitlinear_quantize_act_layout")
 
 
+def bitlinear_norm_quantize_act(X, norm_weight, kind, norm_eps, eps, xq_out, s_out, stream=None,
+                                layout=BL_XQ_ROWMAJOR):
+    M, K = X.shape
+    w = None if norm_weight is None else _dev(norm_weight, torch.float32, "norm_weight", (K,))
+    _check(lib().bitlinear_norm_quantize_act(
+        _dev(X, torch.bfloat16, "X"), w, M, K, int(kind), float(norm_eps), float(eps),
+        _dev(xq_out, torch.int8, "xq_out", (M, K)), _dev(s_out, torch.float32, "s_out", (M,)), int(layout),
+        _stream(stream)), "bitlinear_norm_quantize_act")
+
+
 _OUT_DT = {BL_OUT_F32: torch.float32, BL_OUT_BF16: torch.bfloat16, BL_OUT_I32: torch.int32}
 
 
@@ -189,6 +202,16 @@ def quantize_act(X: torch.Tensor, eps: float = 1e-5, stream=None, layout=BL_XQ_R
     xq = torch.empty(M, K, dtype=torch.int8, device=X.device)
     s = torch.empty(M, dtype=torch.float32, device=X.device)
     bitlinear_quantize_act(X, eps, xq, s, stream, layout)
+    return xq, s
+
+
+def norm_quantize_act(X: torch.Tensor, norm_weight=None, kind=BL_NORM_RMS, norm_eps: float = 1e-5,
+                      eps: float = 1e-5, stream=None, layout=BL_XQ_ROWMAJOR):
+    """(x_q [M, K] int8, s [M] fp32) of RMSNorm / LayerNorm(X) for a bf16 CUDA matrix."""
+    M, K = X.shape
+    xq = torch.empty(M, K, dtype=torch.int8, device=X.device)
+    s = torch.empty(M, dtype=torch.float32, device=X.device)
+    bitlinear_norm_quantize_act(X, norm_weight, kind, norm_eps, eps, xq, s, stream, layout)
     return xq, s
 
 

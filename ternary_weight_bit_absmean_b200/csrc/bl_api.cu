@@ -100,6 +100,24 @@ bl_status bitlinear_quantize_act_layout(const uint16_t* X, int64_t M, int64_t K,
     return cuda_status(e);
 }
 
+bl_status bitlinear_norm_quantize_act(const uint16_t* X, const float* norm_weight, int64_t M, int64_t K,
+                                      bl_norm_kind norm_kind, float norm_eps, float eps, int8_t* xq_out, float* s_out,
+                                      bl_xq_layout layout, void* stream) {
+    if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
+    if (!std::isfinite(norm_eps) || norm_eps < 0.0f) return BL_ERR_INVALID_ARG;
+    if (norm_kind != BL_NORM_RMS && norm_kind != BL_NORM_LAYER) return BL_ERR_INVALID_ARG;
+    if (M <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (layout != BL_XQ_ROWMAJOR && layout != BL_XQ_K16_EVENODD && layout != BL_XQ_K16_STRIDE4)
+        return BL_ERR_INVALID_ARG;
+    if (K % (layout == BL_XQ_ROWMAJOR ? 8 : 16) != 0 || K > (int64_t(1) << 30)) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (M > (int64_t(1) << 40) / K || M >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(X) || !aligned16(xq_out) || !aligned16(s_out)) return BL_ERR_MISALIGNED;
+    if (norm_weight != nullptr && !aligned16(norm_weight)) return BL_ERR_MISALIGNED;
+    cudaError_t e = bl::launch_norm_quantize_act(X, norm_weight, M, K, static_cast<int>(norm_kind), norm_eps, eps,
+                                                 xq_out, s_out, static_cast<int>(layout), as_stream(stream));
+    return cuda_status(e);
+}
+
 bl_status bitlinear_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
                                  float* s_out, void* stream) {
     return bitlinear_quantize_act_layout(X, M, K, eps, xq_out, s_out, BL_XQ_ROWMAJOR, stream);

@@ -26,6 +26,12 @@ enum XqLayout : int { kXqRowMajor = 0, kXqEvenOdd16 = 1, kXqStride4K16 = 2 };
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,
                                 float* s, int layout, cudaStream_t stream);
 
+// RMSNorm (kind 0) or LayerNorm (kind 1), optional per-channel weight, then the per-token
+// quantiser; K % 8 == 0 (K % 16 == 0 for the k16 layouts).
+cudaError_t launch_norm_quantize_act(const uint16_t* X, const float* norm_weight, int64_t M, int64_t K, int kind,
+                                     float norm_eps, float eps, int8_t* xq, float* s, int layout,
+                                     cudaStream_t stream);
+
 // Output kinds (mirror bl_dtype).
 enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
 

@@ -341,6 +341,150 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
     }
 }
 
+// ------------------------------------ normalisation + activation quantisation --
+// Quant(LN(x)) ("1-bit & Ternary LLMs (BitNet b1.58)", block "BitNet (Oct 2023)": the
+// LayerNorm in front of the quantiser; the b1.58 models use RMSNorm):
+//   kind 0 (RMSNorm): mu = 0;   kind 1 (LayerNorm): mu = sum(x) / K
+//   v = sum((x - mu)^2) / K;  r = 1 / sqrt(v + norm_eps);  x_n = (x - mu) r w   (fp64)
+//   x_n rounded once to fp32, then s = 127 / max(max |x_n|, eps), x_q = rint(x_n s).
+// One group of G threads per row; each thread keeps its first units of the row in
+// registers across the passes (mean, variance, absmax of x_n, quantise + store) and
+// re-reads the rest through L1.  Sums run in fp64 (a different order than a sequential
+// sum changes them by ~1e-16 relative, which reaches x_n only when it sits that close
+// to an fp32 rounding boundary).
+
+// bf16 element i (0 .. 8U-1) of a unit, as fp32 (exact)
+template <int U>
+__device__ __forceinline__ float unit_elem(const Unit<U>& u, int i) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(&u.v[0]);
+    const uint32_t x = w[i >> 1];
+    return __uint_as_float((i & 1) ? (x & 0xFFFF0000u) : (x << 16));
+}
+
+__device__ __forceinline__ uint32_t pack4_q(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
+    return __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
+}
+
+// int8 bit patterns (low bytes of q[]) of a unit's E elements, stored in layout L
+template <int L>
+__device__ __forceinline__ void store_q(uint8_t* qrow, int idx, const uint32_t (&q)[8 * kUnitVecs<L>]) {
+    if constexpr (L == kXqRowMajor) {
+        reinterpret_cast<uint2*>(qrow)[idx] = make_uint2(pack4_q(q[0], q[1], q[2], q[3]), pack4_q(q[4], q[5], q[6], q[7]));
+    } else if constexpr (L == kXqEvenOdd16) {
+        reinterpret_cast<uint4*>(qrow)[idx] =
+            make_uint4(pack4_q(q[0], q[2], q[4], q[6]), pack4_q(q[8], q[10], q[12], q[14]),
+                       pack4_q(q[1], q[3], q[5], q[7]), pack4_q(q[9], q[11], q[13], q[15]));
+    } else {
+        reinterpret_cast<uint4*>(qrow)[idx] =
+            make_uint4(pack4_q(q[0], q[4], q[8], q[12]), pack4_q(q[1], q[5], q[9], q[13]),
+                       pack4_q(q[2], q[6], q[10], q[14]), pack4_q(q[3], q[7], q[11], q[15]));
+    }
+}
+
+template <int G, int L, int KIND>
+__global__ void __launch_bounds__(G > 256 ? G : 256)
+    norm_act_quant_kernel(const uint4* __restrict__ X, const float* __restrict__ nw, int64_t M, int K,
+                          float norm_eps, float eps, uint8_t* __restrict__ xq, float* __restrict__ s_out) {
+    pdl_wait_then_release();
+    constexpr int U = kUnitVecs<L>;
+    constexpr int E = 8 * U;  // elements per unit
+    constexpr int CTA = G > 256 ? G : 256;
+    constexpr int RPC = CTA / G;  // rows per block
+    constexpr int WPG = G / 32;   // warps per row group
+    constexpr int NV = 8 / U;     // units kept in registers
+    __shared__ double red_d[CTA / 32];
+    __shared__ float red_f[CTA / 32];
+
+    const int sub = threadIdx.x / G;
+    const int j = threadIdx.x % G;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nunit = K / E;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + sub;
+    const bool active = row < M;
+    const uint4* xr = X + (active ? row : 0) * (K / 8);
+
+    Unit<U> v[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int idx = j + u * G;
+        if (active && idx < nunit) {
+            v[u] = load_unit<U>(xr, idx);
+        } else {
+#pragma unroll
+            for (int i = 0; i < U; ++i) v[u].v[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+    // every unit of this thread's share of the row: the cached ones, then the rest
+    auto for_units = [&](auto&& fn) {
+#pragma unroll
+        for (int u = 0; u < NV; ++u)
+            if (j + u * G < nunit) fn(j + u * G, v[u]);
+        for (int idx = j + NV * G; active && idx < nunit; idx += G) fn(idx, load_unit<U>(xr, idx));
+    };
+    auto group_sum = [&](double x) {
+        for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if constexpr (WPG > 1) {
+            __syncthreads();
+            if (lane == 0) red_d[wid] = x;
+            __syncthreads();
+            x = 0.0;
+#pragma unroll
+            for (int w = 0; w < WPG; ++w) x += red_d[sub * WPG + w];
+        }
+        return x;
+    };
+    auto group_max = [&](float x) {
+        for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+        if constexpr (WPG > 1) {
+            __syncthreads();
+            if (lane == 0) red_f[wid] = x;
+            __syncthreads();
+            x = 0.0f;
+#pragma unroll
+            for (int w = 0; w < WPG; ++w) x = fmaxf(x, red_f[sub * WPG + w]);
+        }
+        return x;
+    };
+
+    double mu = 0.0;
+    if constexpr (KIND == 1) {
+        double sx = 0.0;
+        for_units([&](int, const Unit<U>& un) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) sx += static_cast<double>(unit_elem(un, i));
+        });
+        mu = group_sum(sx) / static_cast<double>(K);
+    }
+    double sd = 0.0;
+    for_units([&](int, const Unit<U>& un) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const double d = static_cast<double>(unit_elem(un, i)) - mu;
+            sd += d * d;
+        }
+    });
+    const double r = 1.0 / sqrt(group_sum(sd) / static_cast<double>(K) + static_cast<double>(norm_eps));
+    auto xn_of = [&](int idx, const Unit<U>& un, int i) {
+        const double wk = nw != nullptr ? static_cast<double>(__ldg(nw + idx * E + i)) : 1.0;
+        return __double2float_rn((static_cast<double>(unit_elem(un, i)) - mu) * r * wk);
+    };
+    float am = 0.0f;
+    for_units([&](int idx, const Unit<U>& un) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) am = fmaxf(am, fabsf(xn_of(idx, un, i)));
+    });
+    const float s = __fdiv_rn(127.0f, fmaxf(group_max(am), eps));
+    if (!active) return;
+    if (j == 0) s_out[row] = s;
+    uint8_t* qrow = xq + row * K;
+    for_units([&](int idx, const Unit<U>& un) {
+        uint32_t q[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) q[i] = q8_bits(xn_of(idx, un, i), s);
+        store_q<L>(qrow, idx, q);
+    });
+}
+
 // Any K: one warp per row, scalar loads.
 __global__ void __launch_bounds__(256) act_quant_scalar_kernel(const uint16_t* __restrict__ X,
                                                               int64_t M, int64_t K, float eps,
@@ -418,6 +562,40 @@ static cudaError_t launch_act_vec(const uint4* X4, int64_t M, int K, float eps, 
     if (nvec <= 512) return launch_act_g<128, 1, L>(X4, M, K, eps, xq, s, stream);
     if (nvec <= 1024) return launch_act_g<256, 1, L>(X4, M, K, eps, xq, s, stream);
     return launch_act_g<512, 1, L>(X4, M, K, eps, xq, s, stream);
+}
+
+template <int G, int L>
+static cudaError_t launch_norm_g(const uint4* X4, const float* nw, int64_t M, int K, int kind, float norm_eps,
+                                 float eps, uint8_t* xq, float* s, cudaStream_t stream) {
+    constexpr int CTA = G > 256 ? G : 256;
+    const dim3 grid(grid_for(M, CTA / G, 1 << 30)), block(CTA);
+    if (kind == 1)
+        return launch_pdl(norm_act_quant_kernel<G, L, 1>, grid, block, 0, stream, dim3(kNoCluster), X4, nw, M, K,
+                          norm_eps, eps, xq, s);
+    return launch_pdl(norm_act_quant_kernel<G, L, 0>, grid, block, 0, stream, dim3(kNoCluster), X4, nw, M, K,
+                      norm_eps, eps, xq, s);
+}
+
+template <int L>
+static cudaError_t launch_norm_l(const uint4* X4, const float* nw, int64_t M, int K, int kind, float norm_eps,
+                                 float eps, uint8_t* xq, float* s, cudaStream_t stream) {
+    const int nvec = K / 8;  // 16-byte vectors per row; a thread holds 8 of them
+    if (nvec <= 8 * 32) return launch_norm_g<32, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+    if (nvec <= 8 * 64) return launch_norm_g<64, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+    if (nvec <= 8 * 128) return launch_norm_g<128, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+    if (nvec <= 8 * 256) return launch_norm_g<256, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+    return launch_norm_g<512, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+}
+
+cudaError_t launch_norm_quantize_act(const uint16_t* X, const float* norm_weight, int64_t M, int64_t K, int kind,
+                                     float norm_eps, float eps, int8_t* xq, float* s, int layout,
+                                     cudaStream_t stream) {
+    uint8_t* q = reinterpret_cast<uint8_t*>(xq);
+    const uint4* X4 = reinterpret_cast<const uint4*>(X);
+    const int k = static_cast<int>(K);
+    if (layout == kXqEvenOdd16) return launch_norm_l<kXqEvenOdd16>(X4, norm_weight, M, k, kind, norm_eps, eps, q, s, stream);
+    if (layout == kXqStride4K16) return launch_norm_l<kXqStride4K16>(X4, norm_weight, M, k, kind, norm_eps, eps, q, s, stream);
+    return launch_norm_l<kXqRowMajor>(X4, norm_weight, M, k, kind, norm_eps, eps, q, s, stream);
 }
 
 cudaError_t launch_quantize_act(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq,

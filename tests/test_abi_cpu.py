@@ -114,6 +114,16 @@ def test_other_entry_points_validation(L):
     # stride-4 x_q on a forced tensor-core path needs K <= 2^17
     for p in (2, 3, 4):
         assert lay(FAKE, FAKE, FAKE, FAKE, 40, 8, (1 << 17) + 64, FAKE, 0, None, 2, p, None) == SHAPE
+    nq = L.bitlinear_norm_quantize_act
+    assert nq(None, None, 4, 64, 0, 1e-5, 1e-5, FAKE, FAKE, 0, None) == INVALID
+    assert nq(FAKE, None, 4, 64, 2, 1e-5, 1e-5, FAKE, FAKE, 0, None) == INVALID        # unknown norm kind
+    assert nq(FAKE, None, 4, 64, 0, -1.0, 1e-5, FAKE, FAKE, 0, None) == INVALID        # norm_eps < 0
+    assert nq(FAKE, None, 4, 64, 1, 1e-5, 0.0, FAKE, FAKE, 0, None) == INVALID         # eps <= 0
+    assert nq(FAKE, None, 4, 64, 0, 1e-5, 1e-5, FAKE, FAKE, 3, None) == INVALID        # unknown layout
+    assert nq(FAKE, None, 4, 60, 0, 1e-5, 1e-5, FAKE, FAKE, 0, None) == SHAPE          # K % 8
+    assert nq(FAKE, None, 4, 40, 1, 1e-5, 1e-5, FAKE, FAKE, 2, None) == SHAPE          # k16 layout needs K % 16
+    assert nq(ODD, None, 4, 64, 0, 1e-5, 1e-5, FAKE, FAKE, 0, None) == MISALIGNED
+    assert nq(FAKE, ODD, 4, 64, 0, 1e-5, 1e-5, FAKE, FAKE, 0, None) == MISALIGNED      # norm weight
     qa = L.bitlinear_quantize_act_layout
     assert qa(FAKE, 4, 24, 1e-5, FAKE, FAKE, 1, None) == SHAPE
     assert qa(FAKE, 4, 24, 1e-5, FAKE, FAKE, 2, None) == SHAPE

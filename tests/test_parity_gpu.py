@@ -514,3 +514,71 @@ def test_forward_stride4_wide_layer_repeated(M):
         acc = B.forward(xq, s, packed, gamma, torch.int32, path=B.BL_PATH_GEMV, layout=B.BL_XQ_K16_STRIDE4)
         sync()
         assert np.array_equal(acc.cpu().numpy(), acc_ref)
+
+
+# ------------------------------------- normalisation fused into the quantiser --
+
+NORM_SHAPES = [(1, 16), (3, 40), (5, 1536), (33, 4096), (4096, 1536), (7, 8192), (3, 28672), (2, 36000)]
+
+
+@pytest.mark.parametrize("M,K", NORM_SHAPES)
+@pytest.mark.parametrize("kind", [B.BL_NORM_RMS, B.BL_NORM_LAYER], ids=["rms", "layer"])
+def test_norm_quantize_act(M, K, kind):
+    X = synth.activations(M, K, seed=M + 3 * K + kind, outlier_frac=0.01, outlier_scale=20.0)
+    if kind == B.BL_NORM_LAYER:
+        X = (X.float() + 0.75).to(torch.bfloat16)  # a nonzero mean for LayerNorm to remove
+    w = torch.from_numpy(np.random.default_rng(M + K).uniform(0.5, 1.5, size=K).astype(np.float32))
+    layouts = [B.BL_XQ_ROWMAJOR] + ([B.BL_XQ_K16_EVENODD, B.BL_XQ_K16_STRIDE4] if K % 16 == 0 else [])
+    for weight in (None, w):
+        xq_ref, s_ref, _ = oracle.norm_quantize_act(bits(X), None if weight is None else weight.numpy(), kind,
+                                                    1e-5, EPS)
+        for lay in layouts:
+            xq = guarded_empty((M, K), torch.int8)
+            s = guarded_empty((M,), torch.float32)
+            B.bitlinear_norm_quantize_act(X.to(DEV), None if weight is None else weight.to(DEV), kind, 1e-5, EPS,
+                                          xq, s, layout=lay)
+            sync()
+            check_guard(xq)
+            check_guard(s)
+            assert np.array_equal(s.cpu().numpy(), s_ref), (kind, lay, weight is None)
+            pos = {B.BL_XQ_ROWMAJOR: np.arange(K), B.BL_XQ_K16_EVENODD: None, B.BL_XQ_K16_STRIDE4: None}[lay]
+            if lay == B.BL_XQ_K16_EVENODD:
+                pos = evenodd_positions(K)
+            elif lay == B.BL_XQ_K16_STRIDE4:
+                pos = stride4_positions(K)
+            assert np.array_equal(xq.cpu().numpy()[:, pos], xq_ref), (kind, lay, weight is None)
+
+
+def test_norm_quantize_act_edge_rows():
+    """Zero tokens, a constant token and tiny tokens (norm_eps dominates)."""
+    M, K = 6, 256
+    X = synth.activations(M, K, seed=5).float()
+    X[0] = 0.0
+    X[1] = 3.0
+    X[2] *= 1e-6
+    X = X.to(torch.bfloat16)
+    for kind in (B.BL_NORM_RMS, B.BL_NORM_LAYER):
+        xq_ref, s_ref, _ = oracle.norm_quantize_act(bits(X), None, kind, 1e-5, EPS)
+        xq, s = B.norm_quantize_act(X.to(DEV), None, kind, 1e-5, EPS)
+        sync()
+        assert np.array_equal(s.cpu().numpy(), s_ref) and np.array_equal(xq.cpu().numpy(), xq_ref), kind
+
+
+def test_norm_quantize_then_forward():
+    """The fused quantiser feeding the forward, against the same two oracle steps."""
+    M, N, K = 8, 2400, 1024
+    X = synth.activations(M, K, seed=9, outlier_frac=0.01, outlier_scale=20.0)
+    W = synth.weight(N, K, seed=9)
+    w = torch.from_numpy(np.random.default_rng(9).uniform(0.5, 1.5, size=K).astype(np.float32))
+    g_ref, _, packed_ref = oracle.quantize_weights(W.numpy(), EPS)
+    xq_ref, s_ref, _ = oracle.norm_quantize_act(bits(X), w.numpy(), B.BL_NORM_RMS, 1e-5, EPS)
+    acc_ref = oracle.forward(xq_ref, s_ref, packed_ref, g_ref, K, oracle.OUT_I32)
+    y_ref = oracle.dequant(acc_ref, s_ref, g_ref)
+    xq, s = B.norm_quantize_act(X.to(DEV), w.to(DEV), B.BL_NORM_RMS, 1e-5, EPS, layout=B.BL_XQ_K16_STRIDE4)
+    pk = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    acc = B.forward(xq, s, pk, gamma, torch.int32, layout=B.BL_XQ_K16_STRIDE4)
+    y = B.forward(xq, s, pk, gamma, torch.float32, layout=B.BL_XQ_K16_STRIDE4)
+    sync()
+    assert np.array_equal(acc.cpu().numpy(), acc_ref)
+    assert_float_close(y.cpu().numpy(), y_ref, "norm + forward fp32")
