@@ -50,6 +50,8 @@ class Oracle:
         L.oracle_dequant.argtypes = [P, P, F, I, I, P]
         L.oracle_dequant.restype = None
         L.oracle_f32_to_bf16.argtypes = [P, I, P]
+        L.oracle_dequant_rows.argtypes = [P, P, P, I, I, P]
+        L.oracle_dequant_rows.restype = None
         L.oracle_f32_to_bf16.restype = None
         L.oracle_forward.argtypes = [P, P, P, F, I, I, I, ctypes.c_int, P, P, P, P]
         L.oracle_forward.restype = I
@@ -141,6 +143,16 @@ class Oracle:
         self.L.oracle_dequant(pa, ps, float(gamma), M, N, _vp(y))
         return y
 
+    def dequant_rows(self, acc, s, gamma_rows):
+        """y = acc * gamma_n / s_m with one gamma per output row (oracle_dequant_rows)."""
+        acc, pa = _c(acc, np.int32)
+        M, N = acc.shape
+        s, ps = _c(np.asarray(s, dtype=np.float32).reshape(M), np.float32)
+        g, pg = _c(np.asarray(gamma_rows, dtype=np.float32).reshape(N), np.float32)
+        y = np.empty((M, N), dtype=np.float32)
+        self.L.oracle_dequant_rows(pa, ps, pg, M, N, _vp(y))
+        return y
+
     def f32_to_bf16(self, y):
         """Round fp32 to bf16 bits, nearest-even (oracle_f32_to_bf16)."""
         y, p = _c(y, np.float32)
@@ -186,6 +198,7 @@ def quantize_act(X_bits, eps): return default().quantize_act(X_bits, eps)
 def norm_quantize_act(X_bits, w, kind, norm_eps, eps): return default().norm_quantize_act(X_bits, w, kind, norm_eps, eps)
 def int_matmul(xq, codes): return default().int_matmul(xq, codes)
 def dequant(acc, s, gamma): return default().dequant(acc, s, gamma)
+def dequant_rows(acc, s, gamma_rows): return default().dequant_rows(acc, s, gamma_rows)
 def f32_to_bf16(y): return default().f32_to_bf16(y)
 def forward(xq, s, packed, gamma, K, out_kind=OUT_F32):
     return default().forward(xq, s, packed, gamma, K, out_kind)

@@ -239,6 +239,18 @@ void oracle_dequant(const int32_t *acc, const float *s, float gamma, int64_t M, 
             y[m * N + n] = (float)((double)acc[m * N + n] * (double)gamma / (double)s[m]);
 }
 
+/* The rescale with one weight scale per output row, for several matrices stacked
+ * along N (each keeps its own absmean gamma, [B158]): y[m][n] = acc[m][n] * gamma_n / s[m],
+ * evaluated in double and rounded once to fp32, as in oracle_dequant. */
+void oracle_dequant_rows(const int32_t *acc, const float *s, const float *gamma_rows, int64_t M, int64_t N,
+                         float *y)
+{
+    int64_t m, n;
+    for (m = 0; m < M; ++m)
+        for (n = 0; n < N; ++n)
+            y[m * N + n] = (float)((double)acc[m * N + n] * (double)gamma_rows[n] / (double)s[m]);
+}
+
 /* fp32 -> bf16 with round to nearest, ties to even (finite inputs). */
 void oracle_f32_to_bf16(const float *y, int64_t n, uint16_t *out)
 {

@@ -372,12 +372,26 @@ def pin_norm_invariants(O):
         assert np.all(s == np.float32(127.0) / np.float32(EPS))
 
 
+def pin_dequant_rows(O):
+    """One gamma per output row: the hand case acc = [10, -4], s = 2, gamma = (0.5, 0.25)
+    gives y = 10 * 0.5 / 2 = 2.5 and -4 * 0.25 / 2 = -0.5; with every row's gamma equal
+    it is the single-gamma rescale, bit for bit."""
+    y = O.dequant_rows(np.array([[10, -4]], dtype=np.int32), np.array([2.0], dtype=np.float32),
+                       np.array([0.5, 0.25], dtype=np.float32))
+    assert np.array_equal(y, np.array([[2.5, -0.5]], dtype=np.float32)), y
+    rng = np.random.default_rng(11)
+    acc = rng.integers(-50000, 50000, size=(7, 33)).astype(np.int32)
+    s = rng.uniform(0.5, 200.0, size=7).astype(np.float32)
+    g = np.float32(0.0173)
+    assert np.array_equal(O.dequant_rows(acc, s, np.full(33, g, dtype=np.float32)), O.dequant(acc, s, g))
+
+
 def _bf16_to_f32(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
 ALL_PINS = [
-    pin_hand_norm, pin_norm_vs_torch, pin_norm_invariants,
+    pin_hand_norm, pin_norm_vs_torch, pin_norm_invariants, pin_dequant_rows,
     pin_hand_ternarise, pin_hand_absmean, pin_hand_act, pin_hand_pack, pin_hand_matmul,
     pin_gaussian_statistics, pin_constant_magnitude, pin_zero_weights, pin_zero_token,
     pin_code_alphabet_and_sign_symmetry, pin_act_range_and_symmetry,
