@@ -244,6 +244,19 @@ BL_API bl_status bitlinear_forward_layout(const int8_t *xq, const float *s, cons
                                           bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,
                                           bl_path path, void *stream);
 
+/* bitlinear_forward_layout with one weight scale per output row, for several BitLinear
+ * matrices stacked along N (q/k/v, or up/gate) that keep their own absmean gamma
+ * ([B158]: gamma is a per-matrix mean), run as one launch:
+ *   y[m, n] = float(acc[m, n]) * (gamma_rows[n] / s[m])
+ *   gamma_rows in : fp32 [N], device, 16-byte aligned; every other argument, result
+ *                   and error as for bitlinear_forward_layout (BL_OUT_I32 ignores it).
+ * Stack the packed rows of the matrices and fill gamma_rows with each matrix's gamma
+ * repeated over its rows. */
+BL_API bl_status bitlinear_forward_rowscale(const int8_t *xq, const float *s, const uint8_t *packed,
+                                            const float *gamma_rows, int64_t M, int64_t N, int64_t K, void *out,
+                                            bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,
+                                            bl_path path, void *stream);
+
 /* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
 BL_API int bitlinear_last_cuda_error(void);
 

@@ -31,7 +31,8 @@ EXPORTED = [
     "bitlinear_workspace_size", "bitlinear_quantize_weights",
     "bitlinear_quantize_weights_with_scale", "bitlinear_pack", "bitlinear_quantize_act",
     "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
-    "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_last_cuda_error",
+    "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_forward_rowscale",
+    "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
 
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_quantize_act_layout.restype = S
         L.bitlinear_forward_layout.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, S, P]
         L.bitlinear_forward_layout.restype = S
+        L.bitlinear_forward_rowscale.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, S, P]
+        L.bitlinear_forward_rowscale.restype = S
         L.bitlinear_norm_quantize_act.argtypes = [P, P, I64, I64, S, F, F, P, P, S, P]
         L.bitlinear_norm_quantize_act.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
@@ -182,6 +185,20 @@ def bitlinear_forward(xq, s, packed, gamma, out, err_word=None, stream=None, pat
         _check(lib().bitlinear_forward(*args, _stream(stream)), "bitlinear_forward")
     else:
         _check(lib().bitlinear_forward_path(*args, int(path), _stream(stream)), "bitlinear_forward_path")
+
+
+def bitlinear_forward_rowscale(xq, s, packed, gamma_rows, out, err_word=None, stream=None, path=BL_PATH_AUTO,
+                               layout=BL_XQ_ROWMAJOR):
+    M, K = xq.shape
+    N = packed.shape[0]
+    kind = {v: k for k, v in _OUT_DT.items()}.get(out.dtype)
+    if kind is None:
+        raise TypeError("out must be float32, bfloat16 or int32")
+    _check(lib().bitlinear_forward_rowscale(
+        _dev(xq, torch.int8, "xq"), _dev(s, torch.float32, "s", (M,)),
+        _dev(packed, torch.uint8, "packed", (N, K // 4)), _dev(gamma_rows, torch.float32, "gamma_rows", (N,)),
+        M, N, K, _dev(out, out.dtype, "out", (M, N)), kind, _opt(err_word, "err_word"), int(layout), int(path),
+        _stream(stream)), "bitlinear_forward_rowscale")
 
 
 # ----------------------------------------------------------- allocating helpers --

@@ -123,9 +123,9 @@ bl_status bitlinear_quantize_act(const uint16_t* X, int64_t M, int64_t K, float 
     return bitlinear_quantize_act_layout(X, M, K, eps, xq_out, s_out, BL_XQ_ROWMAJOR, stream);
 }
 
-bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
-                                   int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
-                                   int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
+static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma, int64_t M,
+                              int64_t N, int64_t K, void* out, bl_dtype out_dtype, int32_t* err_word,
+                              bl_xq_layout xq_layout, bl_path path, bool gamma_per_row, void* stream) {
     if (xq == nullptr || s == nullptr || packed == nullptr || gamma == nullptr || out == nullptr)
         return BL_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
@@ -149,7 +149,8 @@ bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8
     const bool s4_big = xq_layout == BL_XQ_K16_STRIDE4 && K > (int64_t(1) << 17);
     if (tc && s4_big) return BL_ERR_UNSUPPORTED_SHAPE;
     if (path == BL_PATH_AUTO) path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : BL_PATH_TC;
-    const int kind = static_cast<int>(out_dtype);
+    if (gamma_per_row && !aligned16(gamma)) return BL_ERR_MISALIGNED;
+    const int kind = static_cast<int>(out_dtype) | (gamma_per_row ? bl::kGammaPerRow : 0);
     const int lay = static_cast<int>(xq_layout);
     cudaStream_t st = as_stream(stream);
     cudaError_t e;
@@ -165,6 +166,18 @@ bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8
         e = bl::launch_gemv_generic(xq, s, packed, gamma, M, N, K, out, kind, lay, st);
     }
     return cuda_status(e);
+}
+
+bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                                   int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                   int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
+    return forward_impl(xq, s, packed, gamma, M, N, K, out, out_dtype, err_word, xq_layout, path, false, stream);
+}
+
+bl_status bitlinear_forward_rowscale(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma_rows,
+                                     int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                     int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
+    return forward_impl(xq, s, packed, gamma_rows, M, N, K, out, out_dtype, err_word, xq_layout, path, true, stream);
 }
 
 bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,

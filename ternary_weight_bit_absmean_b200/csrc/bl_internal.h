@@ -34,6 +34,11 @@ cudaError_t launch_norm_quantize_act(const uint16_t* X, const float* norm_weight
 
 // Output kinds (mirror bl_dtype).
 enum OutKind : int { kOutF32 = 0, kOutBF16 = 1, kOutI32 = 2 };
+// The forward launchers' `kind` may also carry kGammaPerRow: gamma then points to N
+// weight scales, one per output row, instead of one.
+constexpr int kGammaPerRow = 0x100;
+inline int out_kind_of(int kind) { return kind & 0xFF; }
+inline int gamma_rows_of(int kind) { return (kind & kGammaPerRow) ? 1 : 0; }
 
 // Decode GEMV: register unpack + mma.sync, any M (token groups of 16), K % 64 == 0.
 // With x_q in the stride-4 k16 layout and a shape gemv_tma_applicable accepts, it runs

@@ -79,6 +79,7 @@ struct TcArgs {
     int kind;
     int32_t* err;
     S4Mul mul;
+    int grow;  // gamma holds one scale per output row
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -300,9 +301,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row = n0 + 32 * q + lane;
             const bool row_ok = row < a.N;
+            // with one scale per output row, this thread's row scale
+            const float grow_gamma = (a.grow && a.kind != kOutI32 && row_ok) ? __ldg(a.gamma + row) : 0.0f;
 #pragma unroll 1
             for (int c0 = first; c0 < BT; c0 += 64) {
-                const float fac = __fdiv_rn(gamma, s_next);
+                const float s_cur = s_next;
+                const float fac = __fdiv_rn(gamma, s_cur);
                 const int tk = t0 + c0 + 64 + lane;
                 if (c0 + 64 < BT) s_next = (a.kind != kOutI32 && tk < a.M) ? __ldg(a.s + tk) : 1.0f;
                 uint32_t r[32];
@@ -312,7 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float fj = __shfl_sync(0xffffffffu, fac, j);
+                    const float fj = a.grow ? __fdiv_rn(grow_gamma, __shfl_sync(0xffffffffu, s_cur, j))
+                                            : __shfl_sync(0xffffffffu, fac, j);
                     const int tok = t0 + c0 + j;
                     if (tok < a.M && row_ok)
                         store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
@@ -466,7 +471,7 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     int64_t cost = 0;
     const int bt = tc1_tile(M, N, K, sms, &cost);
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
-             0, out, kind, err, s4_mul()};
+             0, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
     switch (layout) {
         case kXqEvenOdd16: return launch_bt_layout<kXqEvenOdd16>(bt, xq, packed, a, sms, stream);

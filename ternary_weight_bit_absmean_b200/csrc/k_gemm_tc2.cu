@@ -63,6 +63,7 @@ struct Tc2Args {
     int kind;
     int32_t* err;
     S4Mul mul;
+    int grow;  // gamma holds one scale per output row
 };
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -337,7 +338,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) >> 6);
                 }
-                if (tok_ok && n0 + c0 < a.N) store_row32(a.out, a.kind, row_off, n0 + c0, a.N, r, fac, vec_ok);
+                if (!tok_ok || n0 + c0 >= a.N) {
+                    // nothing of this chunk to store for this lane
+                } else if (a.grow && a.kind != kOutI32) {
+                    // one scale per output row: y = acc * (gamma_f / s), element stores
+                    const float st = __ldg(a.s + tok);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int f = n0 + c0 + j;
+                        if (f >= a.N) break;
+                        const float y = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), __fdiv_rn(__ldg(a.gamma + f), st));
+                        if (a.kind == kOutF32)
+                            static_cast<float*>(a.out)[row_off + f] = y;
+                        else
+                            static_cast<__nv_bfloat16*>(a.out)[row_off + f] = __float2bfloat16_rn(y);
+                    }
+                } else {
+                    store_row32(a.out, a.kind, row_off, n0 + c0, a.N, r, fac, vec_ok);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -399,7 +417,7 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
         return cudaErrorInvalidValue;
     Tc2Args a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
               static_cast<int>((N + 255) / 256), static_cast<int>(((N + 255) / 256) * ((M + 255) / 256)),
-              out, kind, err, s4_mul()};
+              out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
     const int clusters = gemm_tc2_clusters(M, N, sms);
     switch (layout) {
         case kXqEvenOdd16: return launch_tc2_layout<kXqEvenOdd16>(tx, tp, a, clusters, stream);

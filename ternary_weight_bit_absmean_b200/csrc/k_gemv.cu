@@ -52,6 +52,7 @@ struct GemvArgs {
     int kind;
     uint32_t mul2, mul16;  // 2^30 and 2^16: right shifts by 2 and 16 as high-half multiplies
     int layout;            // XqLayout of x_q
+    int grow;              // gamma holds one scale per output row
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -314,7 +315,9 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int64_t row = row0 + 16 * tile + g + 8 * h;
-                        if (row < a.N) store_y(a.out, a.kind, tok * a.N + row, acc[tile][j][2 * h + e], fac);
+                        if (row >= a.N) continue;
+                        const float f = (a.grow && a.kind != kOutI32) ? __fdiv_rn(a.gamma[row], a.s[tok]) : fac;
+                        store_y(a.out, a.kind, tok * a.N + row, acc[tile][j][2 * h + e], f);
                     }
                 }
             }
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(kGvThreads, 2) gemv_kernel(GemvArgs a) {
         const int64_t tok = m0 + idx / kGvRows;
         const int64_t row = static_cast<int64_t>(blockIdx.x) * kGvRows + idx % kGvRows;
         if (tok < a.M && row < a.N) {
-            const float fac = (a.kind == kOutI32) ? 0.0f : __fdiv_rn(gamma, a.s[tok]);
+            const float fac = (a.kind == kOutI32) ? 0.0f : __fdiv_rn(a.grow ? a.gamma[row] : gamma, a.s[tok]);
             store_y(a.out, a.kind, tok * a.N + row, sum, fac);
         }
     }
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(256) gemv_generic_kernel(GemvArgs a) {
             acc += c == 1u ? xv : (c == 2u ? -xv : 0);
         }
     }
-    const float fac = (a.kind == kOutI32) ? 0.0f : __fdiv_rn(*a.gamma, a.s[m]);
+    const float fac = (a.kind == kOutI32) ? 0.0f : __fdiv_rn(a.grow ? a.gamma[n] : *a.gamma, a.s[m]);
     store_y(a.out, a.kind, idx, acc, fac);
 }
 
@@ -413,6 +416,8 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
                         cudaStream_t stream) {
     if (layout == kXqStride4K16 && gemv_tma_applicable(M, N, K))
         return launch_gemv_tma(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
+    const int grow = gamma_rows_of(kind);
+    kind = out_kind_of(kind);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -443,7 +448,7 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
     int64_t Kc = ((K + S - 1) / S + kChunk - 1) / kChunk * kChunk;
     S = (K + Kc - 1) / Kc;
     GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(Kc), 0, out, kind, 1u << 30, 1u << 16,
-               layout};
+               layout, grow};
     const int Si = static_cast<int>(S);
     if (MT == 1) {
         if (layout == kXqEvenOdd16) return launch_gemv_mt<1, kXqEvenOdd16>(a, Si, row_blocks, token_blocks, stream);
@@ -458,8 +463,8 @@ cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                                 int kind, int layout, cudaStream_t stream) {
-    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, kind, 1u << 30, 1u << 16,
-               layout};
+    GemvArgs a{xq, s, packed, gamma, M, N, static_cast<int>(K), static_cast<int>(K), 0, out, out_kind_of(kind),
+               1u << 30, 1u << 16, layout, gamma_rows_of(kind)};
     const int64_t total = M * N;
     return launch_pdl(gemv_generic_kernel, dim3(static_cast<unsigned>((total + 255) / 256)), dim3(256), 0, stream,
                       dim3(kNoCluster), a);

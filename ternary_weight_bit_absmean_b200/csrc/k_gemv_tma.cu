@@ -62,6 +62,7 @@ struct GtArgs {
     int kind;
     int32_t* err;
     S4Mul mul;
+    int grow;  // gamma holds one scale per output row
 };
 
 __device__ __forceinline__ void store_y1(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -355,9 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int64_t row = row0 + 16 * tile + g + 8 * hh;
-                            if (row < a.N)
-                                store_y1(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
-                                         acc[tile][j][2 * hh + e] >> 6, fac);
+                            if (row >= a.N) continue;
+                            const float f =
+                                (a.grow && a.kind != kOutI32) ? __fdiv_rn(a.gamma[row], a.s[tok]) : fac;
+                            store_y1(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
+                                     acc[tile][j][2 * hh + e] >> 6, f);
                         }
                     }
                 }
@@ -436,7 +439,7 @@ cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* pac
         return cudaErrorInvalidValue;
     const int64_t ntiles = (N + 15) / 16;
     GtArgs a{xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(ntiles),
-             p.stages, p.tile_slots, p.units, p.wpp, out, kind, err, s4_mul()};
+             p.stages, p.tile_slots, p.units, p.wpp, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
     static bool attr_done[2][64] = {};
     const int mi = MT - 1;
     if (dev < 0 || dev >= 64 || !attr_done[mi][dev]) {

@@ -582,3 +582,71 @@ def test_norm_quantize_then_forward():
     sync()
     assert np.array_equal(acc.cpu().numpy(), acc_ref)
     assert_float_close(y.cpu().numpy(), y_ref, "norm + forward fp32")
+
+
+# ------------------------------------- stacked matrices, one scale per output row --
+
+@pytest.mark.parametrize("M,path,layout", [
+    (1, B.BL_PATH_GEMV, B.BL_XQ_K16_STRIDE4), (8, B.BL_PATH_GEMV, B.BL_XQ_ROWMAJOR),
+    (16, B.BL_PATH_GEMV, B.BL_XQ_K16_STRIDE4), (40, B.BL_PATH_GEMV, B.BL_XQ_ROWMAJOR),
+    (300, B.BL_PATH_TC_1SM, B.BL_XQ_K16_STRIDE4), (300, B.BL_PATH_TC_2SM, B.BL_XQ_K16_STRIDE4),
+    (700, B.BL_PATH_TC, B.BL_XQ_ROWMAJOR), (5, B.BL_PATH_AUTO, B.BL_XQ_K16_EVENODD)])
+def test_forward_rowscale_stacked_matrices(M, path, layout):
+    """q, k and v stacked along N (1536 + 512 + 512 rows; the 2560-row stack puts the
+    decode case on the persistent kernel), each with its own absmean gamma: one launch
+    against the oracle's per-row rescale."""
+    K = 1024
+    parts = [synth.weight(n, K, seed=40 + i) for i, n in enumerate((1536, 512, 512))]
+    packs, grows = [], []
+    for W in parts:
+        g, _, p = oracle.quantize_weights(W.numpy(), EPS)
+        packs.append(p)
+        grows.append(np.full(W.shape[0], g, dtype=np.float32))
+    packed_ref = np.concatenate(packs, axis=0)
+    gamma_rows = np.concatenate(grows)
+    N = packed_ref.shape[0]
+    X = synth.activations(M, K, seed=M + 41, outlier_frac=0.01, outlier_scale=20.0)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    acc_ref = oracle.forward(xq_ref, s_ref, packed_ref, 1.0, K, oracle.OUT_I32)
+    y_ref = oracle.dequant_rows(acc_ref, s_ref, gamma_rows)
+    pos = {B.BL_XQ_ROWMAJOR: np.arange(K), B.BL_XQ_K16_EVENODD: evenodd_positions(K),
+           B.BL_XQ_K16_STRIDE4: stride4_positions(K)}[layout]
+    xl = np.empty_like(xq_ref)
+    xl[:, pos] = xq_ref
+    xq = torch.from_numpy(xl).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    pk = torch.from_numpy(packed_ref).to(DEV)
+    gr = torch.from_numpy(gamma_rows).to(DEV)
+    for dt in (torch.int32, torch.float32, torch.bfloat16):
+        out = guarded_empty((M, N), dt)
+        err = torch.zeros(1, dtype=torch.int32, device=DEV)
+        B.bitlinear_forward_rowscale(xq, s, pk, gr, out, err, path=path, layout=layout)
+        sync()
+        check_guard(out)
+        assert err.item() == 0
+        if dt == torch.int32:
+            assert np.array_equal(out.cpu().numpy(), acc_ref)
+        elif dt == torch.float32:
+            assert_float_close(out.cpu().numpy(), y_ref, "rowscale fp32")
+        else:
+            yb = out.view(torch.int16).cpu().numpy().view(np.uint16)
+            assert_bf16_match(yb, y_ref, oracle.f32_to_bf16(y_ref), "rowscale bf16")
+
+
+def test_forward_rowscale_equal_scales_match_single_scale():
+    """With every row's scale equal to gamma, the per-row forward is the single-gamma
+    forward bit for bit, on every path."""
+    M, N, K = 300, 768, 512
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=12)
+    xq = torch.from_numpy(xq_ref).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    pk = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    gr = torch.full((N,), float(g_ref), device=DEV)
+    for path in (B.BL_PATH_GEMV, B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM):
+        a = guarded_empty((M, N), torch.float32)
+        b = guarded_empty((M, N), torch.float32)
+        B.bitlinear_forward(xq, s, pk, gamma, a, path=path)
+        B.bitlinear_forward_rowscale(xq, s, pk, gr, b, path=path)
+        sync()
+        assert torch.equal(a, b), path
