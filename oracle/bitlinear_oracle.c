@@ -160,9 +160,11 @@ void oracle_quantize_act(const uint16_t *X, int64_t M, int64_t K, float eps,
  * RMSNorm among them).  For each token:
  *   kind 0 (RMSNorm):   mu = 0
  *   kind 1 (LayerNorm): mu = (sum_k x_k) / K
- *   v = (sum_k (x_k - mu)^2) / K;   r = 1 / sqrt(v + norm_eps);
- *   x_n[k] = (x_k - mu) * r * w_k   (w = the per-channel norm weight, 1 when absent),
- * every step in double precision, sums in index order, x_n rounded once to fp32.
+ *   v = (sum_k (x_k - mu)^2) / K;   r = 1 / sqrt(v + norm_eps)
+ * with the sums, mu, v and r in double precision (sums in index order); mu and r are
+ * then rounded once to fp32, and each element is normalised in fp32, one IEEE rounding
+ * per operation, left to right:
+ *   x_n[k] = ((x_k - mu) * r) * w_k   (w = the per-channel norm weight, 1 when absent).
  * x_n then goes through the activation quantiser of oracle_quantize_act, in fp32:
  *   a = max_k |x_n[k]|;  s = 127 / max(a, eps);  x_q = clip(round(x_n * s), -128, 127).
  * xn_out (may be NULL) receives x_n. */
@@ -183,11 +185,14 @@ void oracle_norm_quantize_act(const uint16_t *X, const float *w, int64_t M, int6
             v += d * d;
         }
         v = v / (double)K;
-        double r = 1.0 / sqrt(v + (double)norm_eps);
+        const float mu32 = (float)mu;
+        const float r32 = (float)(1.0 / sqrt(v + (double)norm_eps));
         float a = 0.0f;
         for (k = 0; k < K; ++k) {
-            double wk = (w != NULL) ? (double)w[k] : 1.0;
-            xn[k] = (float)(((double)bf16_bits_to_float(X[m * K + k]) - mu) * r * wk);
+            const float wk = (w != NULL) ? w[k] : 1.0f;
+            const float d32 = bf16_bits_to_float(X[m * K + k]) - mu32;
+            const float t32 = d32 * r32;
+            xn[k] = t32 * wk;
             if (fabsf(xn[k]) > a) a = fabsf(xn[k]);
         }
         const float s = 127.0f / fmaxf(a, eps);

@@ -338,8 +338,9 @@ def _torch_norm_quant(xb, w, kind, norm_eps):
 
 def pin_norm_vs_torch(O):
     """torch's rms_norm / layer_norm in float64 then the quantiser in fp32: the scale
-    within 2^-22 (the two sums run in different orders), the codes equal except where
-    x_n s sits within 1e-3 of a rounding midpoint, and those are rare."""
+    within 2^-21 (the oracle normalises each element in fp32, torch in float64), the
+    codes equal except where x_n s sits within 1e-3 of a rounding midpoint, and those
+    are rare."""
     rng = np.random.default_rng(7)
     for kind in (0, 1):
         for with_w in (False, True):
@@ -349,7 +350,7 @@ def pin_norm_vs_torch(O):
             w = (rng.uniform(0.5, 1.5, size=384).astype(np.float32) if with_w else None)
             xq, s, _ = O.norm_quantize_act(xb, w, kind, 1e-5, EPS)
             tq, ts, tv = _torch_norm_quant(xb, w, kind, 1e-5)
-            assert np.all(np.abs(s / ts - 1.0) < 2.0 ** -22), (kind, with_w)
+            assert np.all(np.abs(s / ts - 1.0) < 2.0 ** -21), (kind, with_w)
             frac = np.abs(tv - np.floor(tv) - 0.5)
             differ = xq.astype(np.int64) != tq
             assert np.all(frac[differ] < 1e-3), (kind, with_w)

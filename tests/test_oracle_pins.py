@@ -47,8 +47,9 @@ MUTANTS = [
      "unsigned c = (byte >> (2 * (3 - k % 4))) & 3u;"),
     ("layernorm_no_mean", "mu = mu / (double)K;", "mu = 0.0;"),
     ("norm_variance_unbiased", "v = v / (double)K;", "v = v / (double)(K - 1);"),
-    ("norm_weight_ignored", "double wk = (w != NULL) ? (double)w[k] : 1.0;", "double wk = 1.0;"),
-    ("norm_eps_dropped", "double r = 1.0 / sqrt(v + (double)norm_eps);", "double r = 1.0 / sqrt(v);"),
+    ("norm_weight_ignored", "const float wk = (w != NULL) ? w[k] : 1.0f;", "const float wk = 1.0f;"),
+    ("norm_eps_dropped", "const float r32 = (float)(1.0 / sqrt(v + (double)norm_eps));",
+     "const float r32 = (float)(1.0 / sqrt(v));"),
     ("norm_round_away", "float q = rintf(xn[k] * s);", "float q = roundf(xn[k] * s);"),
     ("norm_qb_128", "const float s = 127.0f / fmaxf(a, eps);", "const float s = 128.0f / fmaxf(a, eps);"),
     ("row_gamma_by_token", "(double)gamma_rows[n] / (double)s[m]", "(double)gamma_rows[m] / (double)s[m]"),
