@@ -168,12 +168,12 @@ typedef enum {
  * RMSNorm).  Per token m:
  *   mu = 0 (BL_NORM_RMS) or sum_k x_mk / K (BL_NORM_LAYER)
  *   v = sum_k (x_mk - mu)^2 / K;   r = 1 / sqrt(v + norm_eps)
- *   x_n = (x_mk - mu) * r * w_k    (w = norm_weight, or 1 when NULL)
- * mu, v, r and the product in double precision, x_n rounded once to fp32; then the
- * quantiser of bitlinear_quantize_act on x_n:
+ * in double precision, then mu and r rounded once to fp32;
+ *   x_n = ((x_mk - mu) * r) * w_k    (fp32, w = norm_weight, or 1 when NULL)
+ * then the quantiser of bitlinear_quantize_act on x_n:
  *   s_m = 127 / max(max_k |x_n|, eps);   x_q = clip(rint(x_n * s_m), -128, 127).
  * The sums run in a parallel order; a sequential sum differs by ~1e-16 relative, which
- * changes x_n only when it lies that close to an fp32 rounding boundary.
+ * changes mu or r only when they lie that close to an fp32 rounding boundary.
  *   X           in  : bf16 [M, K] as raw uint16 bit patterns, device.  Finite values.
  *   norm_weight in  : fp32 [K], device, or NULL.
  *   norm_kind   in  : bl_norm_kind.

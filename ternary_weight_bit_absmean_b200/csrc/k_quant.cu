@@ -345,13 +345,14 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
 // Quant(LN(x)) ("1-bit & Ternary LLMs (BitNet b1.58)", block "BitNet (Oct 2023)": the
 // LayerNorm in front of the quantiser; the b1.58 models use RMSNorm):
 //   kind 0 (RMSNorm): mu = 0;   kind 1 (LayerNorm): mu = sum(x) / K
-//   v = sum((x - mu)^2) / K;  r = 1 / sqrt(v + norm_eps);  x_n = (x - mu) r w   (fp64)
-//   x_n rounded once to fp32, then s = 127 / max(max |x_n|, eps), x_q = rint(x_n s).
+//   v = sum((x - mu)^2) / K;  r = 1 / sqrt(v + norm_eps)      (fp64, then mu and r to fp32)
+//   x_n = ((x - mu) * r) * w   (fp32, one IEEE rounding per operation)
+//   s = 127 / max(max |x_n|, eps),  x_q = rint(x_n s).
 // One group of G threads per row; each thread keeps its first units of the row in
 // registers across the passes (mean, variance, absmax of x_n, quantise + store) and
-// re-reads the rest through L1.  Sums run in fp64 (a different order than a sequential
-// sum changes them by ~1e-16 relative, which reaches x_n only when it sits that close
-// to an fp32 rounding boundary).
+// re-reads the rest through L1.  The sums run in fp64: a different order than a
+// sequential sum changes them by ~1e-16 relative, which reaches mu or r only when they
+// sit that close to an fp32 rounding boundary; the element-wise part has no order.
 
 // bf16 element i (0 .. 8U-1) of a unit, as fp32 (exact)
 template <int U>
@@ -464,9 +465,10 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
         }
     });
     const double r = 1.0 / sqrt(group_sum(sd) / static_cast<double>(K) + static_cast<double>(norm_eps));
+    const float mu32 = __double2float_rn(mu), r32 = __double2float_rn(r);
     auto xn_of = [&](int idx, const Unit<U>& un, int i) {
-        const double wk = nw != nullptr ? static_cast<double>(__ldg(nw + idx * E + i)) : 1.0;
-        return __double2float_rn((static_cast<double>(unit_elem(un, i)) - mu) * r * wk);
+        const float wk = nw != nullptr ? __ldg(nw + idx * E + i) : 1.0f;
+        return __fmul_rn(__fmul_rn(__fsub_rn(unit_elem(un, i), mu32), r32), wk);
     };
     float am = 0.0f;
     for_units([&](int idx, const Unit<U>& un) {
