@@ -1,7 +1,8 @@
 // bl_device.cuh -- device-side building blocks shared by the libbitlinear kernels:
 // inline-PTX wrappers for mbarriers, TMA tensor loads, tcgen05 (TMEM allocation, MMA,
-// commit, loads), the legacy mma.sync used by the decode GEMV, bounded waits, and the
-// two 2-bit -> int8 unpack routines.  Written for sm_100a only.
+// commit, loads), programmatic dependent launch, bounded waits, streaming loads, and
+// the three 2-bit -> int8 unpack routines (natural, even/odd and stride-4 order).
+// Written for sm_100a only.
 #pragma once
 
 #include <cstdint>
@@ -118,16 +119,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-// 4-D tiled bulk tensor load global -> shared::cta (c0 innermost).
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
 
@@ -307,18 +298,6 @@ __device__ __forceinline__ void tc_commit_pair_multicast(uint32_t bar, uint16_t 
         : "memory");
 }
 
-// ------------------------------------------------------------ legacy mma.sync --
-
-// D = A(16x32, row) * B(32x8, col) + C, int8 inputs, int32 accumulate (warp-wide).
-__device__ __forceinline__ void mma_m16n8k32_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                                uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 // ------------------------------------------------------------- global loads --
 
 // Streaming 16-byte load that bypasses L1 (each packed weight byte is read once).
@@ -364,21 +343,6 @@ __device__ __forceinline__ void unpack16_evenodd(uint32_t p, uint32_t& e0, uint3
     e1 = __byte_perm(kCodeTable, 0u, sa >> 16);
     o0 = __byte_perm(kCodeTable, 0u, sb);
     o1 = __byte_perm(kCodeTable, 0u, sb >> 16);
-}
-
-// unpack16_evenodd with its three right shifts done as high-half multiplies by
-// 2^(32 - shift), which run on the FMA pipe instead of the integer ALU pipe.  The
-// multipliers come in as runtime values (mul2 = 2^30, mul16 = 2^16) so that they stay
-// multiplies.
-__device__ __forceinline__ void unpack16_evenodd_fma(uint32_t p, uint32_t mul2, uint32_t mul16,
-                                                     uint32_t& e0, uint32_t& e1, uint32_t& o0,
-                                                     uint32_t& o1) {
-    const uint32_t sa = p & 0x33333333u;
-    const uint32_t sb = __umulhi(p, mul2) & 0x33333333u;
-    e0 = __byte_perm(kCodeTable, 0u, sa);
-    e1 = __byte_perm(kCodeTable, 0u, __umulhi(sa, mul16));
-    o0 = __byte_perm(kCodeTable, 0u, sb);
-    o1 = __byte_perm(kCodeTable, 0u, __umulhi(sb, mul16));
 }
 
 // Runtime multipliers of the stride-4 unpack: passed in as values so that the shifts

@@ -314,14 +314,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        static_cast<uint32_t>(buf * BT + c0),
                                    r);
                 tmem_ld_wait();
+                if (a.grow) {
+                    // one scale per output row: this row's gamma over each token's s
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float fj = a.grow ? __fdiv_rn(grow_gamma, __shfl_sync(0xffffffffu, s_cur, j))
-                                            : __shfl_sync(0xffffffffu, fac, j);
-                    const int tok = t0 + c0 + j;
-                    if (tok < a.M && row_ok)
-                        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
-                                static_cast<int>(r[j]) >> kAccShift, fj);
+                    for (int j = 0; j < 32; ++j) {
+                        const float fj = __fdiv_rn(grow_gamma, __shfl_sync(0xffffffffu, s_cur, j));
+                        const int tok = t0 + c0 + j;
+                        if (tok < a.M && row_ok)
+                            store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
+                                    static_cast<int>(r[j]) >> kAccShift, fj);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float fj = __shfl_sync(0xffffffffu, fac, j);
+                        const int tok = t0 + c0 + j;
+                        if (tok < a.M && row_ok)
+                            store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row,
+                                    static_cast<int>(r[j]) >> kAccShift, fj);
+                    }
                 }
             }
             tc_fence_before();
@@ -371,27 +382,6 @@ bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// uint8 tensor map of any rank (<= 5): dims[0] is the contiguous dimension, strides[i]
-// the byte stride of dims[i + 1].  The strides need not grow with i, so a box can gather
-// a permutation of the tensor's dimensions into shared memory.
-bool encode_tmap_u8(CUtensorMap* map, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides,
-                    const uint32_t* box, bool swizzle128) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
-    if (fn == nullptr || rank < 1 || rank > 5) return false;
-    cuuint64_t d[5], st[4];
-    cuuint32_t b[5], estr[5];
-    for (int i = 0; i < rank; ++i) {
-        d[i] = dims[i];
-        b[i] = box[i];
-        estr[i] = 1;
-        if (i + 1 < rank) st[i] = strides[i];
-    }
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), d, st, b,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 namespace {
