@@ -350,7 +350,10 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
 //   s = 127 / max(max |x_n|, eps),  x_q = rint(x_n s).
 // One group of G threads per row; each thread keeps its first units of the row in
 // registers across the passes (mean, variance, absmax of x_n, quantise + store) and
-// re-reads the rest through L1.  The sums run in fp64: a different order than a
+// re-reads the rest through L1.  The norm weight w is shared by every row: for K up to
+// kNormStageMaxK the block copies it once into shared memory, as the 16-byte chunks of
+// each unit with an XOR swizzle so that a warp's float4 reads of consecutive units hit
+// distinct bank groups (a direct read has the lanes a whole unit apart).  The sums run in fp64: a different order than a
 // sequential sum changes them by ~1e-16 relative, which reaches mu or r only when they
 // sit that close to an fp32 rounding boundary; the element-wise part has no order.
 
@@ -382,13 +385,26 @@ __device__ __forceinline__ void store_q(uint8_t* qrow, int idx, const uint32_t (
     }
 }
 
+constexpr int kNormStageMaxK = 8192;  // K fp32 weights = 32 KB of shared memory, within the default 48 KB
+
+// position of 16-byte chunk c of unit idx in the staged weights (C chunks per unit):
+// 8 lanes with consecutive idx land on the 8 distinct 16-byte bank groups of 128 bytes
+template <int C>
+__device__ __forceinline__ int norm_w_chunk(int idx, int c) {
+    return idx * C + (c ^ ((idx / (8 / C)) & (C - 1)));
+}
+
+extern __shared__ float4 norm_w_sm[];
+
 template <int G, int L, int KIND>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     norm_act_quant_kernel(const uint4* __restrict__ X, const float* __restrict__ nw, int64_t M, int K,
-                          float norm_eps, float eps, uint8_t* __restrict__ xq, float* __restrict__ s_out) {
+                          float norm_eps, float eps, uint8_t* __restrict__ xq, float* __restrict__ s_out,
+                          int stage_w) {
     pdl_wait_then_release();
     constexpr int U = kUnitVecs<L>;
     constexpr int E = 8 * U;  // elements per unit
+    constexpr int C = E / 4;  // 16-byte weight chunks per unit
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G;  // rows per block
     constexpr int WPG = G / 32;   // warps per row group
@@ -414,6 +430,13 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
 #pragma unroll
             for (int i = 0; i < U; ++i) v[u].v[i] = make_uint4(0, 0, 0, 0);
         }
+    }
+    if (stage_w) {
+        // element e of w: chunk e / 4 (unit e / E, chunk (e % E) / 4), word e % 4
+        float* ws = reinterpret_cast<float*>(norm_w_sm);
+        for (int e = threadIdx.x; e < K; e += CTA)
+            ws[4 * norm_w_chunk<C>(e / E, (e % E) / 4) + (e & 3)] = __ldg(nw + e);
+        __syncthreads();
     }
     // every unit of this thread's share of the row: the cached ones, then the rest
     auto for_units = [&](auto&& fn) {
@@ -466,23 +489,42 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
     });
     const double r = 1.0 / sqrt(group_sum(sd) / static_cast<double>(K) + static_cast<double>(norm_eps));
     const float mu32 = __double2float_rn(mu), r32 = __double2float_rn(r);
-    auto xn_of = [&](int idx, const Unit<U>& un, int i) {
-        const float wk = nw != nullptr ? __ldg(nw + idx * E + i) : 1.0f;
-        return __fmul_rn(__fmul_rn(__fsub_rn(unit_elem(un, i), mu32), r32), wk);
+    // the norm weights of unit idx
+    auto w_unit = [&](int idx, float (&wv)[E]) {
+        if (stage_w) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const float4 t = norm_w_sm[norm_w_chunk<C>(idx, c)];
+                wv[4 * c] = t.x; wv[4 * c + 1] = t.y; wv[4 * c + 2] = t.z; wv[4 * c + 3] = t.w;
+            }
+        } else if (nw != nullptr) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) wv[i] = __ldg(nw + idx * E + i);
+        } else {
+#pragma unroll
+            for (int i = 0; i < E; ++i) wv[i] = 1.0f;
+        }
+    };
+    auto xn_of = [&](const Unit<U>& un, int i, const float (&wv)[E]) {
+        return __fmul_rn(__fmul_rn(__fsub_rn(unit_elem(un, i), mu32), r32), wv[i]);
     };
     float am = 0.0f;
     for_units([&](int idx, const Unit<U>& un) {
+        float wv[E];
+        w_unit(idx, wv);
 #pragma unroll
-        for (int i = 0; i < E; ++i) am = fmaxf(am, fabsf(xn_of(idx, un, i)));
+        for (int i = 0; i < E; ++i) am = fmaxf(am, fabsf(xn_of(un, i, wv)));
     });
     const float s = __fdiv_rn(127.0f, fmaxf(group_max(am), eps));
     if (!active) return;
     if (j == 0) s_out[row] = s;
     uint8_t* qrow = xq + row * K;
     for_units([&](int idx, const Unit<U>& un) {
+        float wv[E];
+        w_unit(idx, wv);
         uint32_t q[E];
 #pragma unroll
-        for (int i = 0; i < E; ++i) q[i] = q8_bits(xn_of(idx, un, i), s);
+        for (int i = 0; i < E; ++i) q[i] = q8_bits(xn_of(un, i, wv), s);
         store_q<L>(qrow, idx, q);
     });
 }
@@ -571,11 +613,13 @@ static cudaError_t launch_norm_g(const uint4* X4, const float* nw, int64_t M, in
                                  float eps, uint8_t* xq, float* s, cudaStream_t stream) {
     constexpr int CTA = G > 256 ? G : 256;
     const dim3 grid(grid_for(M, CTA / G, 1 << 30)), block(CTA);
+    const int stage_w = nw != nullptr && K <= kNormStageMaxK ? 1 : 0;
+    const size_t smem = stage_w ? static_cast<size_t>(K) * sizeof(float) : 0;
     if (kind == 1)
-        return launch_pdl(norm_act_quant_kernel<G, L, 1>, grid, block, 0, stream, dim3(kNoCluster), X4, nw, M, K,
-                          norm_eps, eps, xq, s);
-    return launch_pdl(norm_act_quant_kernel<G, L, 0>, grid, block, 0, stream, dim3(kNoCluster), X4, nw, M, K,
-                      norm_eps, eps, xq, s);
+        return launch_pdl(norm_act_quant_kernel<G, L, 1>, grid, block, smem, stream, dim3(kNoCluster), X4, nw, M,
+                          K, norm_eps, eps, xq, s, stage_w);
+    return launch_pdl(norm_act_quant_kernel<G, L, 0>, grid, block, smem, stream, dim3(kNoCluster), X4, nw, M, K,
+                      norm_eps, eps, xq, s, stage_w);
 }
 
 template <int L>

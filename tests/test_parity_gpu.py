@@ -518,7 +518,8 @@ def test_forward_stride4_wide_layer_repeated(M):
 
 # ------------------------------------- normalisation fused into the quantiser --
 
-NORM_SHAPES = [(1, 16), (3, 40), (5, 1536), (33, 4096), (4096, 1536), (7, 8192), (3, 28672), (2, 36000)]
+NORM_SHAPES = [(1, 16), (3, 40), (5, 1536), (33, 4096), (4096, 1536), (7, 8192), (2, 8208), (2, 12288), (3, 28672),
+               (2, 36000)]
 
 
 @pytest.mark.parametrize("M,K", NORM_SHAPES)
