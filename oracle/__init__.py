@@ -55,6 +55,14 @@ class Oracle:
         L.oracle_f32_to_bf16.restype = None
         L.oracle_forward.argtypes = [P, P, P, F, I, I, I, ctypes.c_int, P, P, P, P]
         L.oracle_forward.restype = I
+        L.oracle_tl5_row_bytes.argtypes = [I]
+        L.oracle_tl5_row_bytes.restype = I
+        L.oracle_pack_tl5.argtypes = [P, I, I, P]
+        L.oracle_pack_tl5.restype = I
+        L.oracle_unpack_tl5.argtypes = [P, I, I, P]
+        L.oracle_unpack_tl5.restype = None
+        L.oracle_forward_tl5.argtypes = [P, P, P, F, I, I, I, ctypes.c_int, P, P, P, P]
+        L.oracle_forward_tl5.restype = I
         self.L = L
         self.path = path
 
@@ -179,6 +187,45 @@ class Oracle:
         return out
 
 
+    def tl5_row_bytes(self, K):
+        """Bytes per row of the 1.6-bit format (oracle_tl5_row_bytes)."""
+        return int(self.L.oracle_tl5_row_bytes(int(K)))
+
+    def pack_tl5(self, codes):
+        """Five codes per byte (oracle_pack_tl5): (packed uint8 [N, row_bytes], bad count)."""
+        codes, pc = _c(codes, np.int8)
+        N, K = codes.shape
+        packed = np.empty((N, self.tl5_row_bytes(K)), dtype=np.uint8)
+        bad = self.L.oracle_pack_tl5(pc, N, K, _vp(packed))
+        return packed, int(bad)
+
+    def unpack_tl5(self, packed, K):
+        """Codes from the 1.6-bit format (oracle_unpack_tl5)."""
+        packed, pp = _c(packed, np.uint8)
+        N = packed.shape[0]
+        assert packed.shape[1] == self.tl5_row_bytes(K)
+        codes = np.empty((N, K), dtype=np.int8)
+        self.L.oracle_unpack_tl5(pp, N, K, _vp(codes))
+        return codes
+
+    def forward_tl5(self, xq, s, packed, gamma, K, out_kind=OUT_F32):
+        """Whole forward from 1.6-bit weights (oracle_forward_tl5)."""
+        xq, px = _c(xq, np.int8)
+        s, ps = _c(s, np.float32)
+        packed, pp = _c(packed, np.uint8)
+        M = xq.shape[0]
+        N = packed.shape[0]
+        assert xq.shape[1] == K and packed.shape[1] == self.tl5_row_bytes(K)
+        dt = {OUT_F32: np.float32, OUT_BF16: np.uint16, OUT_I32: np.int32}[out_kind]
+        out = np.empty((M, N), dtype=dt)
+        codes_tmp = np.empty((N, K), dtype=np.int8)
+        acc_tmp = np.empty((M, N), dtype=np.int32)
+        y_tmp = np.empty((M, N), dtype=np.float32)
+        over = self.L.oracle_forward_tl5(px, ps, pp, float(gamma), M, N, K, out_kind, _vp(out),
+                                         _vp(codes_tmp), _vp(acc_tmp), _vp(y_tmp))
+        assert over == 0, "int32 overflow in the oracle accumulator"
+        return out
+
 _default = None
 
 
@@ -202,3 +249,8 @@ def dequant_rows(acc, s, gamma_rows): return default().dequant_rows(acc, s, gamm
 def f32_to_bf16(y): return default().f32_to_bf16(y)
 def forward(xq, s, packed, gamma, K, out_kind=OUT_F32):
     return default().forward(xq, s, packed, gamma, K, out_kind)
+def pack_tl5(codes): return default().pack_tl5(codes)
+def unpack_tl5(packed, K): return default().unpack_tl5(packed, K)
+def tl5_row_bytes(K): return default().tl5_row_bytes(K)
+def forward_tl5(xq, s, packed, gamma, K, out_kind=OUT_F32):
+    return default().forward_tl5(xq, s, packed, gamma, K, out_kind)

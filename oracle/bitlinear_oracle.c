@@ -119,6 +119,73 @@ void oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *codes)
     }
 }
 
+/* ------------------------------------------------ 1.6-bit packing (TL5) -- */
+
+/* [B158] "What it is (the intuition)": a ternary weight carries log2(3) ~ 1.58 bits
+ * and packs to about 1.6 bits in practice; [CH2]: several ternary values share a
+ * storage unit and are unpacked where they are used.  Reading: five values per byte,
+ * since 3^5 = 243 <= 256, which is 1.6 bits per value exactly.  The layout (reading;
+ * the pages fix none):
+ *   - digit t = c + 1 in {0, 1, 2} for code c in {-1, 0, +1};
+ *   - a row is cut into blocks of 80 values along K, block b taking 16 bytes; byte j
+ *     (0..15) of block b holds the values k = 80 b + 16 p + j for p = 0..4 as the
+ *     base-3 number v = sum_p t_p 3^(4-p) (p = 0 the most significant digit);
+ *   - the byte holds v in 8-bit fixed point, B = ceil(v * 256 / 243), and is read
+ *     back as v = floor(B * 243 / 256), which is defined for every byte value;
+ *   - positions k >= K of the last block are written as code 0 and never read.
+ * A row takes 16 * ceil(K / 80) bytes; K is a multiple of 16. */
+int64_t oracle_tl5_row_bytes(int64_t K)
+{
+    return 16 * ((K + 79) / 80);
+}
+
+/* Codes outside {-1, 0, +1} are written as 0 and counted; the count is returned. */
+int64_t oracle_pack_tl5(const int8_t *codes, int64_t N, int64_t K, uint8_t *packed)
+{
+    int64_t bad = 0, n, b, j;
+    int p;
+    int64_t RB = oracle_tl5_row_bytes(K);
+    for (n = 0; n < N; ++n) {
+        for (b = 0; b < RB / 16; ++b) {
+            for (j = 0; j < 16; ++j) {
+                unsigned v = 0;
+                for (p = 0; p < 5; ++p) {
+                    int64_t k = 80 * b + 16 * p + j;
+                    int t = 1;
+                    if (k < K) {
+                        int8_t code = codes[n * K + k];
+                        if (code == -1 || code == 0 || code == 1)
+                            t = code + 1;
+                        else
+                            ++bad;
+                    }
+                    v = 3 * v + (unsigned)t;
+                }
+                packed[n * RB + 16 * b + j] = (uint8_t)((v * 256u + 242u) / 243u);
+            }
+        }
+    }
+    return bad;
+}
+
+/* Inverse of oracle_pack_tl5 for every byte value. */
+void oracle_unpack_tl5(const uint8_t *packed, int64_t N, int64_t K, int8_t *codes)
+{
+    int64_t n, k;
+    int64_t RB = oracle_tl5_row_bytes(K);
+    for (n = 0; n < N; ++n) {
+        for (k = 0; k < K; ++k) {
+            int64_t b = k / 80, r = k % 80;
+            int p = (int)(r / 16), i;
+            unsigned byte = packed[n * RB + 16 * b + r % 16];
+            unsigned v = byte * 243u / 256u;
+            unsigned w = 1;
+            for (i = 0; i < 4 - p; ++i) w *= 3u;
+            codes[n * K + k] = (int8_t)((int)(v / w % 3u) - 1);
+        }
+    }
+}
+
 /* ------------------------------------------------------------ activations -- */
 
 /* bf16 -> fp32 is exact: the bf16 bit pattern is the top half of the fp32 one. */
@@ -277,6 +344,27 @@ int64_t oracle_forward(const int8_t *xq, const float *s, const uint8_t *packed, 
                        int8_t *codes_tmp, int32_t *acc_tmp, float *y_tmp)
 {
     oracle_unpack(packed, N, K, codes_tmp);
+    int64_t over = oracle_int_matmul(xq, codes_tmp, M, N, K, acc_tmp);
+    if (out_kind == 2) {
+        memcpy(out, acc_tmp, (size_t)(M * N) * sizeof(int32_t));
+        return over;
+    }
+    if (out_kind == 0) {
+        oracle_dequant(acc_tmp, s, gamma, M, N, (float *)out);
+        return over;
+    }
+    oracle_dequant(acc_tmp, s, gamma, M, N, y_tmp);
+    oracle_f32_to_bf16(y_tmp, M * N, (uint16_t *)out);
+    return over;
+}
+
+/* The forward from the 1.6-bit format: decode it, then the same integer products and
+ * rescale as oracle_forward. */
+int64_t oracle_forward_tl5(const int8_t *xq, const float *s, const uint8_t *packed, float gamma,
+                           int64_t M, int64_t N, int64_t K, int out_kind, void *out,
+                           int8_t *codes_tmp, int32_t *acc_tmp, float *y_tmp)
+{
+    oracle_unpack_tl5(packed, N, K, codes_tmp);
     int64_t over = oracle_int_matmul(xq, codes_tmp, M, N, K, acc_tmp);
     if (out_kind == 2) {
         memcpy(out, acc_tmp, (size_t)(M * N) * sizeof(int32_t));

@@ -18,6 +18,7 @@ import numpy as np
 import torch
 
 from conftest import parse_golden
+from oracle import OUT_BF16, OUT_F32, OUT_I32
 
 EPS = 1e-5
 
@@ -387,11 +388,114 @@ def pin_dequant_rows(O):
     assert np.array_equal(O.dequant_rows(acc, s, np.full(33, g, dtype=np.float32)), O.dequant(acc, s, g))
 
 
+# ------------------------------------------------------- 1.6-bit packing (TL5) --
+
+def _row_from_nonzero(K, spec):
+    row = np.zeros(K, dtype=np.int8)
+    for item in spec.split(","):
+        k, c = item.split(":")
+        row[int(k)] = int(c)
+    return row
+
+
+def pin_hand_tl5(O):
+    """Hand-worked bytes of the five-per-byte format (golden file), both directions, and
+    hand-decoded bytes that packing never writes."""
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind == "tl5":
+            K = int(r["K"])
+            row = _row_from_nonzero(K, r["nonzero"])[None, :]
+            want = _ints(r["bytes"], np.uint8)[None, :]
+            packed, bad = O.pack_tl5(row)
+            assert bad == 0
+            assert np.array_equal(packed, want), (K, packed, want)
+            assert np.array_equal(O.unpack_tl5(want, K), row)
+            n += 1
+        elif kind == "tl5dec":
+            blk = np.full((1, 16), 128, dtype=np.uint8)  # 128 = five zero codes
+            blk[0, 0] = int(r["byte"])
+            codes = O.unpack_tl5(blk, 80)
+            assert np.array_equal(codes[0, 0::16], _ints(r["codes"], np.int8)), (r, codes[0, 0::16])
+            assert not codes[0].reshape(5, 16)[:, 1:].any()
+            n += 1
+    assert n >= 7
+
+
+def pin_tl5_every_value(O):
+    """All 3^5 digit patterns of one byte: packing is one to one and order preserving
+    (the stored byte grows with v = sum t_p 3^(4-p), p = 0 most significant), and
+    reading gives each pattern back.  Every byte value 0..255 reads as codes in
+    {-1, 0, +1}, and the value it encodes never decreases with the byte."""
+    import itertools
+    pats = np.array(list(itertools.product((-1, 0, 1), repeat=5)), dtype=np.int8)  # lexicographic = v order
+    rows = np.zeros((pats.shape[0], 80), dtype=np.int8)
+    for p in range(5):
+        rows[:, 16 * p] = pats[:, p]
+    packed, bad = O.pack_tl5(rows)
+    assert bad == 0
+    b0 = packed[:, 0].astype(np.int64)
+    assert np.all(np.diff(b0) > 0) and b0[0] == 0 and b0[-1] == 255
+    assert np.array_equal(O.unpack_tl5(packed, 80), rows)
+    allb = np.full((256, 16), 128, dtype=np.uint8)
+    allb[:, 0] = np.arange(256)
+    dec = O.unpack_tl5(allb, 80)[:, 0::16].astype(np.int64) + 1
+    assert dec.min() >= 0 and dec.max() <= 2
+    v = dec @ np.array([81, 27, 9, 3, 1])
+    assert np.all(np.diff(v) >= 0) and v[0] == 0 and v[-1] == 242
+    # 256 byte values for 243 patterns: each pattern is read from one or two bytes
+    assert len(np.unique(v)) == 243
+
+
+def pin_tl5_size_and_equivalence(O):
+    """Rows take 16 * ceil(K / 80) bytes, 1.6 bits per code when 80 divides K (the
+    pages' ~1.6 bits per weight).  For ragged K and several rows, the codes read back
+    from the five-per-byte format equal the codes read back from the 2-bit format, and
+    the forward from either format is the same, for every output kind."""
+    for K, want in ((16, 16), (80, 16), (96, 32), (160, 32), (8192, 1648), (28672, 5744)):
+        assert O.tl5_row_bytes(K) == want, (K, O.tl5_row_bytes(K))
+    assert O.tl5_row_bytes(8000) * 8 / 8000 == 1.6
+    rng = np.random.default_rng(23)
+    for N, K in ((7, 16), (5, 96), (3, 400), (9, 1040)):
+        c = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        p5, bad = O.pack_tl5(c)
+        assert bad == 0 and p5.shape == (N, O.tl5_row_bytes(K))
+        p2, _ = O.pack(c)
+        assert np.array_equal(O.unpack_tl5(p5, K), O.unpack(p2, K))
+        M = 3
+        xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+        s = rng.uniform(0.5, 100.0, size=M).astype(np.float32)
+        for kind in (OUT_I32, OUT_F32, OUT_BF16):
+            assert np.array_equal(O.forward_tl5(xq, s, p5, 0.0271, K, kind), O.forward(xq, s, p2, 0.0271, K, kind))
+    # invalid codes are counted and written as 0
+    cb = rng.integers(-1, 2, size=(2, 32)).astype(np.int8)
+    cb[0, 3], cb[1, 30] = 2, -5
+    pb, badb = O.pack_tl5(cb)
+    assert badb == 2
+    ub = O.unpack_tl5(pb, 32)
+    assert ub[0, 3] == 0 and ub[1, 30] == 0
+
+
+def pin_tl5_padding_not_read(O):
+    """Positions past K in the last block carry no code: whatever digits a byte holds
+    there, reading gives the same codes for k < K."""
+    rng = np.random.default_rng(29)
+    c = rng.integers(-1, 2, size=(4, 48)).astype(np.int8)  # block of 80, planes 3 and 4 are padding
+    p5, _ = O.pack_tl5(c)
+    t = (c.astype(np.int64) + 1).reshape(4, 3, 16)
+    for pad3, pad4 in ((0, 0), (2, 2), (0, 2), (1, 0)):
+        v = t[:, 0] * 81 + t[:, 1] * 27 + t[:, 2] * 9 + pad3 * 3 + pad4
+        other = ((v * 256 + 242) // 243).astype(np.uint8)
+        assert np.array_equal(O.unpack_tl5(other, 48), c)
+    assert np.array_equal(p5, (((t[:, 0] * 81 + t[:, 1] * 27 + t[:, 2] * 9 + 4) * 256 + 242) // 243).astype(np.uint8))
+
+
 def _bf16_to_f32(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
 ALL_PINS = [
+    pin_hand_tl5, pin_tl5_every_value, pin_tl5_size_and_equivalence, pin_tl5_padding_not_read,
     pin_hand_norm, pin_norm_vs_torch, pin_norm_invariants, pin_dequant_rows,
     pin_hand_ternarise, pin_hand_absmean, pin_hand_act, pin_hand_pack, pin_hand_matmul,
     pin_gaussian_statistics, pin_constant_magnitude, pin_zero_weights, pin_zero_token,

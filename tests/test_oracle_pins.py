@@ -55,6 +55,12 @@ MUTANTS = [
     ("row_gamma_by_token", "(double)gamma_rows[n] / (double)s[m]", "(double)gamma_rows[m] / (double)s[m]"),
     ("row_gamma_dropped", "(double)acc[m * N + n] * (double)gamma_rows[n] / (double)s[m]",
      "(double)acc[m * N + n] / (double)s[m]"),
+    ("tl5_floor_encode", "(uint8_t)((v * 256u + 242u) / 243u)", "(uint8_t)((v * 256u) / 243u)"),
+    ("tl5_digit_order", "for (i = 0; i < 4 - p; ++i) w *= 3u;", "for (i = 0; i < p; ++i) w *= 3u;"),
+    ("tl5_no_offset", "t = code + 1;", "t = code < 0 ? 2 : code;"),
+    ("tl5_interleaved", "int64_t k = 80 * b + 16 * p + j;", "int64_t k = 80 * b + 5 * j + p;"),
+    ("tl5_pad_minus_one", "int t = 1;\n", "int t = 0;\n"),
+    ("tl5_decode_255", "unsigned v = byte * 243u / 256u;", "unsigned v = byte * 243u / 255u;"),
 ]
 
 
