@@ -51,7 +51,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--ref-tokens", type=int, default=4,
                    help="token rows per M in one reference-arm (oracle) step")
-    p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack"],
+    p.add_argument("--weight-format", choices=["2bit", "tl5"], default="2bit",
+                   help="--sweep: the 2-bit forward, or the five-codes-per-byte decode forward (M <= 16 shapes)")
+    p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack",
+                                        "forward_tl5", "repack_tl5"],
                    help="time one entry point on one shape instead of the step (kernel study, ncu)")
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
@@ -376,7 +379,8 @@ def run_ours(args):
         try:
             tj = json.load(open(tpath))
             from ternary_weight_bit_absmean_b200 import build_lib as _bl
-            if tj.get("source_digest") == _bl.source_digest():
+            files = tj.get("digest_files")
+            if files and tj.get("source_digest") == _bl.source_digest(files):
                 traffic = tj.get("gemm_tc_M%d_bytes_per_launch" % Mbig)
         except (ValueError, KeyError, AttributeError):
             traffic = None
@@ -513,6 +517,24 @@ def run_single(args):
         fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=lay)
         ops = 2 * M * N * K
         nbytes = N * K // 4 + M * K + 4 * M + M * N * out.element_size()
+    elif args.single == "forward_tl5":
+        # the 1.6-bit decode forward; x_q row-major
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+        s = torch.rand(M, device=dev) + 1.0
+        tl5 = B.pack_tl5(synth.codes(N, K, seed=1).to(dev))
+        gamma = torch.tensor([0.02], device=dev)
+        odt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[args.out_dtype]
+        out = torch.empty(M, N, dtype=odt, device=dev)
+        fn = lambda: B.bitlinear_forward_tl5(xq, s, tl5, gamma, out)
+        ops = 2 * M * N * K
+        wbytes = N * B.bitlinear_tl5_row_bytes(K)
+        nbytes = wbytes + M * K + 4 * M + M * N * out.element_size()
+    elif args.single == "repack_tl5":
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+        B.bitlinear_pack(synth.codes(N, K, seed=1).to(dev), packed)
+        tl5 = torch.empty(N, B.bitlinear_tl5_row_bytes(K), dtype=torch.uint8, device=dev)
+        fn = lambda: B.bitlinear_repack_tl5(packed, tl5)
+        ops, nbytes = 0, N * K // 4 + tl5.numel()
     elif args.single == "quantize_act":
         X = torch.randn(M, K, device=dev).to(torch.bfloat16)
         xq = torch.empty(M, K, dtype=torch.int8, device=dev)
@@ -546,7 +568,8 @@ def run_single(args):
            "xq_layout": args.xq_layout,
            "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
            "gbs": round(nbytes / t / 1e9, 1), "hbm_frac": round(nbytes / t / 1e9 / P["hbm_gbs"], 4),
-           "weight_gbs": round((N * K // 4) / t / 1e9, 1) if args.single == "forward" else None}
+           "weight_gbs": (round((N * K // 4) / t / 1e9, 1) if args.single == "forward" else
+                          round(wbytes / t / 1e9, 1) if args.single == "forward_tl5" else None)}
     if ops:
         rec["tops"] = round(ops / t / 1e12, 2)
         rec["int8_frac"] = round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4)
@@ -602,9 +625,12 @@ def run_sweep(args):
     torch.cuda.set_device(dev)
     flusher = L2Flusher(dev)
     P = peaks()
-    lay = xq_layout_of(B, args.xq_layout)
+    tl5 = args.weight_format == "tl5"
+    lay = B.BL_XQ_ROWMAJOR if tl5 else xq_layout_of(B, args.xq_layout)
     packed_of = {}
     for M, N, K, tag in sweep_shapes(args.sweep):
+        if tl5 and M > 16:
+            continue
         X = synth.activations(M, K, seed=M + K, outlier_frac=0.01).to(dev)
         xq = torch.empty(M, K, dtype=torch.int8, device=dev)
         s = torch.empty(M, device=dev)
@@ -612,19 +638,28 @@ def run_sweep(args):
         if (N, K) not in packed_of:
             packed_of.clear()
             c = synth.codes(N, K, seed=N + K).to(dev)
-            packed_of[N, K] = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
-            B.bitlinear_pack(c, packed_of[N, K])
+            if tl5:
+                packed_of[N, K] = B.pack_tl5(c)
+            else:
+                packed_of[N, K] = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+                B.bitlinear_pack(c, packed_of[N, K])
             del c
         packed = packed_of[N, K]
         gamma = torch.tensor([0.02], device=dev)
         out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ts = time_calls(lambda: B.bitlinear_forward(xq, s, packed, gamma, out, layout=lay), flusher, args.iters)
+        if tl5:
+            fn = lambda: B.bitlinear_forward_tl5(xq, s, packed, gamma, out)
+        else:
+            fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, layout=lay)
+        ts = time_calls(fn, flusher, args.iters)
         t = statistics.median(ts) * 1e-3
         ops = 2 * M * N * K
-        nbytes = N * K // 4 + M * K + 4 * M + 2 * M * N
-        rec = {"sweep": args.sweep, "tag": tag, "M": M, "N": N, "K": K, "xq_layout": args.xq_layout,
+        wbytes = packed.numel()
+        nbytes = wbytes + M * K + 4 * M + 2 * M * N
+        rec = {"sweep": args.sweep, "tag": tag, "M": M, "N": N, "K": K,
+               "xq_layout": "rowmajor" if tl5 else args.xq_layout, "weight_format": args.weight_format,
                "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
-               "tops": round(ops / t / 1e12, 2), "weight_gbs": round((N * K // 4) / t / 1e9, 1),
+               "tops": round(ops / t / 1e12, 2), "weight_gbs": round(wbytes / t / 1e9, 1),
                "hbm_frac": round(nbytes / t / 1e9 / P["hbm_gbs"], 4),
                "int8_frac": round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4),
                "regime": "hbm" if M <= 16 else "tensor"}

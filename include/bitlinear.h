@@ -257,6 +257,52 @@ BL_API bl_status bitlinear_forward_rowscale(const int8_t *xq, const float *s, co
                                             bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,
                                             bl_path path, void *stream);
 
+/* ----------------------------------------------------------------------------------
+ * 1.6-bit weight format (TL5): five codes per byte.
+ * [B158] "What it is (the intuition)": ternary weights pack to about 1.6 bits each in
+ * practice; [CH2]: several values per storage unit, unpacked where they are used.
+ * 3^5 = 243 <= 256, so a byte holds five codes (1.6 bits each, 20% fewer weight bytes
+ * than the 2-bit format).
+ *   uint8 [N, bitlinear_tl5_row_bytes(K)], row-major, K % 16 == 0.  A row is cut into
+ *   blocks of 80 codes along K, 16 bytes per block; byte j (0..15) of block b holds the
+ *   codes of k = 80 b + 16 p + j for p = 0..4 as the base-3 number
+ *   v = sum_p (c_p + 1) 3^(4-p) (p = 0 most significant), stored in 8-bit fixed point
+ *   B = ceil(256 v / 243) and read back as v = floor(243 B / 256).  Every byte value
+ *   reads as five valid codes.  Codes past K (the missing planes of a last, partial
+ *   block) are written as 0 and ignored by the forward.
+ * ---------------------------------------------------------------------------------- */
+
+/* Bytes per row of the TL5 format: 16 * ceil(K / 80); 0 if K <= 0 or K % 16 != 0. */
+BL_API int64_t bitlinear_tl5_row_bytes(int64_t K);
+
+/* Pack int8 codes into the TL5 format.
+ *   codes   in  : int8 [N, K] in {-1, 0, +1}, device.
+ *   tl5_out out : uint8 [N, bitlinear_tl5_row_bytes(K)], device.
+ *   err_word out: optional; BL_ERRBIT_BAD_CODE is OR-ed in if a code is outside
+ *                 {-1, 0, +1}; such a code is written as 0.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 16), BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_pack_tl5(const int8_t *codes, int64_t N, int64_t K, uint8_t *tl5_out,
+                                    int32_t *err_word, void *stream);
+
+/* Convert the 2-bit packed format (uint8 [N, K/4], as written by
+ * bitlinear_quantize_weights) into the TL5 format; a 2-bit code 11 becomes 0.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE (K % 16), BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_repack_tl5(const uint8_t *packed, int64_t N, int64_t K, uint8_t *tl5_out,
+                                      void *stream);
+
+/* The BitLinear forward of bitlinear_forward with the weights in the TL5 format:
+ *   acc[m, n] = sum_k x_q[m, k] c[n, k] (exact int32), y = float(acc) * (gamma / s[m]).
+ *   xq  in : int8 [M, K] row-major (BL_XQ_ROWMAJOR), device.
+ *   tl5 in : uint8 [N, bitlinear_tl5_row_bytes(K)], device.
+ *   s, gamma, out, out_dtype: as for bitlinear_forward.
+ * A decode kernel (one warp per output row, tokens in groups of up to 16): meant for
+ * small M; larger M re-reads the weights once per 16 tokens.  K % 16 == 0,
+ * K * 128 < 2^31, M <= 65535 * 16.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_forward_tl5(const int8_t *xq, const float *s, const uint8_t *tl5,
+                                       const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
+                                       bl_dtype out_dtype, void *stream);
+
 /* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
 BL_API int bitlinear_last_cuda_error(void);
 

@@ -32,6 +32,7 @@ EXPORTED = [
     "bitlinear_quantize_weights_with_scale", "bitlinear_pack", "bitlinear_quantize_act",
     "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
     "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_forward_rowscale",
+    "bitlinear_tl5_row_bytes", "bitlinear_pack_tl5", "bitlinear_repack_tl5", "bitlinear_forward_tl5",
     "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
@@ -82,6 +83,14 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_forward_rowscale.restype = S
         L.bitlinear_norm_quantize_act.argtypes = [P, P, I64, I64, S, F, F, P, P, S, P]
         L.bitlinear_norm_quantize_act.restype = S
+        L.bitlinear_tl5_row_bytes.argtypes = [I64]
+        L.bitlinear_tl5_row_bytes.restype = I64
+        L.bitlinear_pack_tl5.argtypes = [P, I64, I64, P, P, P]
+        L.bitlinear_pack_tl5.restype = S
+        L.bitlinear_repack_tl5.argtypes = [P, I64, I64, P, P]
+        L.bitlinear_repack_tl5.restype = S
+        L.bitlinear_forward_tl5.argtypes = [P, P, P, P, I64, I64, I64, P, S, P]
+        L.bitlinear_forward_tl5.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
         L.bitlinear_last_cuda_error.restype = ctypes.c_int
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
@@ -201,6 +210,38 @@ def bitlinear_forward_rowscale(xq, s, packed, gamma_rows, out, err_word=None, st
         _stream(stream)), "bitlinear_forward_rowscale")
 
 
+def bitlinear_tl5_row_bytes(K):
+    return int(lib().bitlinear_tl5_row_bytes(int(K)))
+
+
+def bitlinear_pack_tl5(codes, tl5_out, err_word=None, stream=None):
+    N, K = codes.shape
+    _check(lib().bitlinear_pack_tl5(
+        _dev(codes, torch.int8, "codes"), N, K, _dev(tl5_out, torch.uint8, "tl5_out", (N, bitlinear_tl5_row_bytes(K))),
+        _opt(err_word, "err_word"), _stream(stream)), "bitlinear_pack_tl5")
+
+
+def bitlinear_repack_tl5(packed, tl5_out, stream=None):
+    N, KB = packed.shape
+    K = 4 * KB
+    _check(lib().bitlinear_repack_tl5(
+        _dev(packed, torch.uint8, "packed"), N, K,
+        _dev(tl5_out, torch.uint8, "tl5_out", (N, bitlinear_tl5_row_bytes(K))), _stream(stream)),
+        "bitlinear_repack_tl5")
+
+
+def bitlinear_forward_tl5(xq, s, tl5, gamma, out, stream=None):
+    M, K = xq.shape
+    N = tl5.shape[0]
+    kind = {v: k for k, v in _OUT_DT.items()}.get(out.dtype)
+    if kind is None:
+        raise TypeError("out must be float32, bfloat16 or int32")
+    _check(lib().bitlinear_forward_tl5(
+        _dev(xq, torch.int8, "xq"), _dev(s, torch.float32, "s", (M,)),
+        _dev(tl5, torch.uint8, "tl5", (N, bitlinear_tl5_row_bytes(K))), _dev(gamma, torch.float32, "gamma"),
+        M, N, K, _dev(out, out.dtype, "out", (M, N)), kind, _stream(stream)), "bitlinear_forward_tl5")
+
+
 # ----------------------------------------------------------- allocating helpers --
 
 def quantize_weights(W: torch.Tensor, eps: float = 1e-5, stream=None):
@@ -237,4 +278,27 @@ def forward(xq, s, packed, gamma, out_dtype=torch.float32, stream=None, path=BL_
     """y [M, N] of the BitLinear forward from quantised operands."""
     out = torch.empty(xq.shape[0], packed.shape[0], dtype=out_dtype, device=xq.device)
     bitlinear_forward(xq, s, packed, gamma, out, err_word, stream, path, layout)
+    return out
+
+
+def pack_tl5(codes: torch.Tensor, stream=None):
+    """[N, tl5_row_bytes(K)] uint8: int8 codes in the five-per-byte format."""
+    N, K = codes.shape
+    out = torch.empty(N, bitlinear_tl5_row_bytes(K), dtype=torch.uint8, device=codes.device)
+    bitlinear_pack_tl5(codes, out, None, stream)
+    return out
+
+
+def repack_tl5(packed: torch.Tensor, stream=None):
+    """[N, tl5_row_bytes(K)] uint8 from the 2-bit format [N, K/4]."""
+    N, KB = packed.shape
+    out = torch.empty(N, bitlinear_tl5_row_bytes(4 * KB), dtype=torch.uint8, device=packed.device)
+    bitlinear_repack_tl5(packed, out, stream)
+    return out
+
+
+def forward_tl5(xq, s, tl5, gamma, out_dtype=torch.float32, stream=None):
+    """y [M, N] from row-major x_q and weights in the five-per-byte format."""
+    out = torch.empty(xq.shape[0], tl5.shape[0], dtype=out_dtype, device=xq.device)
+    bitlinear_forward_tl5(xq, s, tl5, gamma, out, stream)
     return out

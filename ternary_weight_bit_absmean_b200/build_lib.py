@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbitlinear.so")
-SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_noalloc.cu"]
+SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_noalloc.cu", "k_tl5.cu"]
 HEADERS = ["bl_device.cuh", "bl_internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -29,14 +29,22 @@ def _inputs():
             + [os.path.join(INCLUDE, "bitlinear.h"), os.path.abspath(__file__)])
 
 
-def source_digest() -> str:
-    """SHA-256 over the library's sources and header (identifies a kernel build)."""
+def source_digest(files=None) -> str:
+    """SHA-256 over the library's sources and header (identifies a kernel build), or
+    over the given source files only (identifies the kernels they define)."""
     import hashlib
     h = hashlib.sha256()
-    for p in [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "bitlinear.h")]:
+    paths = ([os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "bitlinear.h")]
+             if files is None else [os.path.join(CSRC, f) for f in files])
+    for p in paths:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+# The files that define the prefill kernels (their device code and the helpers it
+# inlines): DRAM counters taken on these kernels stay valid while these are unchanged.
+PREFILL_KERNEL_FILES = ["k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_device.cuh"]
 
 
 def up_to_date() -> bool:

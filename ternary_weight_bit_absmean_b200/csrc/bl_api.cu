@@ -168,6 +168,51 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     return cuda_status(e);
 }
 
+int64_t bitlinear_tl5_row_bytes(int64_t K) {
+    if (K <= 0 || K % 16 != 0) return 0;
+    return bl::tl5_row_bytes(K);
+}
+
+// Shapes of the TL5 weight entry points: the 2-bit rules plus K % 16 == 0, K < 2^31.
+static bl_status check_tl5_shape(int64_t N, int64_t K) {
+    bl_status st = check_weight_shape(N, K);
+    if (st != BL_OK) return st;
+    if (K % 16 != 0 || K >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
+    return BL_OK;
+}
+
+bl_status bitlinear_pack_tl5(const int8_t* codes, int64_t N, int64_t K, uint8_t* tl5_out, int32_t* err_word,
+                             void* stream) {
+    if (codes == nullptr || tl5_out == nullptr) return BL_ERR_INVALID_ARG;
+    bl_status st = check_tl5_shape(N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(codes) || !aligned16(tl5_out)) return BL_ERR_MISALIGNED;
+    return cuda_status(bl::launch_tl5_pack(codes, N, K, tl5_out, err_word, as_stream(stream)));
+}
+
+bl_status bitlinear_repack_tl5(const uint8_t* packed, int64_t N, int64_t K, uint8_t* tl5_out, void* stream) {
+    if (packed == nullptr || tl5_out == nullptr) return BL_ERR_INVALID_ARG;
+    bl_status st = check_tl5_shape(N, K);
+    if (st != BL_OK) return st;
+    if (!aligned16(packed) || !aligned16(tl5_out)) return BL_ERR_MISALIGNED;
+    return cuda_status(bl::launch_tl5_repack(packed, N, K, tl5_out, as_stream(stream)));
+}
+
+bl_status bitlinear_forward_tl5(const int8_t* xq, const float* s, const uint8_t* tl5, const float* gamma, int64_t M,
+                                int64_t N, int64_t K, void* out, bl_dtype out_dtype, void* stream) {
+    if (xq == nullptr || s == nullptr || tl5 == nullptr || gamma == nullptr || out == nullptr)
+        return BL_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32) return BL_ERR_INVALID_ARG;
+    if (K % 16 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    // |acc| <= 128 K must fit in int32; token groups of 16 go to grid.y (at most 65535)
+    if (K > (int64_t(1) << 31) / 128 - 1) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (M > int64_t(65535) * 16 || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(xq) || !aligned16(s) || !aligned16(tl5) || !aligned16(out)) return BL_ERR_MISALIGNED;
+    return cuda_status(bl::launch_gemv_tl5(xq, s, tl5, gamma, M, N, K, out, static_cast<int>(out_dtype),
+                                           as_stream(stream)));
+}
+
 bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                                    int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
                                    int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {

@@ -67,6 +67,14 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                             int kind, int32_t* err, int layout, cudaStream_t stream);
 
+// The 1.6-bit (five codes per byte) weight format, K % 16 == 0 (k_tl5.cu).
+int64_t tl5_row_bytes(int64_t K);
+cudaError_t launch_tl5_pack(const int8_t* codes, int64_t N, int64_t K, uint8_t* out, int32_t* err,
+                            cudaStream_t stream);
+cudaError_t launch_tl5_repack(const uint8_t* packed, int64_t N, int64_t K, uint8_t* out, cudaStream_t stream);
+cudaError_t launch_gemv_tl5(const int8_t* xq, const float* s, const uint8_t* w5, const float* gamma, int64_t M,
+                            int64_t N, int64_t K, void* out, int kind, cudaStream_t stream);
+
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);
 

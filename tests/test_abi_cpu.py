@@ -130,6 +130,32 @@ def test_other_entry_points_validation(L):
     assert qa(FAKE, 4, 32, 1e-5, FAKE, FAKE, 3, None) == INVALID
 
 
+def test_tl5_entry_points_validation(L):
+    """The five-codes-per-byte entry points reject bad arguments on the host."""
+    rb = L.bitlinear_tl5_row_bytes
+    assert [rb(k) for k in (16, 80, 96, 8192, 28672)] == [16, 16, 32, 1648, 5744]
+    assert rb(0) == 0 and rb(-16) == 0 and rb(24) == 0
+    pk = L.bitlinear_pack_tl5
+    assert pk(None, 8, 64, FAKE, None, None) == INVALID
+    assert pk(FAKE, 0, 64, FAKE, None, None) == INVALID
+    assert pk(FAKE, 8, 72, FAKE, None, None) == SHAPE          # K % 16
+    assert pk(ODD, 8, 64, FAKE, None, None) == MISALIGNED
+    assert pk(FAKE, 8, 64, ODD, None, None) == MISALIGNED
+    rp = L.bitlinear_repack_tl5
+    assert rp(FAKE, 8, 64, None, None) == INVALID
+    assert rp(FAKE, 8, 40, FAKE, None) == SHAPE
+    assert rp(ODD, 8, 64, FAKE, None) == MISALIGNED
+    f = L.bitlinear_forward_tl5
+    assert f(None, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 8, 64, FAKE, 0, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 7, None) == INVALID          # unknown dtype
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 8, 72, FAKE, 0, None) == SHAPE            # K % 16
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 8, 1 << 25, FAKE, 0, None) == SHAPE       # int32 accumulators
+    assert f(FAKE, FAKE, FAKE, FAKE, 65535 * 16 + 1, 8, 64, FAKE, 0, None) == SHAPE
+    assert f(FAKE, FAKE, ODD, FAKE, 4, 8, 64, FAKE, 0, None) == MISALIGNED
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, ODD, 0, None) == MISALIGNED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from ternary_weight_bit_absmean_b200 import binding
     monkeypatch.setattr(binding, "_lib", None)

@@ -651,3 +651,138 @@ def test_forward_rowscale_equal_scales_match_single_scale():
         B.bitlinear_forward_rowscale(xq, s, pk, gr, b, path=path)
         sync()
         assert torch.equal(a, b), path
+
+
+# ------------------------------------------ 1.6-bit weights, five codes per byte --
+
+TL5_PACK_SHAPES = [(1, 16), (3, 80), (5, 96), (7, 1040), (64, 4096), (33, 8192), (2, 28672), (300, 1536)]
+
+
+@pytest.mark.parametrize("N,K", TL5_PACK_SHAPES)
+def test_pack_tl5_and_repack(N, K):
+    """Packing int8 codes and converting the 2-bit format give the oracle's bytes."""
+    c = synth.codes(N, K, seed=N + K).numpy()
+    want, bad = oracle.pack_tl5(c)
+    assert bad == 0
+    out = guarded_empty(want.shape, torch.uint8)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.bitlinear_pack_tl5(torch.from_numpy(c).to(DEV), out, err)
+    sync()
+    check_guard(out)
+    assert err.item() == 0
+    assert np.array_equal(out.cpu().numpy(), want)
+    packed2, _ = oracle.pack(c)
+    out2 = guarded_empty(want.shape, torch.uint8)
+    B.bitlinear_repack_tl5(torch.from_numpy(packed2).to(DEV), out2)
+    sync()
+    check_guard(out2)
+    assert np.array_equal(out2.cpu().numpy(), want)
+
+
+def test_pack_tl5_flags_bad_codes_and_repack_reads_code_11_as_zero():
+    c = synth.codes(4, 160, seed=5).numpy().copy()
+    c[1, 17], c[3, 159] = 3, -2
+    want, bad = oracle.pack_tl5(c)
+    assert bad == 2
+    out = torch.empty(want.shape, dtype=torch.uint8, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.bitlinear_pack_tl5(torch.from_numpy(c).to(DEV), out, err)
+    sync()
+    assert err.item() & B.BL_ERRBIT_BAD_CODE
+    assert np.array_equal(out.cpu().numpy(), want)
+    # a 2-bit byte of 0xFF holds four codes 11, read as 0
+    packed2, _ = oracle.pack(np.zeros((2, 64), np.int8))
+    packed2[0, 3] = 0xFF
+    packed2[1, 15] = 0xBF  # 10 11 11 11: -1 then three codes 11
+    ref_codes = oracle.unpack(packed2, 64)
+    want2, _ = oracle.pack_tl5(ref_codes)
+    out2 = torch.empty(want2.shape, dtype=torch.uint8, device=DEV)
+    B.bitlinear_repack_tl5(torch.from_numpy(packed2).to(DEV), out2)
+    sync()
+    assert np.array_equal(out2.cpu().numpy(), want2)
+
+
+def _tl5_forward(xq_ref, s_ref, tl5_ref, g_ref, out_dtype):
+    M, K = xq_ref.shape
+    N = tl5_ref.shape[0]
+    out = guarded_empty((M, N), out_dtype)
+    B.bitlinear_forward_tl5(torch.from_numpy(xq_ref).to(DEV), torch.from_numpy(s_ref).to(DEV),
+                            torch.from_numpy(tl5_ref).to(DEV),
+                            torch.tensor([g_ref], dtype=torch.float32, device=DEV), out)
+    sync()
+    check_guard(out)
+    return out
+
+
+def check_forward_tl5(xq_ref, s_ref, tl5_ref, g_ref, rows=None):
+    K = xq_ref.shape[1]
+    sel = np.arange(xq_ref.shape[0]) if rows is None else np.asarray(rows)
+    acc_ref = oracle.forward_tl5(xq_ref[sel], s_ref[sel], tl5_ref, g_ref, K, oracle.OUT_I32)
+    y_ref = oracle.dequant(acc_ref, s_ref[sel], g_ref)
+    acc = _tl5_forward(xq_ref, s_ref, tl5_ref, g_ref, torch.int32).cpu().numpy()
+    assert np.array_equal(acc[sel], acc_ref), "int32 accumulators differ"
+    y = _tl5_forward(xq_ref, s_ref, tl5_ref, g_ref, torch.float32).cpu().numpy()
+    assert_float_close(y[sel], y_ref, "fp32 y")
+    yb = _tl5_forward(xq_ref, s_ref, tl5_ref, g_ref, torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert_bf16_match(yb[sel], y_ref, oracle.f32_to_bf16(y_ref), "bf16 y")
+    return acc
+
+
+TL5_FWD_CASES = [(1, 1, 16), (1, 37, 80), (2, 100, 96), (3, 300, 1040), (4, 1536, 1536), (5, 1000, 4096),
+                 (8, 4096, 1536), (13, 3200, 8640), (16, 8192, 512), (17, 200, 1536), (40, 64, 8192),
+                 (1, 3, 28672)]
+
+
+@pytest.mark.parametrize("M,N,K", TL5_FWD_CASES)
+def test_forward_tl5(M, N, K):
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=7 * M + N + K)
+    tl5_ref, _ = oracle.pack_tl5(oracle.unpack(packed_ref, K))
+    check_forward_tl5(xq_ref, s_ref, tl5_ref, g_ref)
+
+
+def test_forward_tl5_reads_every_byte_value():
+    """Arbitrary bytes, including the 13 values packing never writes: the forward reads
+    each as the oracle does (and ignores the missing planes of a partial last block)."""
+    rng = np.random.default_rng(31)
+    for M, N, K in ((1, 64, 400), (3, 50, 1040), (16, 33, 96)):
+        tl5 = rng.integers(0, 256, size=(N, oracle.tl5_row_bytes(K))).astype(np.uint8)
+        tl5[:, :16] = np.arange(256, dtype=np.uint16).reshape(16, 16)[np.arange(N) % 16].astype(np.uint8)
+        xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+        s = rng.uniform(0.5, 50.0, size=M).astype(np.float32)
+        check_forward_tl5(xq, s, tl5, 0.0213)
+
+
+def test_forward_tl5_extreme_accumulators():
+    """x_q = -128 against all +1 and all -1 rows: |acc| = 128 K at the int32 limit's side."""
+    K = 16 * 8192
+    xq = np.full((2, K), -128, dtype=np.int8)
+    c = np.zeros((3, K), dtype=np.int8)
+    c[0] = 1
+    c[1] = -1
+    c[2, ::2] = 1
+    tl5, _ = oracle.pack_tl5(c)
+    s = np.array([1.0, 3.0], dtype=np.float32)
+    acc = check_forward_tl5(xq, s, tl5, 0.5)
+    assert acc[0, 0] == -128 * K and acc[0, 1] == 128 * K and acc[0, 2] == -64 * K
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 28672, 8192), (4, 8192, 28672), (16, 8640, 3200)])
+def test_forward_tl5_full_size_matches_2bit_path(M, N, K):
+    """At full layer sizes: the five-per-byte forward equals the 2-bit decode forward bit
+    for bit (same exact accumulators, same rescale), and sampled rows equal the oracle."""
+    W = synth.weight(N, K, seed=N + K)
+    X = synth.activations(M, K, seed=M + K, outlier_frac=0.01, outlier_scale=20.0)
+    gamma, packed = B.quantize_weights(W.to(DEV), EPS)
+    xq, s = B.quantize_act(X.to(DEV), EPS)
+    tl5 = B.repack_tl5(packed)
+    for dt in (torch.int32, torch.float32, torch.bfloat16):
+        y5 = B.forward_tl5(xq, s, tl5, gamma, dt)
+        y2 = B.forward(xq, s, packed, gamma, dt, path=B.BL_PATH_GEMV)
+        sync()
+        assert torch.equal(y5, y2), dt
+    sel = np.array([0, M - 1])
+    acc = B.forward_tl5(xq, s, tl5, gamma, torch.int32).cpu().numpy()
+    codes = oracle.unpack_tl5(tl5.cpu().numpy(), K)
+    cols = np.random.default_rng(3).choice(N, size=64, replace=False)
+    acc_ref = oracle.int_matmul(xq.cpu().numpy()[sel], codes[cols])
+    assert np.array_equal(acc[np.ix_(sel, cols)], acc_ref)
