@@ -104,15 +104,23 @@ __global__ void __launch_bounds__(256) tl5_repack_kernel(const uint8_t* __restri
     }
 }
 
-// int8 codes (-1, 0, +1 per byte) of plane p for the four bytes of word w, given the
-// previous plane's h (0 before plane 0); h is updated.
+// Digits (0, 1, 2 per byte) of plane P for the four bytes whose even and odd bytes are
+// spread into the 16-bit lanes of `even` and `odd`, given the previous plane's h (0
+// before plane 0); h is updated.
 template <int P>
-__device__ __forceinline__ uint32_t tl5_plane(uint32_t even, uint32_t odd, uint32_t& h) {
+__device__ __forceinline__ uint32_t tl5_digits(uint32_t even, uint32_t odd, uint32_t& h) {
     constexpr uint32_t kMul = P == 0 ? 3u : P == 1 ? 9u : P == 2 ? 27u : P == 3 ? 81u : 243u;
     const uint32_t hn = __byte_perm(even * kMul, odd * kMul, 0x7351);
-    const uint32_t d = hn - 3u * h;  // digits 0..2 per byte, no borrow
+    const uint32_t d = hn - 3u * h;  // no borrow: every byte's difference is in [0, 2]
     h = hn;
-    return (d + 0x7F7F7F7Fu) ^ 0x80808080u;
+    return d;
+}
+
+// acc + sum of the four products of unsigned bytes a with signed bytes b
+__device__ __forceinline__ uint32_t dp4a_us(uint32_t a, uint32_t b, uint32_t acc) {
+    uint32_t d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(acc));
+    return d;
 }
 
 __device__ __forceinline__ void tl5_store(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -130,29 +138,96 @@ __device__ __forceinline__ void tl5_store(void* out, int kind, int64_t idx, int 
 // Decode GEMV: one warp per output row, lanes over the row's 16-byte blocks (kUnroll
 // blocks in flight per lane), MT tokens per pass (blockIdx.y selects the group of MT
 // tokens).  x_q row-major; its 16-byte pieces are read through L1, which every warp of
-// the SM shares.  A plane past K gets zero codes and reads an in-bounds piece of x_q.
+// the SM shares.
+//
+// The dot products use the digits t = c + 1 directly (unsigned bytes against the
+// signed x_q bytes) and subtract each token's sum of x_q once at the end:
+// sum_k c_k x_k = sum_k t_k x_k - sum_k x_k.  The block computes those sums first.  The
+// sums are exact modulo 2^32 and the result's magnitude is at most 128 K < 2^31, so the
+// wrapped unsigned arithmetic gives it exactly.  Only the last block of a row can miss
+// planes (K % 80 != 0): it alone checks each plane against K and skips the missing ones.
 constexpr int kTl5Warps = 8;
+constexpr int kTl5Threads = 32 * kTl5Warps;
 constexpr int kUnroll = 4;
 
+template <int MT, bool PARTIAL>
+__device__ __forceinline__ void tl5_block(const uint4 w, const int8_t* xb, int K, int kb, int mt,
+                                          uint32_t (&acc)[MT]) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    uint32_t ev[4], od[4], h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        ev[q] = __byte_perm(ww[q], 0u, 0x4240);  // bytes 0, 2 -> 16-bit lanes
+        od[q] = __byte_perm(ww[q], 0u, 0x4341);  // bytes 1, 3
+        h[q] = 0u;
+    }
+#pragma unroll
+    for (int p = 0; p < 5; ++p) {
+        if (PARTIAL && kb + 16 * p >= K) break;
+        uint32_t d[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (p == 0) d[q] = tl5_digits<0>(ev[q], od[q], h[q]);
+            if (p == 1) d[q] = tl5_digits<1>(ev[q], od[q], h[q]);
+            if (p == 2) d[q] = tl5_digits<2>(ev[q], od[q], h[q]);
+            if (p == 3) d[q] = tl5_digits<3>(ev[q], od[q], h[q]);
+            if (p == 4) d[q] = tl5_digits<4>(ev[q], od[q], h[q]);
+        }
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+            if (j < mt) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xb + static_cast<int64_t>(j) * K + 16 * p));
+                uint32_t a = acc[j];
+                a = dp4a_us(d[0], xv.x, a);
+                a = dp4a_us(d[1], xv.y, a);
+                a = dp4a_us(d[2], xv.z, a);
+                a = dp4a_us(d[3], xv.w, a);
+                acc[j] = a;
+            }
+        }
+    }
+}
+
 template <int MT>
-__global__ void __launch_bounds__(32 * kTl5Warps) gemv_tl5_kernel(const int8_t* __restrict__ xq,
-                                                                 const float* __restrict__ s,
-                                                                 const uint8_t* __restrict__ w5,
-                                                                 const float* __restrict__ gamma, int M, int N,
-                                                                 int K, int nblk, void* __restrict__ out,
-                                                                 int okind, int grow) {
+__global__ void __launch_bounds__(kTl5Threads) gemv_tl5_kernel(const int8_t* __restrict__ xq,
+                                                              const float* __restrict__ s,
+                                                              const uint8_t* __restrict__ w5,
+                                                              const float* __restrict__ gamma, int M, int N,
+                                                              int K, int nblk, void* __restrict__ out,
+                                                              int okind, int grow) {
     pdl_wait_then_release();
+    __shared__ uint32_t xsum[MT];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kTl5Warps + warp;
-    if (row >= N) return;
     const int m0 = blockIdx.y * MT;
     const int mt = M - m0 < MT ? M - m0 : MT;
-    const uint4* wr = reinterpret_cast<const uint4*>(w5 + row * static_cast<int64_t>(nblk) * kTl5BlockBytes);
     const int8_t* x0 = xq + static_cast<int64_t>(m0) * K;
 
-    int acc[MT];
+    // every token's sum of x_q, shared by the block's rows
+    if (threadIdx.x < MT) xsum[threadIdx.x] = 0u;
+    __syncthreads();
+    for (int j = 0; j < mt; ++j) {
+        uint32_t part = 0u;
+        const uint4* xr = reinterpret_cast<const uint4*>(x0 + static_cast<int64_t>(j) * K);
+        for (int i = threadIdx.x; i < K / 16; i += kTl5Threads) {
+            const uint4 xv = __ldg(xr + i);
+            part = dp4a_us(0x01010101u, xv.x, part);
+            part = dp4a_us(0x01010101u, xv.y, part);
+            part = dp4a_us(0x01010101u, xv.z, part);
+            part = dp4a_us(0x01010101u, xv.w, part);
+        }
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if (lane == 0) atomicAdd(&xsum[j], part);
+    }
+    __syncthreads();
+
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kTl5Warps + warp;
+    if (row >= N) return;
+    const uint4* wr = reinterpret_cast<const uint4*>(w5 + row * static_cast<int64_t>(nblk) * kTl5BlockBytes);
+    const int nfull = K / kTl5BlockCodes;  // blocks with all five planes inside K
+
+    uint32_t acc[MT];
 #pragma unroll
-    for (int j = 0; j < MT; ++j) acc[j] = 0;
+    for (int j = 0; j < MT; ++j) acc[j] = 0u;
 
     for (int b0 = 0; b0 < nblk; b0 += 32 * kUnroll) {
         uint4 wv[kUnroll];
@@ -164,45 +239,11 @@ __global__ void __launch_bounds__(32 * kTl5Warps) gemv_tl5_kernel(const int8_t* 
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int blk = b0 + lane + 32 * u;
-            if (blk >= nblk) break;
-            const uint32_t ww[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-            uint32_t ev[4], od[4], h[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                ev[q] = __byte_perm(ww[q], 0u, 0x4240);  // bytes 0, 2 -> 16-bit lanes
-                od[q] = __byte_perm(ww[q], 0u, 0x4341);  // bytes 1, 3
-                h[q] = 0u;
-            }
             const int kb = blk * kTl5BlockCodes;
-#pragma unroll
-            for (int p = 0; p < 5; ++p) {
-                uint32_t c[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (p == 0) c[q] = tl5_plane<0>(ev[q], od[q], h[q]);
-                    if (p == 1) c[q] = tl5_plane<1>(ev[q], od[q], h[q]);
-                    if (p == 2) c[q] = tl5_plane<2>(ev[q], od[q], h[q]);
-                    if (p == 3) c[q] = tl5_plane<3>(ev[q], od[q], h[q]);
-                    if (p == 4) c[q] = tl5_plane<4>(ev[q], od[q], h[q]);
-                }
-                const int k0 = kb + 16 * p;
-                const bool valid = k0 < K;
-                const int kx = valid ? k0 : 0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) c[q] = valid ? c[q] : 0u;
-#pragma unroll
-                for (int j = 0; j < MT; ++j) {
-                    if (j < mt) {
-                        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x0 + static_cast<int64_t>(j) * K + kx));
-                        int a = acc[j];
-                        a = __dp4a(static_cast<int>(c[0]), static_cast<int>(xv.x), a);
-                        a = __dp4a(static_cast<int>(c[1]), static_cast<int>(xv.y), a);
-                        a = __dp4a(static_cast<int>(c[2]), static_cast<int>(xv.z), a);
-                        a = __dp4a(static_cast<int>(c[3]), static_cast<int>(xv.w), a);
-                        acc[j] = a;
-                    }
-                }
-            }
+            if (blk < nfull)
+                tl5_block<MT, false>(wv[u], x0 + kb, K, kb, mt, acc);
+            else if (blk < nblk)
+                tl5_block<MT, true>(wv[u], x0 + kb, K, kb, mt, acc);
         }
     }
 #pragma unroll
@@ -214,9 +255,10 @@ __global__ void __launch_bounds__(32 * kTl5Warps) gemv_tl5_kernel(const int8_t* 
     for (int j = 0; j < MT; ++j) {
         if (lane == j && j < mt) {
             const int m = m0 + j;
+            const int a = static_cast<int>(acc[j] - xsum[j]);
             float fac = 0.0f;
             if (okind != kOutI32) fac = __fdiv_rn(grow ? gamma[row] : *gamma, s[m]);
-            tl5_store(out, okind, static_cast<int64_t>(m) * N + row, acc[j], fac);
+            tl5_store(out, okind, static_cast<int64_t>(m) * N + row, a, fac);
         }
     }
 }
@@ -233,7 +275,7 @@ template <int MT>
 cudaError_t launch_tl5_mt(const int8_t* xq, const float* s, const uint8_t* w5, const float* gamma, int64_t M,
                           int64_t N, int64_t K, void* out, int kind, cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>((N + kTl5Warps - 1) / kTl5Warps), static_cast<unsigned>((M + MT - 1) / MT));
-    return launch_pdl(gemv_tl5_kernel<MT>, grid, dim3(32 * kTl5Warps), 0, stream, dim3(kNoCluster), xq, s, w5,
+    return launch_pdl(gemv_tl5_kernel<MT>, grid, dim3(kTl5Threads), 0, stream, dim3(kNoCluster), xq, s, w5,
                       gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), tl5_blocks(K), out,
                       out_kind_of(kind), gamma_rows_of(kind));
 }
