@@ -104,12 +104,17 @@ __global__ void __launch_bounds__(256) tl5_repack_kernel(const uint8_t* __restri
     }
 }
 
-// Multipliers held in registers: a multiply by a register is one IMAD on the FMA
-// pipe, where a constant multiplier could become a chain of shifts and adds on the
-// integer ALU pipe, which the byte permutes already load.
-struct Tl5Mul {
-    uint32_t three, neg3;
-};
+// Digits (0, 1, 2 per byte) of plane P for the four bytes whose even and odd bytes are
+// spread into the 16-bit lanes of `even` and `odd`, given the previous plane's h (0
+// before plane 0); h is updated.
+template <int P>
+__device__ __forceinline__ uint32_t tl5_digits(uint32_t even, uint32_t odd, uint32_t& h) {
+    constexpr uint32_t kMul = P == 0 ? 3u : P == 1 ? 9u : P == 2 ? 27u : P == 3 ? 81u : 243u;
+    const uint32_t hn = __byte_perm(even * kMul, odd * kMul, 0x7351);
+    const uint32_t d = hn - 3u * h;  // no borrow: every byte's difference is in [0, 2]
+    h = hn;
+    return d;
+}
 
 // acc + sum of the four products of unsigned bytes a with signed bytes b
 __device__ __forceinline__ uint32_t dp4a_us(uint32_t a, uint32_t b, uint32_t acc) {
@@ -147,14 +152,13 @@ constexpr int kUnroll = 4;
 
 template <int MT, bool PARTIAL>
 __device__ __forceinline__ void tl5_block(const uint4 w, const int8_t* xb, int K, int kb, int mt,
-                                          const Tl5Mul& k, uint32_t (&acc)[MT]) {
+                                          uint32_t (&acc)[MT]) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-    // even / odd bytes of each word in 16-bit lanes, times 3^(p+1) as the planes advance
-    uint32_t ye[4], yo[4], h[4];
+    uint32_t ev[4], od[4], h[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        ye[q] = __byte_perm(ww[q], 0u, 0x4240);  // bytes 0, 2
-        yo[q] = __byte_perm(ww[q], 0u, 0x4341);  // bytes 1, 3
+        ev[q] = __byte_perm(ww[q], 0u, 0x4240);  // bytes 0, 2 -> 16-bit lanes
+        od[q] = __byte_perm(ww[q], 0u, 0x4341);  // bytes 1, 3
         h[q] = 0u;
     }
 #pragma unroll
@@ -163,12 +167,11 @@ __device__ __forceinline__ void tl5_block(const uint4 w, const int8_t* xb, int K
         uint32_t d[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            ye[q] = (ye[q] << 1) + ye[q];  // x 3 as one shift-add
-            yo[q] = yo[q] * k.three;       // x 3 as one multiply
-            // floor(B 3^(p+1) / 256) of the four bytes, then digit p = h_p - 3 h_(p-1)
-            const uint32_t hn = __byte_perm(ye[q], yo[q], 0x7351);
-            d[q] = hn + k.neg3 * h[q];  // no borrow: every byte's difference is in [0, 2]
-            h[q] = hn;
+            if (p == 0) d[q] = tl5_digits<0>(ev[q], od[q], h[q]);
+            if (p == 1) d[q] = tl5_digits<1>(ev[q], od[q], h[q]);
+            if (p == 2) d[q] = tl5_digits<2>(ev[q], od[q], h[q]);
+            if (p == 3) d[q] = tl5_digits<3>(ev[q], od[q], h[q]);
+            if (p == 4) d[q] = tl5_digits<4>(ev[q], od[q], h[q]);
         }
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
@@ -191,12 +194,9 @@ __global__ void __launch_bounds__(kTl5Threads) gemv_tl5_kernel(const int8_t* __r
                                                               const uint8_t* __restrict__ w5,
                                                               const float* __restrict__ gamma, int M, int N,
                                                               int K, int nblk, void* __restrict__ out,
-                                                              int okind, int grow, Tl5Mul mul_arg) {
+                                                              int okind, int grow) {
     pdl_wait_then_release();
     __shared__ uint32_t xsum[MT];
-    Tl5Mul mul;
-    asm volatile("mov.b32 %0, %2;\n\tmov.b32 %1, %3;" : "=r"(mul.three), "=r"(mul.neg3)
-                 : "r"(mul_arg.three), "r"(mul_arg.neg3));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * MT;
     const int mt = M - m0 < MT ? M - m0 : MT;
@@ -241,9 +241,9 @@ __global__ void __launch_bounds__(kTl5Threads) gemv_tl5_kernel(const int8_t* __r
             const int blk = b0 + lane + 32 * u;
             const int kb = blk * kTl5BlockCodes;
             if (blk < nfull)
-                tl5_block<MT, false>(wv[u], x0 + kb, K, kb, mt, mul, acc);
+                tl5_block<MT, false>(wv[u], x0 + kb, K, kb, mt, acc);
             else if (blk < nblk)
-                tl5_block<MT, true>(wv[u], x0 + kb, K, kb, mt, mul, acc);
+                tl5_block<MT, true>(wv[u], x0 + kb, K, kb, mt, acc);
         }
     }
 #pragma unroll
@@ -277,7 +277,7 @@ cudaError_t launch_tl5_mt(const int8_t* xq, const float* s, const uint8_t* w5, c
     const dim3 grid(static_cast<unsigned>((N + kTl5Warps - 1) / kTl5Warps), static_cast<unsigned>((M + MT - 1) / MT));
     return launch_pdl(gemv_tl5_kernel<MT>, grid, dim3(kTl5Threads), 0, stream, dim3(kNoCluster), xq, s, w5,
                       gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), tl5_blocks(K), out,
-                      out_kind_of(kind), gamma_rows_of(kind), Tl5Mul{3u, 0xFFFFFFFDu});
+                      out_kind_of(kind), gamma_rows_of(kind));
 }
 
 }  // namespace
