@@ -63,6 +63,10 @@ class Oracle:
         L.oracle_unpack_tl5.restype = None
         L.oracle_forward_tl5.argtypes = [P, P, P, F, I, I, I, ctypes.c_int, P, P, P, P]
         L.oracle_forward_tl5.restype = I
+        L.oracle_ste_grad_input.argtypes = [P, P, F, I, I, I, P, P]
+        L.oracle_ste_grad_input.restype = None
+        L.oracle_ste_grad_weight.argtypes = [P, P, P, F, I, I, I, P]
+        L.oracle_ste_grad_weight.restype = None
         self.L = L
         self.path = path
 
@@ -226,6 +230,28 @@ class Oracle:
         assert over == 0, "int32 overflow in the oracle accumulator"
         return out
 
+    def ste_grad_input(self, dY, packed, gamma, K):
+        """dX = gamma dY C under the straight-through estimator (oracle_ste_grad_input)."""
+        dY, pd = _c(dY, np.float32)
+        packed, pp = _c(packed, np.uint8)
+        M, N = dY.shape
+        assert packed.shape == (N, K // 4)
+        dX = np.empty((M, K), dtype=np.float32)
+        codes_tmp = np.empty((N, K), dtype=np.int8)
+        self.L.oracle_ste_grad_input(pd, pp, float(gamma), M, N, K, _vp(dX), _vp(codes_tmp))
+        return dX
+
+    def ste_grad_weight(self, dY, xq, s, gamma):
+        """dW = gamma sum_m dY[m,n] x_q[m,k] / s[m] (oracle_ste_grad_weight)."""
+        dY, pd = _c(dY, np.float32)
+        xq, px = _c(xq, np.int8)
+        M, N = dY.shape
+        K = xq.shape[1]
+        s, ps = _c(np.asarray(s, dtype=np.float32).reshape(M), np.float32)
+        dW = np.empty((N, K), dtype=np.float32)
+        self.L.oracle_ste_grad_weight(pd, px, ps, float(gamma), M, N, K, _vp(dW))
+        return dW
+
 _default = None
 
 
@@ -254,3 +280,5 @@ def unpack_tl5(packed, K): return default().unpack_tl5(packed, K)
 def tl5_row_bytes(K): return default().tl5_row_bytes(K)
 def forward_tl5(xq, s, packed, gamma, K, out_kind=OUT_F32):
     return default().forward_tl5(xq, s, packed, gamma, K, out_kind)
+def ste_grad_input(dY, packed, gamma, K): return default().ste_grad_input(dY, packed, gamma, K)
+def ste_grad_weight(dY, xq, s, gamma): return default().ste_grad_weight(dY, xq, s, gamma)

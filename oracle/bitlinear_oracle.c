@@ -378,3 +378,42 @@ int64_t oracle_forward_tl5(const int8_t *xq, const float *s, const uint8_t *pack
     oracle_f32_to_bf16(y_tmp, M * N, (uint16_t *)out);
     return over;
 }
+
+/* ------------------------------------------- straight-through backward (STE) -- */
+
+/* [STE] the forward uses the ternary weights while the gradient reaches the shadow
+ * weights as if the quantisation were the identity.  With this library's forward
+ * y[m,n] = (sum_k c[n,k] x_q[m,k]) * gamma / s[m], and both quantisers passed straight
+ * through (x_q = round(s x) with d x_q / d x = s, gamma and s held constant):
+ *   dX[m,k] = gamma * sum_n dY[m,n] c[n,k]
+ *   dW[n,k] = gamma * sum_m dY[m,n] x_q[m,k] / s[m]
+ * Both sums run in index order in double precision and are rounded once to fp32.
+ * codes_tmp must hold N*K bytes. */
+void oracle_ste_grad_input(const float *dY, const uint8_t *packed, float gamma, int64_t M, int64_t N,
+                           int64_t K, float *dX, int8_t *codes_tmp)
+{
+    int64_t m, n, k;
+    oracle_unpack(packed, N, K, codes_tmp);
+    for (m = 0; m < M; ++m) {
+        for (k = 0; k < K; ++k) {
+            double sum = 0.0;
+            for (n = 0; n < N; ++n)
+                sum += (double)dY[m * N + n] * (double)codes_tmp[n * K + k];
+            dX[m * K + k] = (float)((double)gamma * sum);
+        }
+    }
+}
+
+void oracle_ste_grad_weight(const float *dY, const int8_t *xq, const float *s, float gamma, int64_t M,
+                            int64_t N, int64_t K, float *dW)
+{
+    int64_t m, n, k;
+    for (n = 0; n < N; ++n) {
+        for (k = 0; k < K; ++k) {
+            double sum = 0.0;
+            for (m = 0; m < M; ++m)
+                sum += (double)dY[m * N + n] * (double)xq[m * K + k] / (double)s[m];
+            dW[n * K + k] = (float)((double)gamma * sum);
+        }
+    }
+}

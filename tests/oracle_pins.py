@@ -490,11 +490,65 @@ def pin_tl5_padding_not_read(O):
     assert np.array_equal(p5, (((t[:, 0] * 81 + t[:, 1] * 27 + t[:, 2] * 9 + 4) * 256 + 242) // 243).astype(np.uint8))
 
 
+# ------------------------------------------------ straight-through backward (STE) --
+
+def pin_hand_ste(O):
+    """Hand-worked gradients of the straight-through backward (golden file)."""
+    n = 0
+    for kind, r in parse_golden("hand_cases.txt"):
+        if kind != "ste":
+            continue
+        M, N, K = int(r["M"]), int(r["N"]), int(r["K"])
+        g = float(r["gamma"])
+        dY = _floats(r["dY"]).reshape(M, N)
+        codes = _ints(r["codes"], np.int8).reshape(N, K)
+        xq = _ints(r["xq"], np.int8).reshape(M, K)
+        s = _floats(r["s"]).reshape(M)
+        packed, _ = O.pack(codes)
+        assert np.array_equal(O.ste_grad_input(dY, packed, g, K), _floats(r["dX"]).reshape(M, K))
+        assert np.array_equal(O.ste_grad_weight(dY, xq, s, g), _floats(r["dW"]).reshape(N, K))
+        n += 1
+    assert n >= 2
+
+
+def pin_ste_vs_autograd(O):
+    """The pages' quantisation-aware-training forward, written in torch float64 with the
+    straight-through estimator (W_eff = W_fp + (W_tern - W_fp).detach(), and the same
+    for the activation quantiser), differentiated by autograd: its gradients for the
+    shadow weights and for the quantiser's input equal the oracle's, given the same
+    codes, x_q, s and gamma."""
+    rng = np.random.default_rng(37)
+    for M, N, K in ((1, 3, 8), (5, 7, 12), (9, 16, 40)):
+        W = torch.from_numpy(rng.normal(0.0, 0.02, size=(N, K)))
+        x = torch.from_numpy(rng.normal(0.0, 1.0, size=(M, K)))
+        gamma = torch.tensor(float(np.float32(W.abs().mean().item() + 1e-5)), dtype=torch.float64)
+        W_tern = torch.clamp(torch.round(W / gamma), -1, 1)
+        s = torch.from_numpy((127.0 / x.abs().amax(dim=1).numpy()).astype(np.float32).astype(np.float64))
+        x_q = torch.clamp(torch.round(x * s[:, None]), -128, 127)
+        dY = torch.from_numpy(rng.normal(0.0, 1.0, size=(M, N)).astype(np.float32).astype(np.float64))
+
+        W_fp = W.clone().requires_grad_(True)
+        x_in = x.clone().requires_grad_(True)
+        W_eff = W_fp + (W_tern - W_fp).detach()
+        xs = x_in * s[:, None]
+        x_q_ste = xs + (x_q - xs).detach()
+        y = (x_q_ste @ W_eff.T) * (gamma / s)[:, None]
+        y.backward(dY)
+
+        packed, _ = O.pack(W_tern.numpy().astype(np.int8))
+        dX = O.ste_grad_input(dY.numpy().astype(np.float32), packed, gamma.item(), K)
+        dW = O.ste_grad_weight(dY.numpy().astype(np.float32), x_q.numpy().astype(np.int8),
+                               s.numpy().astype(np.float32), gamma.item())
+        for got, want in ((dX, x_in.grad.numpy()), (dW, W_fp.grad.numpy())):
+            assert np.allclose(got, want, rtol=2.0 ** -22, atol=1e-30), (M, N, K, np.abs(got - want).max())
+
+
 def _bf16_to_f32(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
 ALL_PINS = [
+    pin_hand_ste, pin_ste_vs_autograd,
     pin_hand_tl5, pin_tl5_every_value, pin_tl5_size_and_equivalence, pin_tl5_padding_not_read,
     pin_hand_norm, pin_norm_vs_torch, pin_norm_invariants, pin_dequant_rows,
     pin_hand_ternarise, pin_hand_absmean, pin_hand_act, pin_hand_pack, pin_hand_matmul,

@@ -61,6 +61,14 @@ MUTANTS = [
     ("tl5_interleaved", "int64_t k = 80 * b + 16 * p + j;", "int64_t k = 80 * b + 5 * j + p;"),
     ("tl5_pad_minus_one", "int t = 1;\n", "int t = 0;\n"),
     ("tl5_decode_255", "unsigned v = byte * 243u / 256u;", "unsigned v = byte * 243u / 255u;"),
+    ("ste_dx_no_gamma", "dX[m * K + k] = (float)((double)gamma * sum);", "dX[m * K + k] = (float)sum;"),
+    ("ste_dx_codes_transposed", "sum += (double)dY[m * N + n] * (double)codes_tmp[n * K + k];",
+     "sum += (double)dY[m * N + n] * (double)codes_tmp[k * N + n];"),
+    ("ste_dw_times_s", "sum += (double)dY[m * N + n] * (double)xq[m * K + k] / (double)s[m];",
+     "sum += (double)dY[m * N + n] * (double)xq[m * K + k] * (double)s[m];"),
+    ("ste_dw_no_gamma", "dW[n * K + k] = (float)((double)gamma * sum);", "dW[n * K + k] = (float)sum;"),
+    ("ste_dw_token_index", "sum += (double)dY[m * N + n] * (double)xq[m * K + k] / (double)s[m];",
+     "sum += (double)dY[m * N + n] * (double)xq[m * K + k] / (double)s[0];"),
 ]
 
 
