@@ -54,7 +54,7 @@ def parse():
     p.add_argument("--weight-format", choices=["2bit", "tl5"], default="2bit",
                    help="--sweep: the 2-bit forward, or the five-codes-per-byte decode forward (M <= 16 shapes)")
     p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack",
-                                        "forward_tl5", "repack_tl5"],
+                                        "forward_tl5", "repack_tl5", "ste_input", "ste_weight"],
                    help="time one entry point on one shape instead of the step (kernel study, ncu)")
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
@@ -529,6 +529,23 @@ def run_single(args):
         ops = 2 * M * N * K
         wbytes = N * B.bitlinear_tl5_row_bytes(K)
         nbytes = wbytes + M * K + 4 * M + M * N * out.element_size()
+    elif args.single in ("ste_input", "ste_weight"):
+        # the straight-through backward: dX = gamma dY C, or dW = gamma dY^T (x_q / s)
+        dY = torch.randn(M, N, device=dev) * 1e-3
+        gamma = torch.tensor([0.02], device=dev)
+        if args.single == "ste_input":
+            packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+            B.bitlinear_pack(synth.codes(N, K, seed=1).to(dev), packed)
+            dX = torch.empty(M, K, device=dev)
+            fn = lambda: B.bitlinear_ste_backward_input(dY, packed, gamma, dX)
+            nbytes = 4 * M * N + N * K // 4 + 4 * M * K
+        else:
+            xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev)
+            s = torch.rand(M, device=dev) + 1.0
+            dW = torch.empty(N, K, device=dev)
+            fn = lambda: B.bitlinear_ste_backward_weight(dY, xq, s, gamma, dW)
+            nbytes = 4 * M * N + M * K + 4 * M + 4 * N * K
+        ops = 2 * M * N * K
     elif args.single == "repack_tl5":
         packed = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
         B.bitlinear_pack(synth.codes(N, K, seed=1).to(dev), packed)
@@ -572,7 +589,12 @@ def run_single(args):
                           round(wbytes / t / 1e9, 1) if args.single == "forward_tl5" else None)}
     if ops:
         rec["tops"] = round(ops / t / 1e12, 2)
-        rec["int8_frac"] = round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4)
+        if args.single in ("ste_input", "ste_weight"):
+            # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (nominal)
+            rec["fp32_simt_peak_tflops"] = 74.4
+            rec["fp32_simt_frac"] = round(ops / t / 1e12 / 74.4, 4)
+        else:
+            rec["int8_frac"] = round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4)
     print(json.dumps(rec), flush=True)
 
 

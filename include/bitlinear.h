@@ -303,6 +303,38 @@ BL_API bl_status bitlinear_forward_tl5(const int8_t *xq, const float *s, const u
                                        const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
                                        bl_dtype out_dtype, void *stream);
 
+/* ----------------------------------------------------------------------------------
+ * Straight-through backward (quantisation-aware training).
+ * [STE] the forward uses the ternary weights; the backward treats the quantisation as
+ * the identity, so the gradient reaches the full-precision shadow weights.  For the
+ * forward y[m, n] = (sum_k c[n, k] x_q[m, k]) * gamma / s[m] with both quantisers
+ * passed straight through (d x_q / d x = s; gamma and s held constant):
+ *   dX[m, k] = gamma * sum_n dY[m, n] c[n, k]
+ *   dW[n, k] = gamma * sum_m dY[m, n] x_q[m, k] / s[m]
+ * dX is the gradient for the quantiser's input (the normalised activations), dW the
+ * gradient for the shadow weights.  The sums run in fp32 (each product with a code is
+ * exact; dY / s[m] is one IEEE division), the result is scaled by gamma once.
+ * ---------------------------------------------------------------------------------- */
+
+/*   dY     in  : fp32 [M, N], device.
+ *   packed in  : uint8 [N, K/4] 2-bit codes (the forward's weights), device.
+ *   gamma  in  : device fp32 scalar.
+ *   dX     out : fp32 [M, K], device.
+ * K % 4 == 0; M, N, K < 2^31; M <= 65535 * 64.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_ste_backward_input(const float *dY, const uint8_t *packed, const float *gamma,
+                                              int64_t M, int64_t N, int64_t K, float *dX, void *stream);
+
+/*   dY    in  : fp32 [M, N], device.
+ *   xq, s in  : the forward's int8 [M, K] row-major activations and fp32 [M] scales, device.
+ *   gamma in  : device fp32 scalar.
+ *   dW    out : fp32 [N, K], device.
+ * M, N, K < 2^31; N <= 65535 * 64.
+ * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
+BL_API bl_status bitlinear_ste_backward_weight(const float *dY, const int8_t *xq, const float *s,
+                                               const float *gamma, int64_t M, int64_t N, int64_t K, float *dW,
+                                               void *stream);
+
 /* CUDA error code (cudaError_t as int) of the last BL_ERR_CUDA on the calling thread. */
 BL_API int bitlinear_last_cuda_error(void);
 

@@ -33,6 +33,7 @@ EXPORTED = [
     "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
     "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_forward_rowscale",
     "bitlinear_tl5_row_bytes", "bitlinear_pack_tl5", "bitlinear_repack_tl5", "bitlinear_forward_tl5",
+    "bitlinear_ste_backward_input", "bitlinear_ste_backward_weight",
     "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_repack_tl5.restype = S
         L.bitlinear_forward_tl5.argtypes = [P, P, P, P, I64, I64, I64, P, S, P]
         L.bitlinear_forward_tl5.restype = S
+        L.bitlinear_ste_backward_input.argtypes = [P, P, P, I64, I64, I64, P, P]
+        L.bitlinear_ste_backward_input.restype = S
+        L.bitlinear_ste_backward_weight.argtypes = [P, P, P, P, I64, I64, I64, P, P]
+        L.bitlinear_ste_backward_weight.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
         L.bitlinear_last_cuda_error.restype = ctypes.c_int
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
@@ -242,6 +247,24 @@ def bitlinear_forward_tl5(xq, s, tl5, gamma, out, stream=None):
         M, N, K, _dev(out, out.dtype, "out", (M, N)), kind, _stream(stream)), "bitlinear_forward_tl5")
 
 
+def bitlinear_ste_backward_input(dY, packed, gamma, dX, stream=None):
+    M, N = dY.shape
+    K = 4 * packed.shape[1]
+    _check(lib().bitlinear_ste_backward_input(
+        _dev(dY, torch.float32, "dY"), _dev(packed, torch.uint8, "packed", (N, K // 4)),
+        _dev(gamma, torch.float32, "gamma"), M, N, K, _dev(dX, torch.float32, "dX", (M, K)), _stream(stream)),
+        "bitlinear_ste_backward_input")
+
+
+def bitlinear_ste_backward_weight(dY, xq, s, gamma, dW, stream=None):
+    M, N = dY.shape
+    K = xq.shape[1]
+    _check(lib().bitlinear_ste_backward_weight(
+        _dev(dY, torch.float32, "dY"), _dev(xq, torch.int8, "xq", (M, K)), _dev(s, torch.float32, "s", (M,)),
+        _dev(gamma, torch.float32, "gamma"), M, N, K, _dev(dW, torch.float32, "dW", (N, K)), _stream(stream)),
+        "bitlinear_ste_backward_weight")
+
+
 # ----------------------------------------------------------- allocating helpers --
 
 def quantize_weights(W: torch.Tensor, eps: float = 1e-5, stream=None):
@@ -302,3 +325,14 @@ def forward_tl5(xq, s, tl5, gamma, out_dtype=torch.float32, stream=None):
     out = torch.empty(xq.shape[0], tl5.shape[0], dtype=out_dtype, device=xq.device)
     bitlinear_forward_tl5(xq, s, tl5, gamma, out, stream)
     return out
+
+
+def ste_backward(dY, packed, xq, s, gamma, stream=None):
+    """(dX [M, K], dW [N, K]) fp32: the straight-through gradients of the forward."""
+    M, N = dY.shape
+    K = 4 * packed.shape[1]
+    dX = torch.empty(M, K, dtype=torch.float32, device=dY.device)
+    dW = torch.empty(N, K, dtype=torch.float32, device=dY.device)
+    bitlinear_ste_backward_input(dY, packed, gamma, dX, stream)
+    bitlinear_ste_backward_weight(dY, xq, s, gamma, dW, stream)
+    return dX, dW

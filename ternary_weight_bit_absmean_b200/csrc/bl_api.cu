@@ -213,6 +213,27 @@ bl_status bitlinear_forward_tl5(const int8_t* xq, const float* s, const uint8_t*
                                            as_stream(stream)));
 }
 
+bl_status bitlinear_ste_backward_input(const float* dY, const uint8_t* packed, const float* gamma, int64_t M,
+                                       int64_t N, int64_t K, float* dX, void* stream) {
+    if (dY == nullptr || packed == nullptr || gamma == nullptr || dX == nullptr) return BL_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || N >= lim || K >= lim || M > int64_t(65535) * 64) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(dY) || !aligned16(packed) || !aligned16(dX)) return BL_ERR_MISALIGNED;
+    return cuda_status(bl::launch_ste_grad_input(dY, packed, gamma, M, N, K, dX, as_stream(stream)));
+}
+
+bl_status bitlinear_ste_backward_weight(const float* dY, const int8_t* xq, const float* s, const float* gamma,
+                                        int64_t M, int64_t N, int64_t K, float* dW, void* stream) {
+    if (dY == nullptr || xq == nullptr || s == nullptr || gamma == nullptr || dW == nullptr) return BL_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || N >= lim || K >= lim || N > int64_t(65535) * 64) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(dY) || !aligned16(xq) || !aligned16(s) || !aligned16(dW)) return BL_ERR_MISALIGNED;
+    return cuda_status(bl::launch_ste_grad_weight(dY, xq, s, gamma, M, N, K, dW, as_stream(stream)));
+}
+
 bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                                    int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
                                    int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {

@@ -75,6 +75,12 @@ cudaError_t launch_tl5_repack(const uint8_t* packed, int64_t N, int64_t K, uint8
 cudaError_t launch_gemv_tl5(const int8_t* xq, const float* s, const uint8_t* w5, const float* gamma, int64_t M,
                             int64_t N, int64_t K, void* out, int kind, cudaStream_t stream);
 
+// The straight-through backward (k_ste.cu): dX = gamma dY C, dW = gamma dY^T (x_q / s).
+cudaError_t launch_ste_grad_input(const float* dY, const uint8_t* packed, const float* gamma, int64_t M, int64_t N,
+                                  int64_t K, float* dX, cudaStream_t stream);
+cudaError_t launch_ste_grad_weight(const float* dY, const int8_t* xq, const float* s, const float* gamma, int64_t M,
+                                   int64_t N, int64_t K, float* dW, cudaStream_t stream);
+
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);
 

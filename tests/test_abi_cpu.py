@@ -156,6 +156,21 @@ def test_tl5_entry_points_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, ODD, 0, None) == MISALIGNED
 
 
+def test_ste_backward_validation(L):
+    fi = L.bitlinear_ste_backward_input
+    assert fi(None, FAKE, FAKE, 4, 8, 64, FAKE, None) == INVALID
+    assert fi(FAKE, FAKE, FAKE, 0, 8, 64, FAKE, None) == INVALID
+    assert fi(FAKE, FAKE, FAKE, 4, 8, 66, FAKE, None) == SHAPE          # K % 4
+    assert fi(FAKE, FAKE, FAKE, 65535 * 64 + 1, 8, 64, FAKE, None) == SHAPE
+    assert fi(FAKE, ODD, FAKE, 4, 8, 64, FAKE, None) == MISALIGNED
+    fw = L.bitlinear_ste_backward_weight
+    assert fw(FAKE, FAKE, FAKE, None, 4, 8, 64, FAKE, None) == INVALID
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, -8, 64, FAKE, None) == INVALID
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 65535 * 64 + 1, 64, FAKE, None) == SHAPE
+    assert fw(FAKE, FAKE, ODD, FAKE, 4, 8, 64, FAKE, None) == MISALIGNED
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, ODD, None) == MISALIGNED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     from ternary_weight_bit_absmean_b200 import binding
     monkeypatch.setattr(binding, "_lib", None)

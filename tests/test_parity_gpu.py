@@ -786,3 +786,65 @@ def test_forward_tl5_full_size_matches_2bit_path(M, N, K):
     cols = np.random.default_rng(3).choice(N, size=64, replace=False)
     acc_ref = oracle.int_matmul(xq.cpu().numpy()[sel], codes[cols])
     assert np.array_equal(acc[np.ix_(sel, cols)], acc_ref)
+
+
+# ------------------------------------------------ straight-through backward (STE) --
+
+def _ste_inputs(M, N, K, seed):
+    W = synth.weight(N, K, seed=seed)
+    X = synth.activations(M, K, seed=seed + 1, outlier_frac=0.01, outlier_scale=20.0)
+    g_ref, _, packed_ref = oracle.quantize_weights(W.numpy(), EPS)
+    xq_ref, s_ref = oracle.quantize_act(bits(X), EPS)
+    dY = (torch.randn(M, N, generator=torch.Generator().manual_seed(seed + 2)) * 1e-3).numpy()
+    return g_ref, packed_ref, xq_ref, s_ref, dY
+
+
+def _assert_within_sum_bound(got, want, abs_terms, n_terms, gamma, what):
+    """|got - want| <= gamma (n + 3) 2^-24 sum|terms| + 2^-24 |want|: the worst-case error
+    of an fp32 recursive sum of n terms, one division per term and one final scaling."""
+    bound = float(gamma) * (n_terms + 3) * 2.0 ** -24 * abs_terms + 2.0 ** -24 * np.abs(want) + 1e-30
+    err = np.abs(got.astype(np.float64) - want.astype(np.float64))
+    assert (err <= bound).all(), (what, float((err / bound).max()))
+
+
+STE_CASES = [(1, 1, 4), (3, 17, 36), (64, 64, 64), (65, 100, 132), (7, 1536, 1536), (130, 300, 1000)]
+
+
+@pytest.mark.parametrize("M,N,K", STE_CASES)
+def test_ste_backward(M, N, K):
+    g, packed, xq, s, dY = _ste_inputs(M, N, K, seed=M + 2 * N + 3 * K)
+    gd = torch.tensor([g], dtype=torch.float32, device=DEV)
+    dX = guarded_empty((M, K), torch.float32)
+    dW = guarded_empty((N, K), torch.float32)
+    B.bitlinear_ste_backward_input(torch.from_numpy(dY).to(DEV), torch.from_numpy(packed).to(DEV), gd, dX)
+    B.bitlinear_ste_backward_weight(torch.from_numpy(dY).to(DEV), torch.from_numpy(xq).to(DEV),
+                                    torch.from_numpy(s).to(DEV), gd, dW)
+    sync()
+    check_guard(dX)
+    check_guard(dW)
+    codes = oracle.unpack(packed, K).astype(np.float64)
+    _assert_within_sum_bound(dX.cpu().numpy(), oracle.ste_grad_input(dY, packed, g, K),
+                             np.abs(dY.astype(np.float64)) @ np.abs(codes), N, g, "dX")
+    xs = np.abs(xq.astype(np.float64) / s.astype(np.float64)[:, None])
+    _assert_within_sum_bound(dW.cpu().numpy(), oracle.ste_grad_weight(dY, xq, s, g),
+                             np.abs(dY.astype(np.float64)).T @ xs, M, g, "dW")
+
+
+def test_ste_backward_full_size_sampled():
+    """A LLaMA-700M-shaped q projection at 4096 tokens: sampled rows of dX and dW against
+    the oracle (which sees only those rows / output features)."""
+    M, N, K = 4096, 1536, 1536
+    g, packed, xq, s, dY = _ste_inputs(M, N, K, seed=11)
+    gd = torch.tensor([g], dtype=torch.float32, device=DEV)
+    dX, dW = B.ste_backward(torch.from_numpy(dY).to(DEV), torch.from_numpy(packed).to(DEV),
+                            torch.from_numpy(xq).to(DEV), torch.from_numpy(s).to(DEV), gd)
+    sync()
+    rm = np.array([0, 1, 2047, 4095])
+    codes = oracle.unpack(packed, K).astype(np.float64)
+    _assert_within_sum_bound(dX.cpu().numpy()[rm], oracle.ste_grad_input(dY[rm], packed, g, K),
+                             np.abs(dY[rm].astype(np.float64)) @ np.abs(codes), N, g, "dX rows")
+    rn = np.array([0, 777, 1535])
+    xs = np.abs(xq.astype(np.float64) / s.astype(np.float64)[:, None])
+    want = oracle.ste_grad_weight(np.ascontiguousarray(dY[:, rn]), xq, s, g)
+    _assert_within_sum_bound(dW.cpu().numpy()[rn], want, np.abs(dY[:, rn].astype(np.float64)).T @ xs, M, g,
+                             "dW rows")
