@@ -30,6 +30,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -146,8 +147,10 @@ class ClockSampler:
 
     def start(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % self.index)
+            # the raw samples go to $BITLINEAR_BENCH_OUT (default: the system temp dir)
+            out_dir = os.environ.get("BITLINEAR_BENCH_OUT") or tempfile.gettempdir()
+            os.makedirs(out_dir, exist_ok=True)
+            self.path = os.path.join(out_dir, "clocks_rank%d.csv" % self.index)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
                                           "--format=csv,noheader,nounits", "-lms", "100"],
