@@ -22,8 +22,8 @@
 // of a word are spread into 16-bit lanes (B 3^5 <= 61965 fits a lane), multiplied by
 // 3^(p+1), and byte 1 of every lane (the floor by 256) is gathered back into one word
 // with a byte permute.  h_p - 3 h_(p-1) over a whole word has no borrow (every byte's
-// difference is in [0, 2]); adding 0x7F to each byte and flipping bit 7 turns digits
-// 0, 1, 2 into the int8 codes -1, 0, +1, which a dp4a multiplies with 4 bytes of x_q.
+// difference is in [0, 2]).  The digits t = c + 1 meet 4 bytes of x_q in one dp4a
+// (unsigned by signed bytes), and each token's sum of x_q is subtracted once at the end.
 // The four bytes of a word sit at k = 80 b + 16 p + 4 q .. + 3 for word q of the block,
 // contiguous in a row-major x_q row.
 #include <cuda_bf16.h>
