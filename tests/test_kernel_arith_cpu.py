@@ -157,3 +157,78 @@ def test_tl5_row_sum_with_token_sum_correction():
                             acc = _dp4a_us(digits[p], xw, acc)
                 r = (acc - xs) & M32
                 assert (r - (1 << 32) if r & 0x80000000 else r) == ref[m, n], (K, m, n)
+
+
+# ----------------------------------------- the table unpacks of the other layouts --
+
+def _code_table():
+    return int(re.search(r"constexpr uint32_t kCodeTable = (0x[0-9A-Fa-f]+)u;", _src("bl_device.cuh")).group(1), 16)
+
+
+def _words_under_test():
+    rng = np.random.default_rng(9)
+    words = [int(v) for v in rng.integers(0, 2 ** 32, size=3000, dtype=np.uint64)]
+    words += [0, M32, 0x55555555, 0xAAAAAAAA]
+    for pos in range(4):
+        words += [b << (8 * pos) for b in range(256)]
+    return words
+
+
+def _as_int8(word):
+    return [((word >> (8 * i)) & 0xFF) - (256 if (word >> (8 * i)) & 0x80 else 0) for i in range(4)]
+
+
+def test_natural_and_evenodd_unpacks_match_the_2bit_decode():
+    """unpack16_natural (nibble spread, then a table byte per code) and unpack16_evenodd
+    (two masks, then table bytes) give the oracle's codes in their stated orders."""
+    tab = _code_table()
+    words = _words_under_test()
+    packed = np.array(words, dtype=np.uint32).view(np.uint8).reshape(-1, 4)
+    codes = oracle.unpack(packed, 16)
+    for w, c in zip(words, codes):
+        lo, hi = prmt(w, 0, 0x4140), prmt(w, 0, 0x4342)
+        lo = (lo | (lo << 4)) & 0x0F0F0F0F
+        hi = (hi | (hi << 4)) & 0x0F0F0F0F
+        lo = (lo | (lo << 2)) & 0x33333333
+        hi = (hi | (hi << 2)) & 0x33333333
+        nat = _as_int8(prmt(tab, 0, lo & 0xFFFF)) + _as_int8(prmt(tab, 0, lo >> 16)) + \
+            _as_int8(prmt(tab, 0, hi & 0xFFFF)) + _as_int8(prmt(tab, 0, hi >> 16))
+        assert nat == list(c), hex(w)
+        sa, sb = w & 0x33333333, (w >> 2) & 0x33333333
+        e0, e1 = _as_int8(prmt(tab, 0, sa & 0xFFFF)), _as_int8(prmt(tab, 0, sa >> 16))
+        o0, o1 = _as_int8(prmt(tab, 0, sb & 0xFFFF)), _as_int8(prmt(tab, 0, sb >> 16))
+        assert e0 + e1 == list(c[0::2]) and o0 + o1 == list(c[1::2]), hex(w)
+
+
+# ---------------------------------------------------- the activation quantiser --
+
+def test_act_quant_rounding_by_magic_add_is_rint():
+    """q8_bits rounds x s by adding 1.5 * 2^23 in fp32: the low byte of the sum's bits is
+    rint(x s) (half to even) as int8, for every bf16 x and scales of the form
+    127 / max(a, eps) with |x| <= a, as the quantiser forms them."""
+    src = _src("k_quant.cu")
+    magic = np.float32(float(re.search(r"__fmul_rn\(x, s\), ([0-9.]+)f\)", src).group(1)))
+    assert magic == np.float32(1.5 * 2 ** 23)
+    bits = np.arange(0, 1 << 16, dtype=np.uint32)
+    x = (bits << 16).view(np.float32)
+    x = x[np.isfinite(x)]
+    rng = np.random.default_rng(12)
+    amax = np.concatenate([np.abs(x[rng.integers(0, x.size, 48)]), np.float32([1.0, 3.0e38, 1.0e-38])])
+    for a in amax:
+        s = np.float32(127.0) / np.maximum(np.float32(a), np.float32(1e-5))  # s = 127 / max(a, eps)
+        xs = x[np.abs(x) <= a]
+        prod = xs * s
+        got = ((prod + magic).view(np.uint32) & 0xFF).astype(np.int64)
+        got = np.where(got >= 128, got - 256, got)
+        want = np.clip(np.rint(prod.astype(np.float64)), -128, 127).astype(np.int64)
+        assert np.array_equal(got, want), a
+
+
+def test_bf16_magnitude_order_is_bit_order():
+    """The quantiser takes max |x| as an unsigned max of the bf16 bit patterns with the
+    sign cleared: for finite values that order is the order of the magnitudes."""
+    bits = np.arange(0, 0x7F80, dtype=np.uint32)  # +0 .. the largest finite bf16
+    mags = (bits << 16).view(np.float32)
+    assert np.all(np.diff(mags.astype(np.float64)) > 0)
+    src = _src("k_quant.cu")
+    assert src.count("__vmaxu2(m, v.x & 0x7FFF7FFFu)") == 1
