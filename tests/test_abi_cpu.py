@@ -47,6 +47,21 @@ def test_library_exports_every_declared_symbol(L):
     assert {n for n in exported if n.startswith("bitlinear_")} == set(declared_functions())
 
 
+def test_binding_covers_every_declared_function(L):
+    """The Python binding gives every entry point of the header a ctypes prototype and
+    calls it from a wrapper (the path and layout variants through the keyword arguments
+    of the plain wrapper; the workspace-free weight quantiser through the library handle
+    in its own test)."""
+    import inspect
+    from ternary_weight_bit_absmean_b200 import binding
+    declared = set(declared_functions())
+    assert set(binding.EXPORTED) | {"bitlinear_quantize_weights_noalloc"} == declared
+    src = inspect.getsource(binding)
+    for name in binding.EXPORTED:
+        assert "L.%s.argtypes" % name in src and "L.%s.restype" % name in src, name
+        assert "lib().%s(" % name in src, name
+
+
 def test_library_has_no_driver_or_torch_dependency():
     from ternary_weight_bit_absmean_b200 import binding
     out = subprocess.run(["ldd", binding.LIB_PATH], capture_output=True, text=True).stdout
