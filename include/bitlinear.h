@@ -224,9 +224,13 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
  *     keeps it until the process exits.  Every shape accepted by
  *     bitlinear_quantize_weights fits; a shape that would need more partial sums
  *     than the array holds returns BL_ERR_WORKSPACE.
- *   - The first call on each device looks up the array's device address (with that
- *     device current) and caches it.  Make that first call before any stream capture.
- *   - Nothing is allocated or freed, by this library or by any library it calls.
+ *   - Every call looks up the array's device address with the caller's device current
+ *     (cudaGetSymbolAddress).  On the first call on a device that lookup may make the
+ *     CUDA driver load this library's device code (lazy module loading), which places
+ *     the array, with the kernels, in device memory.  Make that first call before any
+ *     stream capture.
+ *   - The call itself allocates and frees nothing (no cudaMalloc, no cudaFree, no
+ *     allocating library routine).
  *   - All calls share the one array.  Calls that run at the same time on the GPU
  *     (for example on two streams) race and corrupt each other's gamma.  Serialise
  *     them.  A call never reads what an earlier call left in the array.

@@ -4,6 +4,7 @@
 // stream.
 #include <cmath>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "bitlinear.h"
@@ -37,6 +38,33 @@ bl_status check_weight_shape(int64_t N, int64_t K) {
 
 namespace bl {
 void record_cuda_error(int code) { g_last_cuda_error = code; }
+
+unsigned long long current_context_id() {
+    // the driver functions come through the runtime's entry-point query, so the library
+    // does not link the driver library; looked up once (thread-safe static init)
+    struct CtxFns {
+        CUresult (*get_current)(CUcontext*) = nullptr;
+        CUresult (*get_id)(CUcontext, unsigned long long*) = nullptr;
+        CtxFns() {
+            void* p = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+                    cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                get_current = reinterpret_cast<CUresult (*)(CUcontext*)>(p);
+            if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                get_id = reinterpret_cast<CUresult (*)(CUcontext, unsigned long long*)>(p);
+        }
+    };
+    static const CtxFns fns;
+    if (fns.get_current == nullptr || fns.get_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (fns.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (fns.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 }  // namespace bl
 
 extern "C" {

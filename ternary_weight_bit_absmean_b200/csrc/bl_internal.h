@@ -9,6 +9,8 @@
 namespace bl {
 
 // Weight quantisation (absmean partial sums, ternarise + pack, pack of int8 codes).
+// The absmean kernel never uses more than kAbsMaxParts blocks (fp64 partial sums).
+constexpr int kAbsMaxParts = 148 * 8;
 int absmean_num_partials(int64_t numel);
 cudaError_t launch_absmean_partials(const float* W, int64_t numel, double* partials, int nparts,
                                     cudaStream_t stream);
@@ -83,6 +85,34 @@ cudaError_t launch_ste_grad_weight(const float* dY, const int8_t* xq, const floa
 
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);
+
+// Identifier of the calling thread's current CUDA context, unique for the life of the
+// process (a context created after cudaDeviceReset gets a new one); 0 if unknown.
+unsigned long long current_context_id();
+
+// Remembers, for up to kCtxSlots contexts, that a one-time set-up (a kernel attribute)
+// was done in that context, so it is redone in a context that replaced a reset one.
+struct PerContextOnce {
+    static constexpr int kCtxSlots = 64;
+    unsigned long long done[kCtxSlots] = {};
+    // Runs set() unless it already succeeded in the current context.
+    template <typename F>
+    cudaError_t run(F set) {
+        const unsigned long long id = current_context_id();
+        if (id != 0)
+            for (int i = 0; i < kCtxSlots; ++i)
+                if (__atomic_load_n(&done[i], __ATOMIC_ACQUIRE) == id) return cudaSuccess;
+        const cudaError_t e = set();
+        if (e != cudaSuccess || id == 0) return e;
+        for (int i = 0; i < kCtxSlots; ++i) {
+            unsigned long long expect = 0;
+            if (__atomic_compare_exchange_n(&done[i], &expect, id, false, __ATOMIC_ACQ_REL, __ATOMIC_ACQUIRE) ||
+                expect == id)
+                return cudaSuccess;
+        }
+        return cudaSuccess;  // every slot taken: set() simply runs again next time
+    }
+};
 
 // Launch `kernel` on `stream` with programmatic stream serialisation allowed (the kernel
 // calls pdl_wait_then_release() before touching global memory) and, when cluster.x > 0,

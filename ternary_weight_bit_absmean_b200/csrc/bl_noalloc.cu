@@ -12,12 +12,13 @@
 //
 // The array is a file-scope __device__ variable: every GPU that loads this library
 // holds kNoAllocMaxPartials doubles (9472 bytes) of it until the process exits.  Host
-// code cannot use the array's name as a device address, so the first call on each
-// device looks the address up with cudaGetSymbolAddress (with that device current) and
-// caches it.
+// code cannot use the array's name as a device address, so every call looks the
+// address up with cudaGetSymbolAddress, with the caller's device current.  The lookup
+// allocates nothing; it is repeated on every call (it costs little once the module is
+// loaded) so that an address from a context that was since destroyed (after
+// cudaDeviceReset) is never used.
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 #include <cuda_runtime.h>
 
 #include "bitlinear.h"
@@ -25,28 +26,20 @@
 
 namespace {
 
-constexpr int kNoAllocMaxPartials = 148 * 8;  // the most partials the absmean kernel ever uses
-constexpr int kMaxDevices = 64;
+constexpr int kNoAllocMaxPartials = 148 * 8;
+// every partial count the absmean kernel can use fits in the array
+static_assert(kNoAllocMaxPartials >= bl::kAbsMaxParts, "the no-allocation array must hold every partial sum");
 
 static __device__ __align__(256) double g_absmean_partials[kNoAllocMaxPartials];
 
-std::mutex g_setup_mutex;
-void* g_partials_addr[kMaxDevices] = {};
-
-// Device address of g_absmean_partials on the current device (looked up once per device).
+// Device address of g_absmean_partials in the current context.  The first lookup on a
+// device may make the driver load this library's device code (lazy module loading),
+// which is where the array itself is placed in device memory.
 cudaError_t partials_address(double** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_absmean_partials);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (g_partials_addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_absmean_partials);
-        if (e != cudaSuccess) return e;
-        g_partials_addr[dev] = p;
-    }
-    *out = static_cast<double*>(g_partials_addr[dev]);
+    *out = static_cast<double*>(p);
     return cudaSuccess;
 }
 

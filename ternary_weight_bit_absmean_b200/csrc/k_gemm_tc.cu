@@ -394,15 +394,12 @@ cudaError_t launch_bt(const int8_t* xq, const uint8_t* packed, TcArgs a, int sms
         !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N), kBK / 4, kBN,
                            false))
         return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
-    }
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(gemm_tc_kernel<BT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     const int grid = a.num_tiles < sms ? a.num_tiles : sms;
     return launch_pdl(gemm_tc_kernel<BT, LAY>, dim3(grid), dim3(kThreads), C::kSmemBytes, stream, dim3(kNoCluster),
                       tx, tp, a);

@@ -391,15 +391,11 @@ int gemm_tc2_clusters(int64_t M, int64_t N, int sms) {
 template <int LAY>
 static cudaError_t launch_tc2_layout(const CUtensorMap& tx, const CUtensorMap& tp, const Tc2Args& a, int clusters,
                                  cudaStream_t stream) {
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBytes);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
-    }
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(gemm_tc2_kernel<LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     return launch_pdl(gemm_tc2_kernel<LAY>, dim3(static_cast<unsigned>(2 * clusters)), dim3(kThreads), kSmemBytes,
                       stream, dim3(2, 1, 1), tx, tp, a);
 }

@@ -395,15 +395,12 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
     a.xs_bytes = win * MP;
     const size_t smem = static_cast<size_t>(a.xs_bytes) +
                         (S > 1 ? static_cast<size_t>(MP) * kGvRows * sizeof(int) : 0);
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kWindow * MP + MP * kGvRows * static_cast<int>(sizeof(int)));
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
-    }
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(gemv_kernel<MT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kWindow * MP + MP * kGvRows * static_cast<int>(sizeof(int)));
+    });
+    if (e != cudaSuccess) return e;
     return launch_pdl(gemv_kernel<MT, LAY>,
                       dim3(static_cast<unsigned>(row_blocks), static_cast<unsigned>(S), static_cast<unsigned>(token_blocks)),
                       dim3(kGvThreads), smem, stream, S > 1 ? dim3(1, S, 1) : dim3(kNoCluster), a);

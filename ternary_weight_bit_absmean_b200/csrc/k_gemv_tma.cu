@@ -429,8 +429,6 @@ bool gemv_tma_applicable(int64_t M, int64_t N, int64_t K) {
 cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                             int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
                             cudaStream_t stream) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     GtPlan p;
     if (!plan_gemv_tma(M, N, K, sm_count(), &p)) return cudaErrorInvalidValue;
     const int MT = M <= 8 ? 1 : 2;
@@ -440,16 +438,14 @@ cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* pac
     const int64_t ntiles = (N + 15) / 16;
     GtArgs a{xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(ntiles),
              p.stages, p.tile_slots, p.units, p.wpp, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
-    static bool attr_done[2][64] = {};
-    const int mi = MT - 1;
-    if (dev < 0 || dev >= 64 || !attr_done[mi][dev]) {
-        cudaError_t e = MT == 1 ? cudaFuncSetAttribute(gemv_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       kSmemLimit)
-                                : cudaFuncSetAttribute(gemv_tma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       kSmemLimit);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[mi][dev] = true;
-    }
+    static PerContextOnce attr[2];
+    cudaError_t e = attr[MT - 1].run([MT] {
+        return MT == 1 ? cudaFuncSetAttribute(gemv_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kSmemLimit)
+                       : cudaFuncSetAttribute(gemv_tma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kSmemLimit);
+    });
+    if (e != cudaSuccess) return e;
     if (MT == 1) return launch_pdl(gemv_tma_kernel<1>, dim3(p.grid), dim3(kThreads), p.smem, stream, dim3(kNoCluster), tw, a);
     return launch_pdl(gemv_tma_kernel<2>, dim3(p.grid), dim3(kThreads), p.smem, stream, dim3(kNoCluster), tw, a);
 }

@@ -23,7 +23,6 @@ namespace bl {
 namespace {
 
 constexpr int kAbsThreads = 256;
-constexpr int kAbsMaxParts = 148 * 8;
 
 // 2-bit code of round-half-even(t) clipped to [-1, 1]: 01 for +1, 10 for -1, 00 for 0.
 __device__ __forceinline__ uint32_t code_of_ratio(float t) {

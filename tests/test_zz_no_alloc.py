@@ -7,8 +7,11 @@ library instead of a caller workspace.
 The test calls the new entry point through the C ABI and compares gamma and the packed
 codes with those of bitlinear_quantize_weights (the workspace entry point) on the same
 weights, for two calls in a row: a large matrix and then a small one, so the second
-call runs with the first call's partial sums still in the shared array.  It lives in a
-file of its own, collected last, and passes alone in a fresh process too.
+call runs with the first call's partial sums still in the shared array.  Both entry
+points run the same two kernels with the same number of partial sums, summed in the
+same fixed order, so gamma must be bit-identical.  Around the second call, device memory
+in use (the driver's free-memory count and PyTorch's allocator) must not change.  It
+lives in a file of its own, collected last, and passes alone in a fresh process too.
 """
 import ctypes
 
@@ -46,10 +49,18 @@ def test_noalloc_matches_workspace_entry_point_two_calls_in_a_row():
         g_ref, p_ref = B.quantize_weights(W, EPS)
         gamma = torch.full((1,), -1.0, dtype=torch.float32, device=dev)
         packed = torch.full((N, K // 4), 0xFF, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        free_before, _ = torch.cuda.mem_get_info()
+        torch_before = torch.cuda.memory_allocated()
         status = f(W.data_ptr(), N, K, EPS, gamma.data_ptr(), packed.data_ptr(), stream)
         assert status == 0, B.lib().bitlinear_status_string(status)
         torch.cuda.synchronize()
-        assert abs(gamma.item() - g_ref.item()) <= 1e-6 * g_ref.item()
+        if i == 1:
+            # the module (and its array) is loaded by now: this call must allocate nothing
+            free_after, _ = torch.cuda.mem_get_info()
+            assert free_after == free_before, (free_before, free_after)
+            assert torch.cuda.memory_allocated() == torch_before
+        assert torch.equal(gamma, g_ref), (gamma.item(), g_ref.item())
         assert torch.equal(packed, p_ref)
 
 
