@@ -51,6 +51,9 @@ MUTANTS = [
     ("norm_eps_dropped", "const float r32 = (float)(1.0 / sqrt(v + (double)norm_eps));",
      "const float r32 = (float)(1.0 / sqrt(v));"),
     ("norm_round_away", "float q = rintf(xn[k] * s);", "float q = roundf(xn[k] * s);"),
+    ("norm_elementwise_fp64", "const float t32 = d32 * r32;\n            xn[k] = t32 * wk;",
+     "(void)d32;\n            xn[k] = (float)(((double)bf16_bits_to_float(X[m * K + k]) - mu) * "
+     "(1.0 / sqrt(v + (double)norm_eps)) * (double)wk);"),
     ("norm_qb_128", "const float s = 127.0f / fmaxf(a, eps);", "const float s = 128.0f / fmaxf(a, eps);"),
     ("row_gamma_by_token", "(double)gamma_rows[n] / (double)s[m]", "(double)gamma_rows[m] / (double)s[m]"),
     ("row_gamma_dropped", "(double)acc[m * N + n] * (double)gamma_rows[n] / (double)s[m]",
