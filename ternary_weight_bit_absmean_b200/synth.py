@@ -88,3 +88,13 @@ WORKLOADS = {
 
 SWEEP_KN = [1024, 2048, 4096, 8192, 16384]
 SWEEP_M = [1, 4, 16, 64, 256, 1024, 8192]
+# Sweep weight mixtures, named by the share of zero codes they give: the fraction of
+# entries drawn from N(0, 1e-3 sigma) (`small_frac` of weight()).  A plain Gaussian gives
+# about 31% zeros; 0.378 and 0.664 were solved for 50% and 70%.
+SWEEP_SMALL_FRAC = {30: 0.0, 50: 0.378, 70: 0.664}
+# Sweep activations: outlier-channel fractions and their scale.
+SWEEP_OUTLIER_FRACS = [0.001, 0.005, 0.01, 0.02]
+SWEEP_OUTLIER_SCALE = 50.0
+# The grid's default point: 50% zero codes, 1% outlier channels.
+SWEEP_DEFAULT_ZEROS = 50
+SWEEP_DEFAULT_OUTLIERS = 0.01
