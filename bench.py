@@ -1,9 +1,9 @@
 """Benchmark of the BitLinear forward hot path on B200.
 
 One step = one pass of every stage of the hot path over the seven BitLinear projections
-of one LLaMA-700M-shaped layer (hidden 1536, FFN 4096: q/k/v/o 1536x1536, up/gate
-1536->4096, down 4096->1536), fp32 N(0, 0.02) weights, bf16 heavy-tailed activations
-(1% of channels x20), at M = 1, 8, 512 and 4096 tokens:
+of one LLaMA-3B-shaped layer (hidden 3200, FFN 8640: q/k/v/o 3200x3200, up/gate
+3200->8640, down 8640->3200), fp32 N(0, 0.02) weights, bf16 heavy-tailed activations
+(1% of channels x20), at M = 1, 16, 2048 and 8192 tokens:
   a1+a2  absmean ternarisation + 2-bit packing of the 7 weight matrices,
   a3     packing of 7 int8 code matrices of the same shapes,
   a4     per-token int8 quantisation of each projection's input at every M,
@@ -11,19 +11,29 @@ of one LLaMA-700M-shaped layer (hidden 1536, FFN 4096: q/k/v/o 1536x1536, up/gat
          fused gamma / s epilogue, bf16 output.
 `value` is the forward work of the step (2 M N K ops summed over projections and M)
 divided by the device time of the whole step, in TOPS, summed over ranks (each rank
-runs its own step: weak scaling, no collective on the data path).
+runs its own step: weak scaling, no collective on the data path).  `forward_only` is
+the same work over the time of the per-batch part of the step alone (a4 + forward,
+weights prepared once), the inference-time throughput.
 
-Timing: the step is captured once as a CUDA graph.  Each timed replay is bracketed by
-device events; between replays, outside the events, L2 is flushed (256 MiB written and
-another 256 MiB read, so no dirty line is left behind); K replays are bracketed by a
-barrier and a device synchronisation and the time is the maximum over ranks.  A second
-copy of the graph with a timing event around every library call gives the per-call
-breakdown and the roofline of the dominant kernel from the same number of replays.
-`e2e` repeats the step with its inputs copied from pinned host memory and its outputs
-copied back inside the timed region.
+In the same run, the decode regime is measured on the seven projections of one
+LLaMA-70B-shaped layer (q/o 8192x8192, k/v 1024x8192, up/gate 8192->28672, down
+28672->8192; 214 MB of packed weights) at M = 1 ... 64 tokens: for every M the layer's
+act quantisation + forward calls, and its forwards alone, as one CUDA graph each; the
+result is weight GB/s (packed bytes / time) against the HBM copy peak (`decode_70b`,
+`roofline_decode`).
 
---impl reference runs the CPU oracle (plain C, one core) on a bounded sample of the
-same workload and reports the same metric.
+Timing: every measured sequence is captured once as a CUDA graph.  Each timed replay is
+bracketed by device events on the launching stream; between replays, outside the events,
+L2 is flushed (256 MiB written and another 256 MiB read, so no dirty line is left
+behind).  K step replays are bracketed by a barrier and a device synchronisation and the
+time is the maximum over ranks.  A second copy of the step graph with a timing event
+around every library call gives the per-call breakdown and the roofline of the dominant
+kernel from the same number of replays.  `e2e` repeats the step with its inputs copied
+from pinned host memory and its outputs copied back inside the timed region.
+
+--workload llama700m runs the same step on the LLaMA-700M-shaped set (M = 1, 8, 512,
+4096) instead.  --impl reference runs the CPU oracle (plain C, one core) on a bounded
+sample of the same workload and reports the same metric.
 """
 import argparse
 import json
@@ -39,7 +49,11 @@ sys.path.insert(0, ROOT)
 
 EPS = 1e-5
 METRIC = "BitLinear fwd TOPS & weight GB/s at M=1..8192 vs B200 roofline"
-WORKLOAD = "llama700m"
+DECODE_WORKLOAD = "llama70b"
+WORKLOAD_TEXT = {
+    "llama3b": "llama3b BitLinear set: q/k/v/o 3200x3200, up/gate 3200->8640, down 8640->3200",
+    "llama700m": "llama700m BitLinear set: q/k/v/o 1536x1536, up/gate 1536->4096, down 4096->1536",
+}
 
 
 def parse():
@@ -48,19 +62,24 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["llama3b", "llama700m"], default="llama3b",
+                   help="the layer set of the timed step")
+    p.add_argument("--no-decode-set", action="store_true",
+                   help="skip the LLaMA-70B decode measurement")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--ref-tokens", type=int, default=4,
+    p.add_argument("--ref-tokens", type=int, default=1,
                    help="token rows per M in one reference-arm (oracle) step")
     p.add_argument("--weight-format", choices=["2bit", "tl5"], default="2bit",
                    help="--sweep: the 2-bit forward, or the five-codes-per-byte decode forward (M <= 16 shapes)")
     p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack",
-                                        "forward_tl5", "repack_tl5", "ste_input", "ste_weight"],
-                   help="time one entry point on one shape instead of the step (kernel study, ncu)")
+                                        "forward_tl5", "repack_tl5", "ste_input", "ste_weight", "copy"],
+                   help="time one entry point on one shape instead of the step (kernel study, ncu); "
+                        "'copy' times a device-to-device copy of the packed weights' size as a reference")
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
     p.add_argument("--K", type=int, default=4096)
-    p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2"], default="auto")
+    p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2", "skinny"], default="auto")
     p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--step-streams", choices=["branches", "serial"], default="branches",
@@ -82,9 +101,9 @@ def peaks():
             "source": "fallback"}
 
 
-def workload():
+def workload(name):
     from ternary_weight_bit_absmean_b200 import synth
-    spec = synth.WORKLOADS[WORKLOAD]
+    spec = synth.WORKLOADS[name]
     return spec["proj"], spec["M"], spec["outlier_frac"]
 
 
@@ -189,6 +208,119 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ ours --
 
+def capture(torch, stream, fns, branches=None):
+    """A CUDA graph of the calls `fns` on `stream`; with `branches` (a list of index lists
+    and one side stream per list) each list runs on its own stream, forked from and joined
+    back to `stream`, in order within the list."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        if branches is None:
+            for fn in fns:
+                fn()
+        else:
+            groups, side = branches
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            joins = []
+            for idx, st in zip(groups, side):
+                st.wait_event(fork)
+                with torch.cuda.stream(st):
+                    for i in idx:
+                        fns[i]()
+                    j = torch.cuda.Event()
+                    j.record(st)
+                joins.append(j)
+            for j in joins:
+                stream.wait_event(j)
+    return g
+
+
+def timed_replays(torch, stream, graph, flusher, n):
+    """Milliseconds of each of n replays of `graph`: device events on `stream` around each
+    replay, L2 flushed before each one outside the events."""
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for _ in range(n):
+        with torch.cuda.stream(stream):
+            flusher.flush()
+            e_a.record()
+            graph.replay()
+            e_b.record()
+        torch.cuda.synchronize()
+        out.append(e_a.elapsed_time(e_b))
+    return out
+
+
+def traffic_of(key):
+    """DRAM bytes per launch recorded under profiles/traffic.json for `key`, while the
+    kernel sources still hash to the digest recorded with the counters; else None."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tpath):
+        return None
+    try:
+        tj = json.load(open(tpath))
+        from ternary_weight_bit_absmean_b200 import build_lib as _bl
+        entry = tj.get(key)
+        if not isinstance(entry, dict):
+            return None
+        if entry.get("source_digest") != _bl.source_digest(entry.get("digest_files")):
+            return None
+        return entry.get("bytes_per_launch")
+    except (ValueError, KeyError, AttributeError, TypeError):
+        return None
+
+
+def decode_set(args, torch, B, synth, dev, stream, flusher, rank):
+    """The LLaMA-70B-shaped layer's seven projections at M = 1 ... 64: packed weights made
+    once from seeded codes (gamma 0.02: the scale does not change the work), then per M
+    the layer's act quantisation + forward calls and its forwards alone, each a CUDA graph
+    replayed with L2 flushed before each replay."""
+    projs, Ms, ofrac = workload(DECODE_WORKLOAD)
+    lay = xq_layout_of(B, args.xq_layout)
+    pk = []
+    for pi, (_, N, K) in enumerate(projs):
+        c = synth.codes(N, K, seed=pi).to(dev)
+        p = torch.empty(N, K // 4, dtype=torch.uint8, device=dev)
+        B.bitlinear_pack(c, p)
+        del c
+        pk.append(p)
+    gam = [torch.full((1,), 0.02, dtype=torch.float32, device=dev) for _ in projs]
+    wbytes = sum(p.numel() for p in pk)
+    out = {}
+    for M in Ms:
+        X = [synth.activations(M, K, seed=rank_seed(pi, M, rank), outlier_frac=ofrac).to(dev)
+             for pi, (_, N, K) in enumerate(projs)]
+        xq = [torch.empty(M, K, dtype=torch.int8, device=dev) for (_, N, K) in projs]
+        sc = [torch.empty(M, dtype=torch.float32, device=dev) for _ in projs]
+        Y = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for (_, N, K) in projs]
+        q_calls = [lambda i=i: B.bitlinear_quantize_act(X[i], EPS, xq[i], sc[i], layout=lay) for i in range(len(projs))]
+        f_calls = [lambda i=i: B.bitlinear_forward(xq[i], sc[i], pk[i], gam[i], Y[i], layout=lay)
+                   for i in range(len(projs))]
+        with torch.cuda.stream(stream):
+            for fn in q_calls + f_calls:
+                fn()
+        torch.cuda.synchronize()
+        g_layer = capture(torch, stream, [f for pair in zip(q_calls, f_calls) for f in pair])
+        g_fwd = capture(torch, stream, f_calls)
+        for _ in range(max(3, args.warmup)):
+            timed_replays(torch, stream, g_layer, flusher, 1)
+            timed_replays(torch, stream, g_fwd, flusher, 1)
+        t_layer = statistics.median(timed_replays(torch, stream, g_layer, flusher, args.steps))
+        t_fwd = statistics.median(timed_replays(torch, stream, g_fwd, flusher, args.steps))
+        alg = wbytes + sum(M * K + 4 * M + 2 * M * N for (_, N, K) in projs)  # forward's algorithmic bytes
+        out[str(M)] = {"layer_us": round(t_layer * 1e3, 2), "fwd_us": round(t_fwd * 1e3, 2),
+                       "weight_gbs": round(wbytes / (t_fwd * 1e-3) / 1e9, 1),
+                       "fwd_bytes": alg, "fwd_gbs": round(alg / (t_fwd * 1e-3) / 1e9, 1),
+                       "layer_weight_gbs": round(wbytes / (t_layer * 1e-3) / 1e9, 1),
+                       "tops": round(sum(2 * M * N * K for (_, N, K) in projs) / (t_fwd * 1e-3) / 1e12, 2)}
+        g_layer.reset()
+        g_fwd.reset()
+        del X, xq, sc, Y
+    return {"workload": "llama70b layer: q/o 8192x8192, k/v 1024x8192 (GQA 8 kv heads x 128), up/gate "
+                        "8192->28672, down 28672->8192; %.1f MB of packed weights" % (wbytes / 1e6),
+            "M": Ms, "weight_bytes": wbytes, "by_M": out}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -212,7 +344,7 @@ def run_ours(args):
         dist.barrier()
     B.lib()
 
-    projs, Ms, ofrac = workload()
+    projs, Ms, ofrac = workload(args.workload)
     XQ_LAYOUT = xq_layout_of(B, args.xq_layout)
     # inputs: weights are the same model replica on every rank; tokens differ per rank
     W = [synth.weight(N, K, seed=pi).to(dev) for pi, (_, N, K) in enumerate(projs)]
@@ -242,11 +374,13 @@ def run_ours(args):
                 xq[pi, M], sc[pi, M], pk[pi], gam[pi], Y[pi, M], layout=XQ_LAYOUT)))
     launches_per_call = {"a1a2": 2, "a3": 1, "a4": 1, "fwd": 1}
     launches_per_step = sum(launches_per_call[lab[0]] for lab, _ in calls)
+    fns = [fn for _, fn in calls]
+    per_batch = [i for i, (lab, _) in enumerate(calls) if lab[0] in ("a4", "fwd")]
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for _ in range(2):  # eager warm-up: first-call set-up (attributes, entry points)
-            for _, fn in calls:
+            for fn in fns:
                 fn()
     torch.cuda.synchronize()
 
@@ -255,46 +389,23 @@ def run_ours(args):
     # that order) is captured on its own stream: seven concurrent graph branches, forked
     # from and joined back to the capture stream.  A second, single-stream copy of the
     # step carries a timing event around every call (per-call breakdown and roofline).
+    # A third graph holds the per-batch calls only (act quant + forward at every M).
     side = [torch.cuda.Stream(device=dev) for _ in projs]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        if args.step_streams == "serial":
-            for _, fn in calls:
-                fn()
-        else:
-            fork = torch.cuda.Event()
-            fork.record(stream)
-            joins = []
-            for pi in range(len(projs)):
-                side[pi].wait_event(fork)
-                with torch.cuda.stream(side[pi]):
-                    for lab, fn in calls:
-                        if lab[1] == pi:
-                            fn()
-                    j = torch.cuda.Event()
-                    j.record(side[pi])
-                joins.append(j)
-            for j in joins:
-                stream.wait_event(j)
+    chains = [[i for i, (lab, _) in enumerate(calls) if lab[1] == pi] for pi in range(len(projs))]
+    branch = None if args.step_streams == "serial" else (chains, side)
+    graph = capture(torch, stream, fns, branch)
+    fwd_chains = [[i for i in ch if i in per_batch] for ch in chains]
+    graph_fwd = (capture(torch, stream, [fns[i] for i in per_batch]) if branch is None
+                 else capture(torch, stream, fns, (fwd_chains, side)))
     ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
           for _ in calls]
     graph_ev = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_ev, stream=stream):
-        for (lab, fn), (e0, e1) in zip(calls, ev):
+        for fn, (e0, e1) in zip(fns, ev):
             e0.record()
             fn()
             e1.record()
     torch.cuda.synchronize()
-    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def one_step():
-        with torch.cuda.stream(stream):
-            flusher.flush()
-            e_a.record()
-            graph.replay()
-            e_b.record()
-        torch.cuda.synchronize()
-        return e_a.elapsed_time(e_b)
 
     def one_instrumented_step():
         with torch.cuda.stream(stream):
@@ -304,7 +415,7 @@ def run_ours(args):
         return [e0.elapsed_time(e1) for e0, e1 in ev]
 
     for _ in range(max(3, args.warmup)):
-        one_step()
+        timed_replays(torch, stream, graph, flusher, 1)
         one_instrumented_step()
 
     clocks = ClockSampler(local)
@@ -313,17 +424,24 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [one_step() for _ in range(args.steps)]
+    step_ms = timed_replays(torch, stream, graph, flusher, args.steps)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
     total_ms = max_over_ranks(sum(step_ms), dev)
+    # the per-batch part alone (weights prepared), the same number of replays
+    for _ in range(max(3, args.warmup)):
+        timed_replays(torch, stream, graph_fwd, flusher, 1)
+    fwd_total_ms = max_over_ranks(sum(timed_replays(torch, stream, graph_fwd, flusher, args.steps)), dev)
     # per-call device times from the same number of instrumented replays of the step
     call_ms = [0.0] * len(calls)
     for _ in range(args.steps):
         call_ms = [a + b for a, b in zip(call_ms, one_instrumented_step())]
     call_ms = [c / args.steps for c in call_ms]
+    dec = None
+    if not args.no_decode_set:
+        dec = decode_set(args, torch, B, synth, dev, stream, flusher, rank)
+    clk = clocks.stop()
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> pinned host
     h_W = [w.cpu().pin_memory() for w in W]
@@ -332,6 +450,7 @@ def run_ours(args):
     h_Y = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in Y.items()}
     h2d = sum(t.numel() * t.element_size() for t in h_W + h_C + list(h_X.values()))
     d2h = sum(t.numel() * t.element_size() for t in h_Y.values())
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_ms = []
     for i in range(args.e2e_steps + 1):
         with torch.cuda.stream(stream):
@@ -354,6 +473,7 @@ def run_ours(args):
 
     ops_step = fwd_ops(projs, Ms)
     value = whole_job_tops(ops_step, args.steps, world, total_ms)
+    fwd_value = whole_job_tops(ops_step, args.steps, world, fwd_total_ms)
     e2e_value = whole_job_tops(ops_step, len(e2e_ms), world, e2e_total) if e2e_ms else None
 
     # ---- per-row breakdown and the dominant kernel's roofline
@@ -376,20 +496,10 @@ def run_ours(args):
     dom_ms = by["fwd_M%d" % Mbig] / len(projs)
     dom_ops = sum(2 * Mbig * N * K for (_, N, K) in projs) / len(projs)
     achieved = dom_ops / (dom_ms * 1e-3) / 1e12
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            tj = json.load(open(tpath))
-            from ternary_weight_bit_absmean_b200 import build_lib as _bl
-            files = tj.get("digest_files")
-            if files and tj.get("source_digest") == _bl.source_digest(files):
-                traffic = tj.get("gemm_tc_M%d_bytes_per_launch" % Mbig)
-        except (ValueError, KeyError, AttributeError):
-            traffic = None
-    roofline = {"kernel": "gemm_tc (tcgen05 kind::i8), M=%d, mean over the 7 projections" % Mbig,
+    roofline = {"kernel": "gemm_tc / gemm_tc2 (tcgen05 kind::i8), M=%d, mean over the 7 projections" % Mbig,
                 "bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
-                "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4), "traffic": traffic,
+                "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
+                "traffic": traffic_of("%s_prefill_M%d" % (args.workload, Mbig)),
                 "peak_note": "int8 dense = 2 x %s bf16 %.0f TFLOP/s (burst)" % (P["source"], P["bf16_tflops"])}
     step_mean = total_ms / args.steps
     result = {
@@ -397,10 +507,12 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_mean, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
         "data": "synthetic (seeded N(0,0.02) fp32 weights, bf16 N(0,1) activations with 1% x20 outlier channels)",
-        "config": {"workload": "llama700m BitLinear set: q/k/v/o 1536x1536, up/gate 1536->4096, down 4096->1536",
+        "config": {"workload": WORKLOAD_TEXT[args.workload],
                    "M": Ms, "out_dtype": "bf16", "eps": EPS, "xq_layout": args.xq_layout,
-                   "stages": "a1+a2 quantize_weights x7, a3 pack x7, a4 quantize_act x28, a5/a6 forward x28",
-                   "l2": "flushed between steps outside the timed events (256 MiB written, then another 256 MiB read so no dirty line is left)",
+                   "stages": "a1+a2 quantize_weights x7, a3 pack x7, a4 quantize_act x%d, a5/a6 forward x%d"
+                             % (len(projs) * len(Ms), len(projs) * len(Ms)),
+                   "decode_set": None if dec is None else dec["workload"] + ", M=1..64, forward only and with act quant",
+                   "l2": "flushed between replays outside the timed events (256 MiB written, then another 256 MiB read so no dirty line is left)",
                    "timing": "CUDA graph replay of the step bracketed by device events, summed over steps, max over ranks; per-call breakdown and roofline from the same number of replays of an instrumented single-stream copy of the graph",
                    "step_streams": ("the 7 projections as concurrent graph branches (each projection's calls in order)"
                                     if args.step_streams == "branches" else "one stream, calls in order"),
@@ -409,14 +521,29 @@ def run_ours(args):
         "e2e": {"value": round(e2e_value, 4) if e2e_value is not None else None, "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": roofline,
+        "forward_only": {"value": round(fwd_value, 3), "unit": "TOPS",
+                         "ms_per_step": round(fwd_total_ms / args.steps, 4),
+                         "what": "act quantisation + forward at every M (weights prepared once), same graph "
+                                 "structure, same number of replays"},
         "breakdown_us_per_step": {k: round(v * 1e3, 2) for k, v in sorted(by.items())},
         "forward_by_M": fwd,
         "hbm_peak_gbs": P["hbm_gbs"],
         "clocks": clk,
     }
+    if dec is not None:
+        m1 = dec["by_M"]["1"]
+        result["decode_70b"] = dec["by_M"]
+        result["roofline_decode"] = {
+            "kernel": "decode forward (gemv_tma / gemv), the 70B layer's 7 projections at M=1 as one graph",
+            "bound": "hbm", "achieved": m1["fwd_gbs"], "peak": P["hbm_gbs"], "unit": "GB/s",
+            "frac": round(m1["fwd_gbs"] / P["hbm_gbs"], 4), "weight_gbs": m1["weight_gbs"],
+            "weight_frac": round(m1["weight_gbs"] / P["hbm_gbs"], 4),
+            "traffic": traffic_of("llama70b_decode_M1"),
+            "peak_note": "%s HBM copy bandwidth" % P["source"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(projs, Ms, ofrac, tokens=48)
+        result["cpu_baseline"] = cpu_baseline(projs, Ms, ofrac, tokens=4)
     graph.reset()
+    graph_fwd.reset()
     graph_ev.reset()
     if world > 1:
         dist.barrier()
@@ -427,35 +554,53 @@ def run_ours(args):
 
 # ---------------------------------------------------------- CPU oracle --
 
-def oracle_sample(projs, Ms, ofrac, tokens, seed_base=0):
-    """Run the oracle on a bounded sample of one step: the full weight quantisation of
-    every projection, plus activation quantisation and forward of min(M, tokens) token
-    rows at every M.  Returns (forward ops in the sample, seconds)."""
-    import numpy as np
+_PACKED = {}  # weights and packed codes of the oracle, per projection, reused across steps
 
+
+def oracle_sample(projs, Ms, ofrac, tokens, seed_base=0, weight_projs=None):
+    """Run the oracle on a bounded sample of one step: the weight quantisation of the
+    projections in `weight_projs` (all by default), plus activation quantisation and
+    forward of min(M, tokens) token rows at every M for every projection.  Returns
+    (forward ops in the sample, seconds)."""
     import oracle
     from ternary_weight_bit_absmean_b200 import synth
+    if weight_projs is None:
+        weight_projs = range(len(projs))
     inputs = []
     for pi, (_, N, K) in enumerate(projs):
-        Wn = synth.weight(N, K, seed=pi).numpy()
+        if (pi, N, K, "W") not in _PACKED:  # the weights depend on the projection only
+            _PACKED[pi, N, K, "W"] = synth.weight(N, K, seed=pi).numpy()
+        Wn = _PACKED[pi, N, K, "W"]
         Xs = {M: synth.bf16_bits(synth.activations(min(M, tokens), K, seed=seed_base + pi + 97 * M,
                                                    outlier_frac=ofrac)) for M in Ms}
         inputs.append((Wn, Xs, K))
     oracle.default()
+    # the packed codes of projections whose quantisation is not in the sample come from an
+    # earlier step (made once, outside the timed part)
+    for pi in range(len(projs)):
+        key = (pi,) + tuple(projs[pi][1:])
+        if pi not in weight_projs and key not in _PACKED:
+            _PACKED[key] = oracle.quantize_weights(inputs[pi][0], EPS)[:3:2]
     t0 = time.perf_counter()
     ops = 0
-    for Wn, Xs, K in inputs:
-        g, codes, packed = oracle.quantize_weights(Wn, EPS)
+    packed = {}
+    for pi, (Wn, Xs, K) in enumerate(inputs):
+        key = (pi,) + tuple(projs[pi][1:])
+        if pi in weight_projs:
+            g, codes, packed[pi] = oracle.quantize_weights(Wn, EPS)
+            _PACKED[key] = (g, packed[pi])
+        else:
+            g, packed[pi] = _PACKED[key]
         for M in Ms:
             xq, s = oracle.quantize_act(Xs[M], EPS)
-            y = oracle.forward(xq, s, packed, g, K, oracle.OUT_BF16)
-            ops += 2 * xq.shape[0] * packed.shape[0] * K
+            y = oracle.forward(xq, s, packed[pi], g, K, oracle.OUT_BF16)
+            ops += 2 * xq.shape[0] * packed[pi].shape[0] * K
             assert y.shape[0] == xq.shape[0]
-    return ops, time.perf_counter() - t0, np
+    return ops, time.perf_counter() - t0
 
 
 def cpu_baseline(projs, Ms, ofrac, tokens):
-    ops, secs, _ = oracle_sample(projs, Ms, ofrac, tokens)
+    ops, secs = oracle_sample(projs, Ms, ofrac, tokens)
     return {"value": round(ops / secs / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
             "sample": "full weight quantisation of the 7 projections + act quantisation and forward of "
                       "min(M, %d) token rows at each M (%.2f GOP forward, %.1f s)" % (tokens, ops / 1e9, secs)}
@@ -466,22 +611,25 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    projs, Ms, ofrac = workload()
+    projs, Ms, ofrac = workload(args.workload)
+    # each step: the weight quantisation of one projection (in turn) and the act
+    # quantisation + forward of ref_tokens rows at every M for every projection
     for i in range(args.warmup):
-        oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=i)
+        oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=i, weight_projs={i % len(projs)})
     total_ops, total_s = 0, 0.0
     for i in range(args.steps):
-        ops, secs, _ = oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=1000 + i)
+        ops, secs = oracle_sample(projs, Ms, ofrac, args.ref_tokens, seed_base=1000 + i,
+                                  weight_projs={i % len(projs)})
         total_ops += ops
         total_s += secs
     value = total_ops / total_s / 1e12
-    sample = ("per step: full weight quantisation of the 7 projections + act quantisation and forward "
-              "of min(M, %d) token rows at each M (CPU oracle, plain C, one core)" % args.ref_tokens)
+    sample = ("per step: weight quantisation of one of the 7 projections (in turn) + act quantisation and "
+              "forward of min(M, %d) token rows at each M for all 7 (CPU oracle, plain C, one core)" % args.ref_tokens)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_s / args.steps * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
-        "data": "synthetic", "config": {"workload": "llama700m BitLinear set (bounded oracle sample)",
+        "data": "synthetic", "config": {"workload": WORKLOAD_TEXT[args.workload] + " (bounded oracle sample)",
                                         "M": Ms, "tokens_per_M": args.ref_tokens},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
                          "sample": sample},
@@ -515,7 +663,7 @@ def run_single(args):
         odt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[args.out_dtype]
         out = torch.empty(M, N, dtype=odt, device=dev)
         path = {"auto": B.BL_PATH_AUTO, "gemv": B.BL_PATH_GEMV, "tc": B.BL_PATH_TC, "tc1": B.BL_PATH_TC_1SM,
-                "tc2": B.BL_PATH_TC_2SM}[args.path]
+                "tc2": B.BL_PATH_TC_2SM, "skinny": B.BL_PATH_SKINNY}[args.path]
         lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=lay)
         ops = 2 * M * N * K
@@ -570,6 +718,13 @@ def run_single(args):
         lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_norm_quantize_act(X, nw, B.BL_NORM_RMS, 1e-5, EPS, xq, s, layout=lay)
         ops, nbytes = 0, 3 * M * K + 4 * M + 4 * K
+    elif args.single == "copy":
+        # reference for one launch's reachable bandwidth at this size: a device-to-device
+        # copy (read + write) of as many bytes as the packed weights of an N x K matrix
+        src = torch.ones(N * K // 4, dtype=torch.uint8, device=dev)
+        dst = torch.empty_like(src)
+        fn = lambda: dst.copy_(src)
+        ops, nbytes = 0, 2 * src.numel()
     elif args.single == "quantize_weights":
         W = torch.randn(N, K, device=dev) * 0.02
         gamma = torch.empty(1, device=dev)

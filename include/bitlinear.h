@@ -78,11 +78,14 @@ typedef enum {
 } bl_dtype;
 
 typedef enum {
-    BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core path cannot tile), else tcgen05 */
+    BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core paths cannot tile), the
+                           small-batch tcgen05 kernel for 16 < M <= 64, else tiled tcgen05 */
     BL_PATH_GEMV = 1,   /* register-unpack GEMV, any M (token tiles of 16) */
     BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
     BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
-    BL_PATH_TC_2SM = 4  /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
+    BL_PATH_TC_2SM = 4, /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
+    BL_PATH_SKINNY = 5  /* the tcgen05 small-batch kernel (expanded weights in tensor memory,
+                           K split over a cluster when rows are few); K % 64 == 0 */
 } bl_path;
 
 /* Storage order of x_q within each row.
@@ -200,8 +203,9 @@ BL_API bl_status bitlinear_norm_quantize_act(const uint16_t *X, const float *nor
  *   out     out : [M, N] of out_dtype, device.
  *   err_word out: optional; BL_ERRBIT_TIMEOUT if a bounded device wait gave up (the
  *                 output is then incomplete).
- * M <= 16 runs the register-unpack GEMV; larger M runs the tcgen05 kind::i8 path when
- * K % 64 == 0 (else the GEMV).  K * 127 must stay below 2^31.
+ * M <= 16 runs the register-unpack GEMV; 16 < M <= 64 the small-batch tcgen05 kernel and
+ * larger M the tiled tcgen05 kind::i8 path, when K % 64 == 0 (else the GEMV).  K * 127
+ * must stay below 2^31.
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
 BL_API bl_status bitlinear_forward(const int8_t *xq, const float *s, const uint8_t *packed,
                             const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
@@ -316,15 +320,19 @@ BL_API bl_status bitlinear_forward_tl5(const int8_t *xq, const float *s, const u
  *   dX[m, k] = gamma * sum_n dY[m, n] c[n, k]
  *   dW[n, k] = gamma * sum_m dY[m, n] x_q[m, k] / s[m]
  * dX is the gradient for the quantiser's input (the normalised activations), dW the
- * gradient for the shadow weights.  The sums run in fp32 (each product with a code is
- * exact; dY / s[m] is one IEEE division), the result is scaled by gamma once.
+ * gradient for the shadow weights.  Both run on the tensor cores (bf16 operands, fp32
+ * accumulation): the codes and x_q are exact in bf16, and the fp32 factor (dY, or
+ * dY * (1 / s[m]) with the reciprocal rounded to fp32) is split into two bf16 parts
+ * hi + lo that together carry it to within 2^-16 relative; both parts meet the same
+ * exact operand, so every product is exact and the sums round in fp32 (in the tensor
+ * cores' order).  The result is scaled by gamma once.
  * ---------------------------------------------------------------------------------- */
 
 /*   dY     in  : fp32 [M, N], device.
  *   packed in  : uint8 [N, K/4] 2-bit codes (the forward's weights), device.
  *   gamma  in  : device fp32 scalar.
  *   dX     out : fp32 [M, K], device.
- * K % 4 == 0; M, N, K < 2^31; M <= 65535 * 64.
+ * K % 4 == 0; M, N, K < 2^31.
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
 BL_API bl_status bitlinear_ste_backward_input(const float *dY, const uint8_t *packed, const float *gamma,
                                               int64_t M, int64_t N, int64_t K, float *dX, void *stream);
@@ -333,7 +341,7 @@ BL_API bl_status bitlinear_ste_backward_input(const float *dY, const uint8_t *pa
  *   xq, s in  : the forward's int8 [M, K] row-major activations and fp32 [M] scales, device.
  *   gamma in  : device fp32 scalar.
  *   dW    out : fp32 [N, K], device.
- * M, N, K < 2^31; N <= 65535 * 64.
+ * K % 4 == 0; M, N, K < 2^31.
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
 BL_API bl_status bitlinear_ste_backward_weight(const float *dY, const int8_t *xq, const float *s,
                                                const float *gamma, int64_t M, int64_t N, int64_t K, float *dW,

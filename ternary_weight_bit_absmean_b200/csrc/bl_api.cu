@@ -76,6 +76,7 @@ size_t bitlinear_workspace_size(int64_t N, int64_t K) {
 
 bl_status bitlinear_quantize_weights(const float* W, int64_t N, int64_t K, float eps, float* gamma_out,
                                      uint8_t* packed_out, void* ws, size_t ws_bytes, void* stream) {
+    BL_RANGE("bitlinear_quantize_weights");
     if (W == nullptr || gamma_out == nullptr || packed_out == nullptr || !eps_ok(eps))
         return BL_ERR_INVALID_ARG;
     bl_status st = check_weight_shape(N, K);
@@ -96,6 +97,7 @@ bl_status bitlinear_quantize_weights(const float* W, int64_t N, int64_t K, float
 
 bl_status bitlinear_quantize_weights_with_scale(const float* W, int64_t N, int64_t K, const float* gamma,
                                                 uint8_t* packed_out, void* stream) {
+    BL_RANGE("bitlinear_quantize_weights_with_scale");
     if (W == nullptr || gamma == nullptr || packed_out == nullptr) return BL_ERR_INVALID_ARG;
     bl_status st = check_weight_shape(N, K);
     if (st != BL_OK) return st;
@@ -107,6 +109,7 @@ bl_status bitlinear_quantize_weights_with_scale(const float* W, int64_t N, int64
 
 bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, uint8_t* packed_out, int32_t* err_word,
                          void* stream) {
+    BL_RANGE("bitlinear_pack");
     if (codes == nullptr || packed_out == nullptr) return BL_ERR_INVALID_ARG;
     bl_status st = check_weight_shape(N, K);
     if (st != BL_OK) return st;
@@ -117,6 +120,7 @@ bl_status bitlinear_pack(const int8_t* codes, int64_t N, int64_t K, uint8_t* pac
 
 bl_status bitlinear_quantize_act_layout(const uint16_t* X, int64_t M, int64_t K, float eps, int8_t* xq_out,
                                         float* s_out, bl_xq_layout layout, void* stream) {
+    BL_RANGE("bitlinear_quantize_act_layout");
     if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
     if (M <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
     if (layout != BL_XQ_ROWMAJOR && layout != BL_XQ_K16_EVENODD && layout != BL_XQ_K16_STRIDE4)
@@ -131,6 +135,7 @@ bl_status bitlinear_quantize_act_layout(const uint16_t* X, int64_t M, int64_t K,
 bl_status bitlinear_norm_quantize_act(const uint16_t* X, const float* norm_weight, int64_t M, int64_t K,
                                       bl_norm_kind norm_kind, float norm_eps, float eps, int8_t* xq_out, float* s_out,
                                       bl_xq_layout layout, void* stream) {
+    BL_RANGE("bitlinear_norm_quantize_act");
     if (X == nullptr || xq_out == nullptr || s_out == nullptr || !eps_ok(eps)) return BL_ERR_INVALID_ARG;
     if (!std::isfinite(norm_eps) || norm_eps < 0.0f) return BL_ERR_INVALID_ARG;
     if (norm_kind != BL_NORM_RMS && norm_kind != BL_NORM_LAYER) return BL_ERR_INVALID_ARG;
@@ -160,7 +165,7 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32)
         return BL_ERR_INVALID_ARG;
     if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
-        path != BL_PATH_TC_2SM)
+        path != BL_PATH_TC_2SM && path != BL_PATH_SKINNY)
         return BL_ERR_INVALID_ARG;
     if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD && xq_layout != BL_XQ_K16_STRIDE4)
         return BL_ERR_INVALID_ARG;
@@ -171,12 +176,13 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(xq) || !aligned16(s) || !aligned16(packed) || !aligned16(out)) return BL_ERR_MISALIGNED;
     const bool k64 = (K % 64) == 0;
-    const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM;
+    const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM || path == BL_PATH_SKINNY;
     if (tc && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
     // the tensor-core kernels expand stride-4 codes as 64 * code: 64 * 128 * K must fit
     const bool s4_big = xq_layout == BL_XQ_K16_STRIDE4 && K > (int64_t(1) << 17);
     if (tc && s4_big) return BL_ERR_UNSUPPORTED_SHAPE;
-    if (path == BL_PATH_AUTO) path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : BL_PATH_TC;
+    if (path == BL_PATH_AUTO)
+        path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : (M <= 64 ? BL_PATH_SKINNY : BL_PATH_TC);
     if (gamma_per_row && !aligned16(gamma)) return BL_ERR_MISALIGNED;
     const int kind = static_cast<int>(out_dtype) | (gamma_per_row ? bl::kGammaPerRow : 0);
     const int lay = static_cast<int>(xq_layout);
@@ -188,6 +194,8 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
         e = bl::launch_gemm_tc1(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (path == BL_PATH_TC_2SM) {
         e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
+    } else if (path == BL_PATH_SKINNY) {
+        e = bl::launch_gemv_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (k64 && M <= int64_t(65535) * 16) {
         e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else {
@@ -211,6 +219,7 @@ static bl_status check_tl5_shape(int64_t N, int64_t K) {
 
 bl_status bitlinear_pack_tl5(const int8_t* codes, int64_t N, int64_t K, uint8_t* tl5_out, int32_t* err_word,
                              void* stream) {
+    BL_RANGE("bitlinear_pack_tl5");
     if (codes == nullptr || tl5_out == nullptr) return BL_ERR_INVALID_ARG;
     bl_status st = check_tl5_shape(N, K);
     if (st != BL_OK) return st;
@@ -219,6 +228,7 @@ bl_status bitlinear_pack_tl5(const int8_t* codes, int64_t N, int64_t K, uint8_t*
 }
 
 bl_status bitlinear_repack_tl5(const uint8_t* packed, int64_t N, int64_t K, uint8_t* tl5_out, void* stream) {
+    BL_RANGE("bitlinear_repack_tl5");
     if (packed == nullptr || tl5_out == nullptr) return BL_ERR_INVALID_ARG;
     bl_status st = check_tl5_shape(N, K);
     if (st != BL_OK) return st;
@@ -228,6 +238,7 @@ bl_status bitlinear_repack_tl5(const uint8_t* packed, int64_t N, int64_t K, uint
 
 bl_status bitlinear_forward_tl5(const int8_t* xq, const float* s, const uint8_t* tl5, const float* gamma, int64_t M,
                                 int64_t N, int64_t K, void* out, bl_dtype out_dtype, void* stream) {
+    BL_RANGE("bitlinear_forward_tl5");
     if (xq == nullptr || s == nullptr || tl5 == nullptr || gamma == nullptr || out == nullptr)
         return BL_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
@@ -243,21 +254,24 @@ bl_status bitlinear_forward_tl5(const int8_t* xq, const float* s, const uint8_t*
 
 bl_status bitlinear_ste_backward_input(const float* dY, const uint8_t* packed, const float* gamma, int64_t M,
                                        int64_t N, int64_t K, float* dX, void* stream) {
+    BL_RANGE("bitlinear_ste_backward_input");
     if (dY == nullptr || packed == nullptr || gamma == nullptr || dX == nullptr) return BL_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
     if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
     const int64_t lim = int64_t(1) << 31;
-    if (M >= lim || N >= lim || K >= lim || M > int64_t(65535) * 64) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (M >= lim || N >= lim || K >= lim) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(dY) || !aligned16(packed) || !aligned16(dX)) return BL_ERR_MISALIGNED;
     return cuda_status(bl::launch_ste_grad_input(dY, packed, gamma, M, N, K, dX, as_stream(stream)));
 }
 
 bl_status bitlinear_ste_backward_weight(const float* dY, const int8_t* xq, const float* s, const float* gamma,
                                         int64_t M, int64_t N, int64_t K, float* dW, void* stream) {
+    BL_RANGE("bitlinear_ste_backward_weight");
     if (dY == nullptr || xq == nullptr || s == nullptr || gamma == nullptr || dW == nullptr) return BL_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;
+    if (K % 4 != 0) return BL_ERR_UNSUPPORTED_SHAPE;
     const int64_t lim = int64_t(1) << 31;
-    if (M >= lim || N >= lim || K >= lim || N > int64_t(65535) * 64) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (M >= lim || N >= lim || K >= lim) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(dY) || !aligned16(xq) || !aligned16(s) || !aligned16(dW)) return BL_ERR_MISALIGNED;
     return cuda_status(bl::launch_ste_grad_weight(dY, xq, s, gamma, M, N, K, dW, as_stream(stream)));
 }
@@ -265,12 +279,14 @@ bl_status bitlinear_ste_backward_weight(const float* dY, const int8_t* xq, const
 bl_status bitlinear_forward_layout(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                                    int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
                                    int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
+    BL_RANGE("bitlinear_forward_layout");
     return forward_impl(xq, s, packed, gamma, M, N, K, out, out_dtype, err_word, xq_layout, path, false, stream);
 }
 
 bl_status bitlinear_forward_rowscale(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma_rows,
                                      int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
                                      int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
+    BL_RANGE("bitlinear_forward_rowscale");
     return forward_impl(xq, s, packed, gamma_rows, M, N, K, out, out_dtype, err_word, xq_layout, path, true, stream);
 }
 

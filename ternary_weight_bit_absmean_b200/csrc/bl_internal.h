@@ -5,8 +5,20 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 namespace bl {
+
+// A named NVTX range around an entry point, so that a profiler's timeline shows which
+// library call enqueued which kernels; without an attached tool it costs a test of one
+// function pointer.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define BL_RANGE(name) ::bl::NvtxRange bl_nvtx_range_(name)
 
 // Weight quantisation (absmean partial sums, ternarise + pack, pack of int8 codes).
 // The absmean kernel never uses more than kAbsMaxParts blocks (fp64 partial sums).
@@ -68,6 +80,11 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
 cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* packed,
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                             int kind, int32_t* err, int layout, cudaStream_t stream);
+
+// Small-batch tcgen05 kernel (expanded weights in tensor memory, K split over a cluster
+// when rows are few), K % 64 == 0, any M (token tiles of up to 128).
+cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma, int64_t M,
+                           int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout, cudaStream_t stream);
 
 // The 1.6-bit (five codes per byte) weight format, K % 16 == 0 (k_tl5.cu).
 int64_t tl5_row_bytes(int64_t K);

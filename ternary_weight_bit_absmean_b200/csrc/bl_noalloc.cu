@@ -51,6 +51,7 @@ extern "C" {
 
 bl_status bitlinear_quantize_weights_noalloc(const float* W, int64_t N, int64_t K, float eps,
                                              float* gamma_out, uint8_t* packed_out, void* stream) {
+    BL_RANGE("bitlinear_quantize_weights_noalloc");
     if (W == nullptr || gamma_out == nullptr || packed_out == nullptr) return BL_ERR_INVALID_ARG;
     if (!std::isfinite(eps) || !(eps > 0.0f)) return BL_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0) return BL_ERR_INVALID_ARG;

@@ -1,0 +1,404 @@
+// k_gemv_tc.cu -- BitLinear forward for small and middling token counts (decode and small
+// batches, up to 128 tokens) on the tcgen05 tensor cores, with the expanded weights kept
+// in tensor memory.
+//
+// What is computed ("What 1.58 Bits Actually Changes", "How the low-bit linear path
+// works": +1 adds, -1 subtracts, 0 skips; "1-bit & Ternary LLMs", block "BitNet (Oct
+// 2023)": one float rescale at the end):
+//   acc[m, n] = sum_k x_q[m, k] * c[n, k],   y[m, n] = acc[m, n] * gamma / s[m].
+//
+// Why this shape of kernel.  With few tokens the work per weight byte is small and the
+// path is bound by streaming the packed weights from HBM; each SM has to turn about 22
+// packed bytes (88 codes) per cycle into tensor-core operands.  Expanding the codes into
+// shared memory (the prefill kernels) costs two shared-memory passes per expanded byte,
+// which caps the rate near half of that.  Here the expanded int8 codes go straight from
+// registers into tensor memory (tcgen05.st), and the MMA reads its A operand from there
+// (tcgen05.mma ... [a_tmem]), so shared memory carries only the packed weights and the
+// activation tile, each written once by TMA and read once.
+//
+// Tile: 128 weight rows (MMA M, TMEM lanes) x BT tokens (MMA N; 16 to 128) x a slice of
+// K in stages of 128 codes.  Per stage:
+//   warp 0 (one lane)   TMA: packed weights [128 rows x 32 B] and the x_q tile
+//                       [BT x 128 B] (128-byte swizzle) on one mbarrier;
+//   warps 2-9           expanders, two per TMEM lane quarter: each thread owns one weight
+//                       row and half the stage (64 codes), unpacks them in registers in
+//                       the order of the x_q layout and stores 16 columns of tensor
+//                       memory; after tcgen05.wait::st one lane per warp arrives;
+//   warp 1 (one lane)   MMA issuer: four tcgen05.mma kind::i8 (K = 32) per stage, A from
+//                       tensor memory, B (x_q) from shared memory; tcgen05.commit frees
+//                       the stage.
+// After the last stage the expander warps read the int32 accumulator back (one weight
+// row per thread).  When rows are few (N / 128 tiles leave SMs idle), K is split over the
+// blocks of a thread-block cluster: each block writes its partial sums to its shared
+// memory and the blocks add them through distributed shared memory, each finishing a
+// share of the tokens.  Integer sums are exact, so the split changes nothing.  Rows and
+// tokens past the edges read the TMA's zero fill and are not stored.  Every wait is
+// bounded; a block that gives up drains its copies and MMAs, sets BL_ERRBIT_TIMEOUT and
+// still takes part in the cluster barriers, so no block waits forever.
+#include <cuda_bf16.h>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "bl_device.cuh"
+#include "bl_internal.h"
+
+namespace bl {
+
+bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer, bool swizzle128);
+
+namespace {
+
+constexpr int kRows = 128;       // weight rows per tile (MMA M)
+constexpr int kBK = 128;         // K codes per stage
+constexpr int kPBytes = kRows * (kBK / 4);  // packed weights per stage: 4 KB
+constexpr int kStages = 6;
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2, kExpWarps = 8;
+constexpr int kMaxCluster = 8;
+constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s
+
+template <int BT>
+struct GvCfg {
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 128, "token tile");
+    static constexpr int kXBytes = BT * kBK;
+    static constexpr int kStageBytes = kPBytes + kXBytes;
+    static constexpr int kACols = kBK / 4;  // TMEM columns of one expanded stage
+    // accumulator (BT columns) after the expanded stages, allocated as a power of two
+    static constexpr int kTmemUsed = kStages * kACols + BT;
+    static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kRedBytes = BT * kRows * 4;  // partial sums, aliasing the stages
+    static constexpr int kBarBytes = 8 * (3 * kStages + 2) + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
+    // The request also caps the blocks per SM so that their tensor memory always fits
+    // (2 x 256 or 1 x 512 columns of the SM's 512): a block that waited in tcgen05.alloc
+    // for a block of its own cluster could never be served.  An SM has 228 KB of shared
+    // memory, each block 1 KB more than it asks for.
+    static constexpr int kSmemFloor = kTmemCols == 256 ? 80 * 1024 : 116 * 1024;
+    static constexpr int kSmemLaunch = kSmemBytes > kSmemFloor ? kSmemBytes : kSmemFloor;
+    static_assert(kRedBytes <= kStages * kStageBytes, "reduction buffer");
+    static_assert(kSmemLaunch <= 227 * 1024, "shared memory");
+};
+
+struct GvArgs {
+    const float* s;
+    const float* gamma;
+    int M, N, K;
+    int stages_per_split;  // K stages of each block of a cluster (the last one takes the rest)
+    int nstages;           // K stages in all
+    void* out;
+    int kind;
+    int32_t* err;
+    S4Mul mul;
+    int grow;              // gamma holds one scale per output row
+};
+
+__device__ __forceinline__ void store_out(void* out, int kind, int64_t idx, int acc, float fac) {
+    if (kind == kOutI32) {
+        static_cast<int*>(out)[idx] = acc;
+        return;
+    }
+    const float y = __fmul_rn(__int2float_rn(acc), fac);
+    if (kind == kOutF32)
+        static_cast<float*>(out)[idx] = y;
+    else
+        static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(y);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kDrainNs) return;
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// grid: x = the K split (the blocks of one cluster), y = 128-row weight tiles, z = token
+// tiles of BT.
+template <int BT, int LAY>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
+                   const GvArgs a) {
+    using C = GvCfg<BT>;
+    constexpr int ST = kStages;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sX = base;                       // x tiles first: 1024-aligned for the swizzle
+    const uint32_t sP = sX + ST * C::kXBytes;
+    const uint32_t sBar = sP + ST * kPBytes;
+    auto full = [&](int s) { return sBar + 8u * s; };
+    auto afull = [&](int s) { return sBar + 8u * (ST + s); };
+    auto empty = [&](int s) { return sBar + 8u * (2 * ST + s); };
+    const uint32_t done_bar = sBar + 8u * (3 * ST);
+    const uint32_t drain_bar = sBar + 8u * (3 * ST + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (sBar - base) + 8 * (3 * ST + 2));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* red = reinterpret_cast<int*>(gbase);  // [BT][128] partial sums, after the main loop
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, nsplit = gridDim.x;
+    const int n0 = blockIdx.y * kRows;
+    const int t0 = blockIdx.z * BT;
+    const int kt_begin = split * a.stages_per_split;
+    const int kt_end = split + 1 == nsplit ? a.nstages : kt_begin + a.stages_per_split;
+    const int nk = kt_end - kt_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(afull(s), kExpWarps);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(done_bar, 1);
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_x);
+        tma_prefetch_desc(&tmap_p);
+    }
+    pdl_wait_then_release();
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t acc_col = static_cast<uint32_t>(ST * C::kACols);
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ producer --
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int kt = kt_begin; kt < kt_end; ++kt) {
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(full(stage), C::kXBytes + kPBytes);
+                tma_load_2d(sX + stage * C::kXBytes, &tmap_x, full(stage), kt * kBK, t0);
+                tma_load_2d(sP + stage * kPBytes, &tmap_p, full(stage), kt * (kBK / 4), n0);
+                ++issued;
+                if (++stage == ST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                // wait for every load still in flight before the block may go on
+                for (int s = 0; s < ST; ++s) {
+                    const long long fills = (issued - s + ST - 1) / ST;
+                    if (fills > 0) drain_wait(full(s), static_cast<uint32_t>((fills - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc = idesc_i8(kRows, BT);
+            const uint32_t d_tmem = tmem_base + acc_col;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int i = 0; i < nk; ++i) {
+                if (!mbar_wait_bounded(full(stage), phase, abort_flag) ||
+                    !mbar_wait_bounded(afull(stage), phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(stage * C::kACols);
+                const uint32_t b_addr = sX + stage * C::kXBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 32; ++kk)
+                    tc_mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + 32 * kk), idesc,
+                                     (i | kk) != 0 ? 1u : 0u);
+                tc_commit(empty(stage));
+                if (++stage == ST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // the accumulator is complete (or, after an abort, no MMA is in flight) when
+            // this arrives
+            tc_commit(ok ? done_bar : drain_bar);
+            if (!ok) {
+                drain_wait(drain_bar, 0);
+                mbar_arrive(done_bar);  // let the expander warps leave their wait
+            }
+        }
+    } else {
+        // ------------------------------------------------------------- expanders --
+        // thread: weight row r (its TMEM lane) and half h of each stage (64 codes)
+        const int q = warp & 3, h = (warp - kWarpExp) >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int i = 0; i < nk; ++i) {
+            if (!mbar_wait_bounded(full(stage), phase, abort_flag)) break;
+            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + stage * kPBytes + r * (kBK / 4) +
+                                                            16 * h);
+            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
+            uint32_t v[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                // 16 codes -> 16 int8 in the order of the x_q layout (natural, even/odd,
+                // or stride-4 as 64 * code)
+                if constexpr (LAY == kXqEvenOdd16)
+                    unpack16_evenodd(words[c], v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                else if constexpr (LAY == kXqStride4K16)
+                    unpack16_stride4_x64(words[c], a.mul, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                else
+                    unpack16_natural(words[c], v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+            tmem_st_32x32b_x16(tmem_base + lane_addr + static_cast<uint32_t>(stage * C::kACols + 16 * h), v);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull(stage));
+            if (++stage == ST) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        // ------------------------------------------------------------- epilogue --
+        // both warps of a lane quarter read half of the tokens each
+        constexpr int kAccShift = LAY == kXqStride4K16 ? 6 : 0;
+        const bool got = mbar_wait_bounded(done_bar, 0, abort_flag);
+        tc_fence_after();
+        const int row = n0 + r;
+        const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
+        const float grow_gamma = (a.grow && a.kind != kOutI32 && row < a.N) ? __ldg(a.gamma + row) : 0.0f;
+#pragma unroll 1
+        for (int c0 = 16 * h; c0 < BT; c0 += 32) {
+            uint32_t acc[16];
+            tmem_ld_32x32b_x16(tmem_base + lane_addr + acc_col + static_cast<uint32_t>(c0), acc);
+            tmem_ld_wait();
+            if (!got) continue;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int v = static_cast<int>(acc[j]) >> kAccShift;
+                if (nsplit > 1) {
+                    red[(c0 + j) * kRows + r] = v;
+                } else {
+                    const int tok = t0 + c0 + j;
+                    if (tok < a.M && row < a.N) {
+                        const float sv = a.kind == kOutI32 ? 1.0f : __ldg(a.s + tok);
+                        const float fac = a.kind == kOutI32 ? 0.0f : __fdiv_rn(a.grow ? grow_gamma : gamma, sv);
+                        store_out(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row, v, fac);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (nsplit > 1) {
+        // every block's partial sums are in its shared memory: each block adds, for the
+        // tokens t with t % nsplit == split, the partials of all blocks (fixed order)
+        cluster_sync_all();
+        const int tid = threadIdx.x;
+        const int rr = tid & (kRows - 1);
+        const int row = n0 + rr;
+        const float gamma = (a.kind == kOutI32 || row >= a.N) ? 0.0f : (a.grow ? __ldg(a.gamma + row) : *a.gamma);
+        const uint32_t red_addr = smem_u32(red);
+        for (int tt = split + nsplit * (tid / kRows); tid < 2 * kRows && tt < BT; tt += 2 * nsplit) {
+            const int tok = t0 + tt;
+            if (tok >= a.M || row >= a.N) continue;
+            int sum = 0;
+            for (int b = 0; b < nsplit; ++b)
+                sum += static_cast<int>(ld_shared_cluster_u32(mapa_shared(red_addr + 4u * (tt * kRows + rr), b)));
+            const float fac = a.kind == kOutI32 ? 0.0f : __fdiv_rn(gamma, __ldg(a.s + tok));
+            store_out(a.out, a.kind, static_cast<int64_t>(tok) * a.N + row, sum, fac);
+        }
+        // no block leaves while another may still read its shared memory
+        cluster_sync_all();
+    }
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+    if (threadIdx.x == 0 && *abort_flag && a.err != nullptr) atomicOr(a.err, kErrBitTimeout);
+}
+
+int sm_count_gtc() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+template <int BT, int LAY>
+cudaError_t launch_bt(const CUtensorMap& tx, const CUtensorMap& tp, const GvArgs& a, dim3 grid, cudaStream_t stream) {
+    using C = GvCfg<BT>;
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(gemv_tc_kernel<BT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemLaunch);
+    });
+    if (e != cudaSuccess) return e;
+    return launch_pdl(gemv_tc_kernel<BT, LAY>, grid, dim3(kThreads), C::kSmemLaunch, stream,
+                      grid.x > 1 ? dim3(grid.x, 1, 1) : dim3(kNoCluster), tx, tp, a);
+}
+
+template <int LAY>
+cudaError_t launch_layout(int bt, const CUtensorMap& tx, const CUtensorMap& tp, const GvArgs& a, dim3 grid,
+                          cudaStream_t stream) {
+    switch (bt) {
+        case 16: return launch_bt<16, LAY>(tx, tp, a, grid, stream);
+        case 32: return launch_bt<32, LAY>(tx, tp, a, grid, stream);
+        case 64: return launch_bt<64, LAY>(tx, tp, a, grid, stream);
+        default: return launch_bt<128, LAY>(tx, tp, a, grid, stream);
+    }
+}
+
+}  // namespace
+
+// Token tile for M tokens: the smallest of 16, 32, 64, 128 that holds them (M > 128 runs
+// several token tiles, each streaming the weights again).
+int gemv_tc_token_tile(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma, int64_t M,
+                           int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout, cudaStream_t stream) {
+    const int bt = gemv_tc_token_tile(M);
+    const int sms = sm_count_gtc();
+    const int64_t row_tiles = (N + kRows - 1) / kRows;
+    const int64_t tok_tiles = (M + bt - 1) / bt;
+    const int nstages = static_cast<int>((K + kBK - 1) / kBK);
+    // split K over a cluster until the blocks cover every SM twice (two blocks fit an SM),
+    // keeping at least two stages per block
+    int64_t split = (2 * sms + row_tiles * tok_tiles - 1) / (row_tiles * tok_tiles);
+    if (split > kMaxCluster) split = kMaxCluster;
+    if (split > nstages / 2) split = nstages / 2;
+    if (split < 1) split = 1;
+    if (row_tiles > 65535 || tok_tiles > 65535) return cudaErrorInvalidValue;
+    CUtensorMap tx, tp;
+    if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, bt, true) ||
+        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kBK / 4, kRows,
+                           false))
+        return cudaErrorInvalidValue;
+    GvArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+             static_cast<int>(nstages / split), nstages, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
+    const dim3 grid(static_cast<unsigned>(split), static_cast<unsigned>(row_tiles), static_cast<unsigned>(tok_tiles));
+    switch (layout) {
+        case kXqEvenOdd16: return launch_layout<kXqEvenOdd16>(bt, tx, tp, a, grid, stream);
+        case kXqStride4K16: return launch_layout<kXqStride4K16>(bt, tx, tp, a, grid, stream);
+        default: return launch_layout<kXqRowMajor>(bt, tx, tp, a, grid, stream);
+    }
+}
+
+}  // namespace bl

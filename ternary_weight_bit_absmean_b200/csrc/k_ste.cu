@@ -1,4 +1,5 @@
-// k_ste.cu -- the straight-through backward of the BitLinear forward.
+// k_ste.cu -- the straight-through backward of the BitLinear forward, on the 5th-generation
+// tensor cores (tcgen05.mma kind::f16, fp32 accumulators in tensor memory).
 //
 // "1-bit & Ternary LLMs (BitNet b1.58)", "Training: shadow weights + the straight-through
 // estimator": the forward uses the ternary weights, and the backward treats the
@@ -9,17 +10,39 @@
 //   dW[n,k] = gamma sum_m dY[m,n] x_q[m,k] / s[m]    (a contraction over the tokens)
 // The next forward re-ternarises the updated shadow weights (the quantisation kernels).
 //
-// Both are output-stationary SIMT tiles: a 128 x 128 output tile per block of 256
-// threads, 8 x 8 outputs per thread in fp32 registers (rows 4ty..4ty+3 and 64+4ty..,
-// columns likewise, so the shared-memory reads of a warp are conflict-free float4s), the
-// contraction in chunks of 16 staged through two shared-memory buffers: the next
-// chunk's global loads are issued before the current chunk's products and stored into
-// the other buffer after them.  Operands are expanded to fp32 on the way in (codes to
-// -1/0/+1, x_q to its integer value, dY divided by s for dW).  The products with a code
-// are exact and the sums round in fp32 in contraction order; gamma scales once.
-#include <cuda_runtime.h>
-
+// Both are one GEMM shape, D[i][j] = sum_c A[i][c] B[j][c], written out as
+// out[i][j] = gamma D[i][j]:
+//   dX: i = token m, j = column k, c = n;  A[m][n] = dY[m][n],        B[k][n] = c[n][k]
+//   dW: i = row n,   j = column k, c = m;  A[n][m] = dY[m][n] / s[m], B[k][m] = x_q[m][k]
+// B is exact in bf16 (codes are -1/0/+1; |x_q| <= 128 needs 8 significant bits).  The
+// fp32 operand A is split into two bf16 parts, A = hi + lo + d with hi = bf16(A),
+// lo = bf16(A - hi) (A - hi is exact in fp32) and |d| <= 2^-16 |A|; both parts are
+// multiplied by the same B tile into one fp32 accumulator, so each product hi*b and lo*b
+// is exact and the result carries the fp32 accumulation error plus 2^-16 relative per
+// term -- near the precision of an fp32 contraction, at the bf16 tensor-core rate (two
+// MMAs per K step).  For dW, A = dY * (1 / s[m]) with the reciprocal rounded to fp32
+// (2^-23 relative per term more).
+//
+// Tile: 128 rows i (MMA M, TMEM lanes) x BJ columns j (MMA N, BJ = 128 or 256), the
+// contraction in stages of 64 (one 128-byte swizzled bf16 row).  No operand is in a
+// layout TMA could load directly (dY must be split; the codes and x_q must be transposed
+// to put the contraction index innermost), so every operand is written by threads:
+//   warp 0 (one lane)  MMA issuer: per stage, for each 16-wide K step, one MMA with A_hi
+//                      and one with A_lo against B; tcgen05.commit frees the stage;
+//   warps 1-4          A producers: load fp32 dY, scale by 1/s for dW, split, and write
+//                      A_hi and A_lo in the 128-byte-swizzled K-major layout;
+//   warps 5-12         B producers: expand 2-bit codes (dX) or int8 x_q (dW) to bf16,
+//                      transposed into the same layout;
+//   warps 13-16        epilogue: tcgen05.ld of the finished accumulator (one row i per
+//                      thread, 32 columns at a time), times gamma, row-contiguous stores.
+// Two TMEM accumulators let the epilogue of one tile overlap the main loop of the next
+// (persistent blocks, one per SM).  Rows, columns and contraction entries past the
+// matrix edges are written as zeros.  Every wait is bounded (BL_ERRBIT_TIMEOUT is not
+// reported here: the backward has no error word, so a timed-out launch returns early and
+// leaves its output incomplete).
+#include <cuda_bf16.h>
 #include <cstdint>
+#include <cuda_runtime.h>
 
 #include "bl_device.cuh"
 #include "bl_internal.h"
@@ -27,178 +50,486 @@
 namespace bl {
 namespace {
 
-constexpr int kTile = 128;  // output tile edge
-constexpr int kChunk = 16;  // contraction chunk
-constexpr int kThreads = 256;
-constexpr int kPad = 4;
+constexpr int kBI = 128;           // rows per tile (MMA M)
+constexpr int kBC = 64;            // contraction elements per stage (128 bytes of bf16)
+constexpr int kRowBytes = 128;     // one swizzled K-major row
+constexpr int kThreads = 544;      // 17 warps
+constexpr int kWarpMma = 0, kWarpA = 1, kWarpB = 5, kWarpEpi = 13;
+constexpr int kAWarps = kWarpB - kWarpA, kBWarps = kWarpEpi - kWarpB, kEpiWarps = 4;
+constexpr int kSmemBudget = 200 * 1024;
+constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s
 
-__device__ __forceinline__ float code_of(uint32_t byte, int i) {
-    const uint32_t c = (byte >> (2 * i)) & 3u;
-    return c == 1u ? 1.0f : (c == 2u ? -1.0f : 0.0f);  // 11 reads as 0
+enum SteKind : int { kDX = 0, kDW = 1 };
+
+template <int BJ>
+struct SteCfg {
+    static_assert(BJ == 128 || BJ == 256, "column tile");
+    static constexpr int kATile = kBI * kRowBytes;  // one bf16 part of A
+    static constexpr int kBTile = BJ * kRowBytes;
+    static constexpr int kStageBytes = 2 * kATile + kBTile;
+    static constexpr int kStages = kSmemBudget / kStageBytes;
+    static constexpr int kTmemCols = 2 * BJ;
+    static constexpr int kBarBytes = 8 * (2 * kStages + 5) + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
+    static_assert(kStages >= 2, "stages");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct SteArgs {
+    const float* dY;        // [M, N]
+    const uint8_t* packed;  // dX: [N, K/4]
+    const int8_t* xq;       // dW: [M, K]
+    const float* s;         // dW: [M]
+    const float* gamma;
+    float* out;             // dX [M, K] or dW [N, K]
+    int M, N, K;
+    int I, J, C;            // rows, columns and contraction length of D
+    int tiles_i, num_tiles;
+};
+
+// Instruction descriptor: kind::f16 with A and B bf16, K-major, D fp32, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4)                                // D format: F32
+           | (1u << 7)                              // A format: BF16
+           | (1u << 10)                             // B format: BF16
+           | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
-// acc[i][j] += A[c][row i] * B[c][col j] over one staged chunk; the thread's rows are
-// 4ty + (0..3) and 64 + 4ty + (0..3), its columns 4tx + (0..3) and 64 + 4tx + (0..3).
-__device__ __forceinline__ void chunk_fma(const float (*sA)[kTile + kPad], const float (*sB)[kTile + kPad], int ty,
-                                          int tx, float (&acc)[8][8]) {
-#pragma unroll
-    for (int c = 0; c < kChunk; ++c) {
-        const float4 a0 = *reinterpret_cast<const float4*>(&sA[c][4 * ty]);
-        const float4 a1 = *reinterpret_cast<const float4*>(&sA[c][64 + 4 * ty]);
-        const float4 b0 = *reinterpret_cast<const float4*>(&sB[c][4 * tx]);
-        const float4 b1 = *reinterpret_cast<const float4*>(&sB[c][64 + 4 * tx]);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(av[i], bv[j], acc[i][j]);
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, issued by one thread.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_drain_ste(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kDrainNs) return;
     }
 }
 
-__device__ __forceinline__ int out_index(int t, int h) { return h * 64 + 4 * t; }
+// Byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ uint32_t sw128(int r, int ch) {
+    return static_cast<uint32_t>(r) * kRowBytes + (static_cast<uint32_t>(ch ^ (r & 7)) << 4);
+}
 
-// dX tile (tokens m0.., columns k0..): A = dY[m, n] staged as [n][m], B = codes[n, k].
-// Per chunk a thread loads 8 dY values (e = tid + 256 u: token e / 16, n e % 16) and
-// 2 packed bytes (e = tid + 256 u: row e / 32, byte e % 32).
-__global__ void __launch_bounds__(kThreads) ste_grad_input_kernel(const float* __restrict__ dY,
-                                                                 const uint8_t* __restrict__ packed,
-                                                                 const float* __restrict__ gamma, int M, int N,
-                                                                 int K, float* __restrict__ dX) {
+// Split 8 fp32 values into bf16 hi and lo parts (x = hi + lo + d, |d| <= 2^-16 |x|),
+// each as one 16-byte chunk (element e in the low half of word e / 2 when e is even).
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * p], x[2 * p + 1]);
+        const uint32_t hw = *reinterpret_cast<const uint32_t*>(&hb);
+        const float r0 = __fsub_rn(x[2 * p], __uint_as_float(hw << 16));          // exact
+        const float r1 = __fsub_rn(x[2 * p + 1], __uint_as_float(hw & 0xFFFF0000u));  // exact
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(r0, r1);
+        h[p] = hw;
+        l[p] = *reinterpret_cast<const uint32_t*>(&lb);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Byte table for the code expansion: for a 2-bit code c, byte c of kLoTab and byte c of
+// kHiTab are the low and high bytes of bf16(c): 00 -> 0, 01 -> +1 (0x3F80), 10 -> -1
+// (0xBF80), 11 -> 0.
+constexpr uint32_t kLoTab = 0x00808000u;
+constexpr uint32_t kHiTab = 0x00BF3F00u;
+
+// Four codes, one per byte of x (bits 0..1 of each byte), to four bf16 values: the two
+// words (bf16 of byte 0 | bf16 of byte 1 << 16) and (byte 2 | byte 3 << 16).
+__device__ __forceinline__ void codes4_to_bf16(uint32_t x, uint32_t& w01, uint32_t& w23) {
+    // selector nibbles c and 4 + c per byte: c * 0x11 + 0x40, no carries (c <= 3)
+    const uint32_t y = x * 0x11u + 0x40404040u;
+    w01 = __byte_perm(kLoTab, kHiTab, y);
+    w23 = __byte_perm(kLoTab, kHiTab, y >> 16);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_of_s8(uint32_t a, uint32_t b) {
+    // a, b: int8 values in the low byte; exact in bf16
+    const __nv_bfloat162 v = __floats2bfloat162_rn(static_cast<float>(static_cast<int8_t>(a & 0xFFu)),
+                                                   static_cast<float>(static_cast<int8_t>(b & 0xFFu)));
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int KIND, int BJ>
+__global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
+    using Cfg = SteCfg<BJ>;
+    constexpr int ST = Cfg::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    auto sAhi = [&](int s) { return static_cast<uint32_t>(s * Cfg::kStageBytes); };
+    auto sAlo = [&](int s) { return static_cast<uint32_t>(s * Cfg::kStageBytes + Cfg::kATile); };
+    auto sB = [&](int s) { return static_cast<uint32_t>(s * Cfg::kStageBytes + 2 * Cfg::kATile); };
+    const uint32_t sBar = base + ST * Cfg::kStageBytes;
+    auto full = [&](int s) { return sBar + 8u * s; };
+    auto empty = [&](int s) { return sBar + 8u * (ST + s); };
+    auto tfull = [&](int b) { return sBar + 8u * (2 * ST + b); };
+    auto tempty = [&](int b) { return sBar + 8u * (2 * ST + 2 + b); };
+    const uint32_t drain_bar = sBar + 8u * (2 * ST + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + ST * Cfg::kStageBytes + 8 * (2 * ST + 5));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(full(s), kAWarps + kBWarps);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
     pdl_wait_then_release();
-    __shared__ __align__(16) float sA[2][kChunk][kTile + kPad];
-    __shared__ __align__(16) float sB[2][kChunk][kTile + kPad];
-    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-    const int m0 = blockIdx.y * kTile, k0 = blockIdx.x * kTile;
-    const int KB = K / 4;
-    float ra[8];
-    uint32_t rb[2];
-    auto load = [&](int n0) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + kThreads * u;
-            const int m = m0 + e / kChunk, n = n0 + e % kChunk;
-            ra[u] = (m < M && n < N) ? __ldg(dY + static_cast<int64_t>(m) * N + n) : 0.0f;
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + kThreads * u;
-            const int n = n0 + e / (kTile / 4), kb = k0 / 4 + e % (kTile / 4);
-            rb[u] = (n < N && kb < KB) ? __ldg(packed + static_cast<int64_t>(n) * KB + kb) : 0u;
-        }
-    };
-    auto store = [&](int buf) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + kThreads * u;
-            sA[buf][e % kChunk][e / kChunk] = ra[u];
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + kThreads * u;
-            const int r = e / (kTile / 4), b = e % (kTile / 4);
-            *reinterpret_cast<float4*>(&sB[buf][r][4 * b]) =
-                make_float4(code_of(rb[u], 0), code_of(rb[u], 1), code_of(rb[u], 2), code_of(rb[u], 3));
-        }
-    };
-    float acc[8][8] = {};
-    load(0);
-    store(0);
-    __syncthreads();
-    int buf = 0;
-    for (int n0 = 0; n0 < N; n0 += kChunk) {
-        const bool more = n0 + kChunk < N;
-        if (more) load(n0 + kChunk);
-        chunk_fma(sA[buf], sB[buf], ty, tx, acc);
-        if (more) store(buf ^ 1);
-        __syncthreads();
-        buf ^= 1;
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+        tmem_relinquish();
     }
-    const float g = *gamma;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nC = (a.C + kBC - 1) / kBC;
+
+    if (warp == kWarpMma) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc = idesc_bf16(kBI, BJ);
+            int stage = 0, buf = 0;
+            uint32_t phase = 0, bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+                if (!mbar_wait_bounded(tempty(buf), bphase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BJ);
+                for (int kc = 0; kc < nC; ++kc) {
+                    if (!mbar_wait_bounded(full(stage), phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int m = m0 + out_index(ty, i / 4) + i % 4;
-        if (m >= M) continue;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int k = k0 + out_index(tx, j / 4) + j % 4;
-            if (k < K) dX[static_cast<int64_t>(m) * K + k] = __fmul_rn(g, acc[i][j]);
+                    for (int kk = 0; kk < kBC / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(base + sB(stage) + 32 * kk);
+                        tc_mma_bf16(d_tmem, smem_desc_sw128(base + sAhi(stage) + 32 * kk), bd, idesc,
+                                    (kc | kk) != 0 ? 1u : 0u);
+                        tc_mma_bf16(d_tmem, smem_desc_sw128(base + sAlo(stage) + 32 * kk), bd, idesc, 1u);
+                    }
+                    tc_commit(empty(stage));
+                    if (++stage == ST) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(tfull(buf));
+                if (++buf == 2) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+            if (!ok) {
+                // let every MMA already issued finish before TMEM is released
+                tc_commit(drain_bar);
+                mbar_drain_ste(drain_bar, 0);
+            }
         }
+    } else if (warp < kWarpB) {
+        // ------------------------------------------------------------ A producers --
+        const int t = threadIdx.x - 32 * kWarpA;  // 0 .. 127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+            const int i0 = (tile % a.tiles_i) * kBI;
+            for (int kc = 0; kc < nC; ++kc) {
+                const int c0 = kc * kBC;
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* ahi = gbase + sAhi(stage);
+                uint8_t* alo = gbase + sAlo(stage);
+                if constexpr (KIND == kDX) {
+                    // A[m][n] = dY[m][n]: eight threads per row, each eight consecutive n
+                    const int r_off = t >> 3, ch = t & 7;
+                    const int n = c0 + 8 * ch;
+                    const bool vec = (a.N & 3) == 0 && n + 8 <= a.N;
+#pragma unroll 2
+                    for (int p = 0; p < kBI / 16; ++p) {
+                        const int r = 16 * p + r_off;
+                        const int m = i0 + r;
+                        float x[8];
+                        if (m < a.M && vec) {
+                            const float4* src = reinterpret_cast<const float4*>(a.dY + static_cast<int64_t>(m) * a.N + n);
+                            const float4 u = __ldg(src), v = __ldg(src + 1);
+                            x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+                            x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                x[e] = (m < a.M && n + e < a.N) ? __ldg(a.dY + static_cast<int64_t>(m) * a.N + n + e)
+                                                                : 0.0f;
+                        }
+                        uint4 hi, lo;
+                        split8(x, hi, lo);
+                        *reinterpret_cast<uint4*>(ahi + sw128(r, ch)) = hi;
+                        *reinterpret_cast<uint4*>(alo + sw128(r, ch)) = lo;
+                    }
+                } else {
+                    // A[n][m] = dY[m][n] / s[m]: one thread per row n, the stage's 64 tokens.
+                    // Each warp forms the 64 reciprocals itself (two per lane) and hands them
+                    // round by shuffles, so the producer warps never wait on one another.
+                    const int mA = c0 + lane, mB = c0 + 32 + lane;
+                    const float rA = mA < a.M ? __frcp_rn(__ldg(a.s + mA)) : 0.0f;
+                    const float rB = mB < a.M ? __frcp_rn(__ldg(a.s + mB)) : 0.0f;
+                    const int n = i0 + t;
+                    const bool row_ok = n < a.N;
+#pragma unroll 1
+                    for (int ch = 0; ch < kBC / 8; ++ch) {
+                        const float rsrc = ch < 4 ? rA : rB;
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int m = c0 + 8 * ch + e;
+                            const float rm = __shfl_sync(0xffffffffu, rsrc, (8 * ch + e) & 31);
+                            x[e] = (row_ok && m < a.M)
+                                       ? __fmul_rn(__ldg(a.dY + static_cast<int64_t>(m) * a.N + n), rm)
+                                       : 0.0f;
+                        }
+                        uint4 hi, lo;
+                        split8(x, hi, lo);
+                        *reinterpret_cast<uint4*>(ahi + sw128(t, ch)) = hi;
+                        *reinterpret_cast<uint4*>(alo + sw128(t, ch)) = lo;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full(stage));
+                if (++stage == ST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp < kWarpEpi) {
+        // ------------------------------------------------------------ B producers --
+        const int t = threadIdx.x - 32 * kWarpB;  // 0 .. 255
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+            const int j0 = (tile / a.tiles_i) * BJ;
+            for (int kc = 0; kc < nC; ++kc) {
+                const int c0 = kc * kBC;
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* bt = gbase + sB(stage);
+                if constexpr (KIND == kDX) {
+                    // B[k][n] = c[n][k]: a unit is 8 consecutive k (two packed bytes per n)
+                    // x 8 consecutive n; the warp's lanes take consecutive k groups of one
+                    // n chunk, so each load of a warp reads one packed row contiguously
+                    const int KB = a.K >> 2;
+                    for (int u = t; u < (BJ / 8) * 8; u += 32 * kBWarps) {
+                        const int kg = u % (BJ / 8), nch = u / (BJ / 8);
+                        const int k = j0 + 8 * kg, n = c0 + 8 * nch;
+                        uint32_t w[8];  // bytes k/4 and k/4 + 1 of row n + q, in bits 0..15
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            w[q] = 0;
+                            if (n + q < a.N) {
+                                const uint8_t* row = a.packed + static_cast<int64_t>(n + q) * KB;
+                                if (k + 8 <= a.K && (KB & 1) == 0) {
+                                    w[q] = __ldg(reinterpret_cast<const uint16_t*>(row + (k >> 2)));
+                                } else {
+                                    if (k < a.K) w[q] = __ldg(row + (k >> 2));
+                                    if (k + 4 < a.K) w[q] |= static_cast<uint32_t>(__ldg(row + (k >> 2) + 1)) << 8;
+                                }
+                            }
+                        }
+                        // gather byte b (k rows 4b .. 4b + 3) of n = q into byte q % 4 of
+                        // g[b][q / 4]
+                        uint32_t g[2][2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t t01 = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
+                            const uint32_t t23 = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
+                            g[0][h] = __byte_perm(t01, t23, 0x5410);
+                            g[1][h] = __byte_perm(t01, t23, 0x7632);
+                        }
+#pragma unroll
+                        for (int kr = 0; kr < 8; ++kr) {
+                            const int b = kr >> 2, sh = 2 * (kr & 3);
+                            uint4 o;
+                            codes4_to_bf16((g[b][0] >> sh) & 0x03030303u, o.x, o.y);
+                            codes4_to_bf16((g[b][1] >> sh) & 0x03030303u, o.z, o.w);
+                            *reinterpret_cast<uint4*>(bt + sw128(8 * kg + kr, nch)) = o;
+                        }
+                    }
+                } else {
+                    // B[k][m] = x_q[m][k]: a unit is 4 consecutive k (one word per token) x 8
+                    // consecutive m; lanes take consecutive k words of one m chunk
+                    for (int u = t; u < (BJ / 4) * 8; u += 32 * kBWarps) {
+                        const int kw = u % (BJ / 4), mch = u / (BJ / 4);
+                        const int k = j0 + 4 * kw, m = c0 + 8 * mch;
+                        uint32_t w[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            w[q] = (m + q < a.M && k < a.K)
+                                       ? __ldg(reinterpret_cast<const uint32_t*>(a.xq + static_cast<int64_t>(m + q) * a.K + k))
+                                       : 0u;
+#pragma unroll
+                        for (int kr = 0; kr < 4; ++kr) {
+                            uint4 o;
+                            o.x = bf16x2_of_s8(w[0] >> (8 * kr), w[1] >> (8 * kr));
+                            o.y = bf16x2_of_s8(w[2] >> (8 * kr), w[3] >> (8 * kr));
+                            o.z = bf16x2_of_s8(w[4] >> (8 * kr), w[5] >> (8 * kr));
+                            o.w = bf16x2_of_s8(w[6] >> (8 * kr), w[7] >> (8 * kr));
+                            *reinterpret_cast<uint4*>(bt + sw128(4 * kw + kr, mch)) = o;
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full(stage));
+                if (++stage == ST) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue --
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const float g = *a.gamma;
+        const bool vec = (a.J & 3) == 0;
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+            const int i0 = (tile % a.tiles_i) * kBI, j0 = (tile / a.tiles_i) * BJ;
+            if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag)) break;
+            tc_fence_after();
+            const int i = i0 + 32 * q + lane;
+            float* orow = a.out + static_cast<int64_t>(i) * a.J;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BJ; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(buf * BJ + c0),
+                                   r);
+                tmem_ld_wait();
+                if (i >= a.I) continue;
+                const int j = j0 + c0;
+                if (vec && j + 32 <= a.J) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(orow + j + e) =
+                            make_float4(__fmul_rn(g, __uint_as_float(r[e])), __fmul_rn(g, __uint_as_float(r[e + 1])),
+                                        __fmul_rn(g, __uint_as_float(r[e + 2])),
+                                        __fmul_rn(g, __uint_as_float(r[e + 3])));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j + e < a.J) orow[j + e] = __fmul_rn(g, __uint_as_float(r[e]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty(buf));
+            if (++buf == 2) {
+                buf = 0;
+                bphase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }
 }
 
-// dW tile (rows n0.., columns k0..): A = dY[m, n] / s[m] staged as [m][n], B = x_q[m, k].
-// Per chunk a thread loads 8 dY values and 8 x_q values (e = tid + 256 u: token e / 128,
-// column e % 128).
-__global__ void __launch_bounds__(kThreads) ste_grad_weight_kernel(const float* __restrict__ dY,
-                                                                  const int8_t* __restrict__ xq,
-                                                                  const float* __restrict__ s,
-                                                                  const float* __restrict__ gamma, int M, int N,
-                                                                  int K, float* __restrict__ dW) {
-    pdl_wait_then_release();
-    __shared__ __align__(16) float sA[2][kChunk][kTile + kPad];
-    __shared__ __align__(16) float sB[2][kChunk][kTile + kPad];
-    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
-    const int n0 = blockIdx.y * kTile, k0 = blockIdx.x * kTile;
-    float ra[8], rb[8];
-    auto load = [&](int mc) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + kThreads * u;
-            const int m = mc + e / kTile, c = e % kTile;
-            const int n = n0 + c, k = k0 + c;
-            ra[u] = (m < M && n < N) ? __fdiv_rn(__ldg(dY + static_cast<int64_t>(m) * N + n), __ldg(s + m)) : 0.0f;
-            rb[u] = (m < M && k < K) ? static_cast<float>(__ldg(xq + static_cast<int64_t>(m) * K + k)) : 0.0f;
-        }
-    };
-    auto store = [&](int buf) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = tid + kThreads * u;
-            sA[buf][e / kTile][e % kTile] = ra[u];
-            sB[buf][e / kTile][e % kTile] = rb[u];
-        }
-    };
-    float acc[8][8] = {};
-    load(0);
-    store(0);
-    __syncthreads();
-    int buf = 0;
-    for (int mc = 0; mc < M; mc += kChunk) {
-        const bool more = mc + kChunk < M;
-        if (more) load(mc + kChunk);
-        chunk_fma(sA[buf], sB[buf], ty, tx, acc);
-        if (more) store(buf ^ 1);
-        __syncthreads();
-        buf ^= 1;
-    }
-    const float g = *gamma;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int n = n0 + out_index(ty, i / 4) + i % 4;
-        if (n >= N) continue;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int k = k0 + out_index(tx, j / 4) + j % 4;
-            if (k < K) dW[static_cast<int64_t>(n) * K + k] = __fmul_rn(g, acc[i][j]);
+int sm_count_ste() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// Column tile: the one with fewer waves x columns per tile (a tile's time is about
+// proportional to its columns once the producers keep up); ties go to 256.
+int ste_tile(int64_t I, int64_t J, int sms) {
+    const int64_t ti = (I + kBI - 1) / kBI;
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bj : {256, 128}) {
+        const int64_t tiles = ti * ((J + bj - 1) / bj);
+        const int64_t cost = (tiles + sms - 1) / sms * bj;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bj;
         }
     }
+    return best;
+}
+
+template <int KIND, int BJ>
+cudaError_t launch_ste_bj(SteArgs a, int sms, cudaStream_t stream) {
+    using Cfg = SteCfg<BJ>;
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(ste_tc_kernel<KIND, BJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
+    a.tiles_i = (a.I + kBI - 1) / kBI;
+    a.num_tiles = a.tiles_i * ((a.J + BJ - 1) / BJ);
+    const int grid = a.num_tiles < sms ? a.num_tiles : sms;
+    return launch_pdl(ste_tc_kernel<KIND, BJ>, dim3(grid), dim3(kThreads), Cfg::kSmemBytes, stream,
+                      dim3(kNoCluster), a);
+}
+
+template <int KIND>
+cudaError_t launch_ste(SteArgs a, cudaStream_t stream) {
+    const int sms = sm_count_ste();
+    if (ste_tile(a.I, a.J, sms) == 256) return launch_ste_bj<KIND, 256>(a, sms, stream);
+    return launch_ste_bj<KIND, 128>(a, sms, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_ste_grad_input(const float* dY, const uint8_t* packed, const float* gamma, int64_t M, int64_t N,
                                   int64_t K, float* dX, cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>((K + kTile - 1) / kTile), static_cast<unsigned>((M + kTile - 1) / kTile));
-    return launch_pdl(ste_grad_input_kernel, grid, dim3(kThreads), 0, stream, dim3(kNoCluster), dY, packed, gamma,
-                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), dX);
+    SteArgs a{dY, packed, nullptr, nullptr, gamma, dX, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+              static_cast<int>(M), static_cast<int>(K), static_cast<int>(N), 0, 0};
+    return launch_ste<kDX>(a, stream);
 }
 
 cudaError_t launch_ste_grad_weight(const float* dY, const int8_t* xq, const float* s, const float* gamma, int64_t M,
                                    int64_t N, int64_t K, float* dW, cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>((K + kTile - 1) / kTile), static_cast<unsigned>((N + kTile - 1) / kTile));
-    return launch_pdl(ste_grad_weight_kernel, grid, dim3(kThreads), 0, stream, dim3(kNoCluster), dY, xq, s, gamma,
-                      static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), dW);
+    SteArgs a{dY, nullptr, xq, s, gamma, dW, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+              static_cast<int>(N), static_cast<int>(K), static_cast<int>(M), 0, 0};
+    return launch_ste<kDW>(a, stream);
 }
 
 }  // namespace bl

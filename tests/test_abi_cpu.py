@@ -176,12 +176,13 @@ def test_ste_backward_validation(L):
     assert fi(None, FAKE, FAKE, 4, 8, 64, FAKE, None) == INVALID
     assert fi(FAKE, FAKE, FAKE, 0, 8, 64, FAKE, None) == INVALID
     assert fi(FAKE, FAKE, FAKE, 4, 8, 66, FAKE, None) == SHAPE          # K % 4
-    assert fi(FAKE, FAKE, FAKE, 65535 * 64 + 1, 8, 64, FAKE, None) == SHAPE
+    assert fi(FAKE, FAKE, FAKE, 1 << 31, 8, 64, FAKE, None) == SHAPE
     assert fi(FAKE, ODD, FAKE, 4, 8, 64, FAKE, None) == MISALIGNED
     fw = L.bitlinear_ste_backward_weight
     assert fw(FAKE, FAKE, FAKE, None, 4, 8, 64, FAKE, None) == INVALID
     assert fw(FAKE, FAKE, FAKE, FAKE, 4, -8, 64, FAKE, None) == INVALID
-    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 65535 * 64 + 1, 64, FAKE, None) == SHAPE
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 1 << 31, 64, FAKE, None) == SHAPE
+    assert fw(FAKE, FAKE, FAKE, FAKE, 4, 8, 66, FAKE, None) == SHAPE      # K % 4
     assert fw(FAKE, FAKE, ODD, FAKE, 4, 8, 64, FAKE, None) == MISALIGNED
     assert fw(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, ODD, None) == MISALIGNED
 
