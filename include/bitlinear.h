@@ -217,6 +217,24 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
                                  bl_dtype out_dtype, int32_t *err_word, bl_path path,
                                  void *stream);
 
+/* A test of the bounded device waits (the source pages have no counterpart): the forward
+ * of bitlinear_forward_layout on one of the kernels that wait for TMA loads
+ * (BL_PATH_TC_1SM, BL_PATH_SKINNY, or BL_PATH_GEMV where it runs its TMA-fed form:
+ * x_q in BL_XQ_K16_STRIDE4 and a layer wide enough), in which every wait gives up after
+ * wait_limit_ns (0 < wait_limit_ns <= 2 s; the forward entry points use 2 s) and the
+ * load producer of each block stops after stall_after_loads loads.  The waits for the
+ * next load then run out: the kernel stops its other roles, lets every copy and MMA in
+ * flight finish, frees its tensor memory, ORs BL_ERRBIT_TIMEOUT into err_word and
+ * returns; the output is left incomplete.  If a block needs no more loads than
+ * stall_after_loads it finishes normally.  The next call on the stream runs as usual.
+ * Errors: those of bitlinear_forward_layout; BL_ERR_INVALID_ARG for another path or a
+ * limit out of range, BL_ERR_UNSUPPORTED_SHAPE for a GEMV shape without the TMA form. */
+BL_API bl_status bitlinear_forward_stall_test(const int8_t *xq, const float *s, const uint8_t *packed,
+                                              const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
+                                              bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,
+                                              bl_path path, uint64_t wait_limit_ns, int32_t stall_after_loads,
+                                              void *stream);
+
 /* bitlinear_quantize_weights for callers that cannot allocate device memory.  The
  * source pages have no counterpart to this entry point; it exists for the library's
  * users.  Callers such as a serving loop that must not call cudaMalloc (which can

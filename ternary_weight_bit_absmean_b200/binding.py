@@ -33,7 +33,7 @@ EXPORTED = [
     "bitlinear_forward", "bitlinear_forward_path", "bitlinear_quantize_act_layout",
     "bitlinear_forward_layout", "bitlinear_norm_quantize_act", "bitlinear_forward_rowscale",
     "bitlinear_tl5_row_bytes", "bitlinear_pack_tl5", "bitlinear_repack_tl5", "bitlinear_forward_tl5",
-    "bitlinear_ste_backward_input", "bitlinear_ste_backward_weight",
+    "bitlinear_ste_backward_input", "bitlinear_ste_backward_weight", "bitlinear_forward_stall_test",
     "bitlinear_last_cuda_error",
     "bitlinear_status_string",
 ]
@@ -96,6 +96,9 @@ def lib() -> ctypes.CDLL:
         L.bitlinear_ste_backward_input.restype = S
         L.bitlinear_ste_backward_weight.argtypes = [P, P, P, P, I64, I64, I64, P, P]
         L.bitlinear_ste_backward_weight.restype = S
+        L.bitlinear_forward_stall_test.argtypes = [P, P, P, P, I64, I64, I64, P, S, P, S, S, ctypes.c_uint64,
+                                                   ctypes.c_int32, P]
+        L.bitlinear_forward_stall_test.restype = S
         L.bitlinear_last_cuda_error.argtypes = []
         L.bitlinear_last_cuda_error.restype = ctypes.c_int
         L.bitlinear_status_string.argtypes = [ctypes.c_int]
@@ -199,6 +202,22 @@ def bitlinear_forward(xq, s, packed, gamma, out, err_word=None, stream=None, pat
         _check(lib().bitlinear_forward(*args, _stream(stream)), "bitlinear_forward")
     else:
         _check(lib().bitlinear_forward_path(*args, int(path), _stream(stream)), "bitlinear_forward_path")
+
+
+def bitlinear_forward_stall_test(xq, s, packed, gamma, out, err_word, wait_limit_ns, stall_after_loads,
+                                 stream=None, path=BL_PATH_TC_1SM, layout=BL_XQ_ROWMAJOR):
+    """The forward with every device wait limited to wait_limit_ns and each block's load
+    producer stopped after stall_after_loads loads (a test of the bounded waits)."""
+    M, K = xq.shape
+    N = packed.shape[0]
+    kind = {v: k for k, v in _OUT_DT.items()}.get(out.dtype)
+    if kind is None:
+        raise TypeError("out must be float32, bfloat16 or int32")
+    _check(lib().bitlinear_forward_stall_test(
+        _dev(xq, torch.int8, "xq"), _dev(s, torch.float32, "s", (M,)),
+        _dev(packed, torch.uint8, "packed", (N, K // 4)), _dev(gamma, torch.float32, "gamma", (1,)),
+        M, N, K, _dev(out, out.dtype, "out", (M, N)), kind, _opt(err_word, "err_word"), int(layout), int(path),
+        int(wait_limit_ns), int(stall_after_loads), _stream(stream)), "bitlinear_forward_stall_test")
 
 
 def bitlinear_forward_rowscale(xq, s, packed, gamma_rows, out, err_word=None, stream=None, path=BL_PATH_AUTO,

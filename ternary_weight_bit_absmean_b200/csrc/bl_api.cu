@@ -39,6 +39,12 @@ bl_status check_weight_shape(int64_t N, int64_t K) {
 namespace bl {
 void record_cuda_error(int code) { g_last_cuda_error = code; }
 
+namespace {
+thread_local WaitTest g_wait_test = {kDefaultWaitNs, -1};
+}  // namespace
+
+WaitTest wait_test() { return g_wait_test; }
+
 unsigned long long current_context_id() {
     // the driver functions come through the runtime's entry-point query, so the library
     // does not link the driver library; looked up once (thread-safe static init)
@@ -288,6 +294,25 @@ bl_status bitlinear_forward_rowscale(const int8_t* xq, const float* s, const uin
                                      int32_t* err_word, bl_xq_layout xq_layout, bl_path path, void* stream) {
     BL_RANGE("bitlinear_forward_rowscale");
     return forward_impl(xq, s, packed, gamma_rows, M, N, K, out, out_dtype, err_word, xq_layout, path, true, stream);
+}
+
+bl_status bitlinear_forward_stall_test(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                                      int64_t M, int64_t N, int64_t K, void* out, bl_dtype out_dtype,
+                                      int32_t* err_word, bl_xq_layout xq_layout, bl_path path, uint64_t wait_limit_ns,
+                                      int32_t stall_after_loads, void* stream) {
+    BL_RANGE("bitlinear_forward_stall_test");
+    if (wait_limit_ns == 0 || wait_limit_ns > bl::kDefaultWaitNs || stall_after_loads < 0) return BL_ERR_INVALID_ARG;
+    // only the kernels that wait on TMA loads: the single-SM tcgen05 kernel, the small-
+    // batch tcgen05 kernel, and the decode GEMV where it takes its TMA-fed form
+    if (path != BL_PATH_TC_1SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV) return BL_ERR_INVALID_ARG;
+    if (path == BL_PATH_GEMV && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
+        return BL_ERR_UNSUPPORTED_SHAPE;
+    const bl::WaitTest saved = bl::g_wait_test;
+    bl::g_wait_test = bl::WaitTest{wait_limit_ns, stall_after_loads};
+    const bl_status st =
+        forward_impl(xq, s, packed, gamma, M, N, K, out, out_dtype, err_word, xq_layout, path, false, stream);
+    bl::g_wait_test = saved;
+    return st;
 }
 
 bl_status bitlinear_forward_path(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,

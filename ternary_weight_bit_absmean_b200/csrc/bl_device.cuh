@@ -79,18 +79,29 @@ constexpr uint32_t kSuspendHintNs = 200000;  // 0.2 ms per suspended try_wait
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up after
 // kWaitTimeoutNs, or as soon as another role of the CTA has raised *abort; returns
 // false then (and raises *abort itself on a timeout).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                  unsigned long long limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
+    const uint32_t hint = limit_ns < kSuspendHintNs ? static_cast<uint32_t>(limit_ns) : kSuspendHintNs;
     for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+        if (mbar_try_wait_sleep(bar, parity, hint)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;
             return false;
         }
     }
+}
+
+// The stall of the bounded-wait test: a producer that has stopped issuing loads spins
+// here until another role of the block gives up waiting for them (raising *abort), or
+// for at most limit_ns, then raises *abort itself.
+__device__ __forceinline__ void stall_until_abort(volatile int* abort, unsigned long long limit_ns) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (!*abort && globaltimer_ns() - t0 <= limit_ns) {
+    }
+    *abort = 1;
 }
 
 // ------------------------------------------------ programmatic dependent launch --
@@ -279,9 +290,9 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // As mbar_wait_bounded, for barriers that also receive arrivals from the peer CTA.
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity,
-                                                          volatile int* abort) {
-    return mbar_wait_bounded(bar, parity, abort);
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                          unsigned long long limit_ns = kWaitTimeoutNs) {
+    return mbar_wait_bounded(bar, parity, abort, limit_ns);
 }
 
 __device__ __forceinline__ void cluster_sync_all() {

@@ -103,6 +103,19 @@ cudaError_t launch_ste_grad_weight(const float* dY, const int8_t* xq, const floa
 // Keep a CUDA error code for bitlinear_last_cuda_error() on the calling thread.
 void record_cuda_error(int code);
 
+// Limits of the device-side waits of the TMA-fed forward kernels, as the launchers copy
+// them into the kernel arguments.  Outside a call of bitlinear_forward_stall_test they
+// are {2 s, -1}: every wait gives up after 2 s, and producers never stall.  That test
+// entry point sets them on the calling thread for the duration of its call only: the
+// waits give up after wait_ns, and each block's producer stops issuing loads after
+// stall_after of them, so that the waits for the next load run out.
+struct WaitTest {
+    unsigned long long wait_ns;
+    int stall_after;
+};
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+WaitTest wait_test();
+
 // Identifier of the calling thread's current CUDA context, unique for the life of the
 // process (a context created after cudaDeviceReset gets a new one); 0 if unknown.
 unsigned long long current_context_id();

@@ -80,6 +80,8 @@ struct TcArgs {
     int32_t* err;
     S4Mul mul;
     int grow;  // gamma holds one scale per output row
+    unsigned long long wait_ns;  // limit of every wait (2 s outside the bounded-wait test)
+    int stall_after;             // the producer stops after this many loads (< 0: never)
 };
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -166,7 +168,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n0 = (tile % a.n_tiles_n) * kBN;
                 const int t0 = (tile / a.n_tiles_n) * BT;
                 for (int kt = 0; kt < nK; ++kt) {
-                    if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                    if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (issued == a.stall_after) {  // the bounded-wait test: stop issuing
+                        stall_until_abort(abort_flag, 4 * a.wait_ns);
                         ok = false;
                         break;
                     }
@@ -198,15 +205,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t bphase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
-                if (!mbar_wait_bounded(tempty(buf), bphase ^ 1u, abort_flag)) {
+                if (!mbar_wait_bounded(tempty(buf), bphase ^ 1u, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BT);
                 for (int kt = 0; kt < nK; ++kt) {
-                    if (!mbar_wait_bounded(full(stage), phase, abort_flag) ||
-                        !mbar_wait_bounded(afull(stage), phase, abort_flag)) {
+                    if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns) ||
+                        !mbar_wait_bounded(afull(stage), phase, abort_flag, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -249,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
             for (int kt = 0; kt < nK; ++kt) {
-                if (!mbar_wait_bounded(full(stage), phase, abort_flag)) {
+                if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // s of the first chunk's tokens is fetched before the accumulator is ready;
             // each chunk then fetches the next chunk's while it converts and stores
             float s_next = (a.kind != kOutI32 && t0 + first + lane < a.M) ? __ldg(a.s + t0 + first + lane) : 1.0f;
-            if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag)) break;
+            if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag, a.wait_ns)) break;
             tc_fence_after();
             const int row = n0 + 32 * q + lane;
             const bool row_ok = row < a.N;
@@ -457,8 +464,9 @@ cudaError_t launch_gemm_tc1(const int8_t* xq, const float* s, const uint8_t* pac
     const int64_t nN = (N + kBN - 1) / kBN;
     int64_t cost = 0;
     const int bt = tc1_tile(M, N, K, sms, &cost);
+    const WaitTest wt = wait_test();
     TcArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(nN),
-             0, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
+             0, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind), wt.wait_ns, wt.stall_after};
     a.num_tiles = static_cast<int>(nN * ((M + bt - 1) / bt));
     switch (layout) {
         case kXqEvenOdd16: return launch_bt_layout<kXqEvenOdd16>(bt, xq, packed, a, sms, stream);

@@ -92,6 +92,8 @@ struct GvArgs {
     int32_t* err;
     S4Mul mul;
     int grow;              // gamma holds one scale per output row
+    unsigned long long wait_ns;  // limit of every wait (2 s outside the bounded-wait test)
+    int stall_after;             // the producer stops after this many loads (< 0: never)
 };
 
 __device__ __forceinline__ void store_out(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -183,7 +185,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long issued = 0;
             bool ok = true;
             for (int kt = kt_begin; kt < kt_end; ++kt) {
-                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (issued == a.stall_after) {  // the bounded-wait test: stop issuing
+                    stall_until_abort(abort_flag, 4 * a.wait_ns);
                     ok = false;
                     break;
                 }
@@ -213,8 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int i = 0; i < nk; ++i) {
-                if (!mbar_wait_bounded(full(stage), phase, abort_flag) ||
-                    !mbar_wait_bounded(afull(stage), phase, abort_flag)) {
+                if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns) ||
+                    !mbar_wait_bounded(afull(stage), phase, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -248,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         for (int i = 0; i < nk; ++i) {
-            if (!mbar_wait_bounded(full(stage), phase, abort_flag)) break;
+            if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns)) break;
             const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + stage * kPBytes + r * (kBK / 4) +
                                                             16 * h);
             const uint32_t words[4] = {p.x, p.y, p.z, p.w};
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------- epilogue --
         // both warps of a lane quarter read half of the tokens each
         constexpr int kAccShift = LAY == kXqStride4K16 ? 6 : 0;
-        const bool got = mbar_wait_bounded(done_bar, 0, abort_flag);
+        const bool got = mbar_wait_bounded(done_bar, 0, abort_flag, a.wait_ns);
         tc_fence_after();
         const int row = n0 + r;
         const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
@@ -391,8 +398,10 @@ cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* pack
         !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kBK / 4, kRows,
                            false))
         return cudaErrorInvalidValue;
+    const WaitTest wt = wait_test();
     GvArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-             static_cast<int>(nstages / split), nstages, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
+             static_cast<int>(nstages / split), nstages, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind),
+             wt.wait_ns, wt.stall_after};
     const dim3 grid(static_cast<unsigned>(split), static_cast<unsigned>(row_tiles), static_cast<unsigned>(tok_tiles));
     switch (layout) {
         case kXqEvenOdd16: return launch_layout<kXqEvenOdd16>(bt, tx, tp, a, grid, stream);

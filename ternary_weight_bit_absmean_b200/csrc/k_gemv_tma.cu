@@ -63,6 +63,8 @@ struct GtArgs {
     int32_t* err;
     S4Mul mul;
     int grow;  // gamma holds one scale per output row
+    unsigned long long wait_ns;  // limit of every wait (2 s outside the bounded-wait test)
+    int stall_after;             // the producer stops after this many stages (< 0: never)
 };
 
 __device__ __forceinline__ void store_y1(void* out, int kind, int64_t idx, int acc, float fac) {
@@ -198,7 +200,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long issued = 0;
             bool ok = true;
             for (int kt = 0; kt < nstep; ++kt) {
-                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (issued == a.stall_after) {  // the bounded-wait test: stop issuing
+                    stall_until_abort(abort_flag, 4 * a.wait_ns);
                     ok = false;
                     break;
                 }
@@ -283,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // while the previous quarter computes
             uint4 b[4], bb[4];
             if (active && part < 4 * uk) load_x(4 * kt * U + part, b, bb);
-            if (active && !mbar_wait_bounded(full(stage, pair), phase, abort_flag)) break;
+            if (active && !mbar_wait_bounded(full(stage, pair), phase, abort_flag, a.wait_ns)) break;
             if (active) {
                 const uint8_t* sw = gbase + stage * stage_bytes;
                 for (int c = part; c < 4 * uk; c += R) {
@@ -436,8 +443,10 @@ cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* pac
     if (!encode_tmap_u8_2d(&tw, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), 256, 16, false))
         return cudaErrorInvalidValue;
     const int64_t ntiles = (N + 15) / 16;
+    const WaitTest wt = wait_test();
     GtArgs a{xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(ntiles),
-             p.stages, p.tile_slots, p.units, p.wpp, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind)};
+             p.stages, p.tile_slots, p.units, p.wpp, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind),
+             wt.wait_ns, wt.stall_after};
     static PerContextOnce attr[2];
     cudaError_t e = attr[MT - 1].run([MT] {
         return MT == 1 ? cudaFuncSetAttribute(gemv_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -861,3 +861,56 @@ def test_ste_backward_full_size_sampled(M, N, K):
     want = oracle.ste_grad_weight(np.ascontiguousarray(dY[:, rn]), xq, s, g)
     _assert_within_sum_bound(dW.cpu().numpy()[rn], want, np.abs(dY[:, rn].astype(np.float64)).T @ xs, M, g,
                              "dW rows", split_err=2.0 ** -16 + 2.0 ** -23, precise=True)
+
+
+# ------------------------------------------------------------ bounded device waits --
+
+@pytest.mark.parametrize("path,M,N,K,layout", [
+    (B.BL_PATH_TC_1SM, 256, 1024, 4096, B.BL_XQ_K16_STRIDE4),
+    (B.BL_PATH_TC_1SM, 300, 640, 2048, B.BL_XQ_ROWMAJOR),
+    (B.BL_PATH_SKINNY, 32, 1024, 4096, B.BL_XQ_K16_STRIDE4),
+    (B.BL_PATH_SKINNY, 64, 40000, 1024, B.BL_XQ_ROWMAJOR),
+    (B.BL_PATH_GEMV, 4, 4736, 32768, B.BL_XQ_K16_STRIDE4),
+], ids=["tc1-stride4", "tc1-rowmajor", "skinny-split", "skinny-nosplit", "gemv-tma"])
+def test_bounded_wait_runs_out_then_next_call_is_exact(path, M, N, K, layout):
+    """Each block's load producer stops after 3 loads and every wait is limited to 1 ms:
+    the waits for the fourth load run out, the kernel drains what is in flight, frees its
+    tensor memory and reports BL_ERRBIT_TIMEOUT.  The context stays usable: the next
+    normal call on the same stream matches the oracle bit for bit."""
+    g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=M + N + K)
+    pos = {B.BL_XQ_ROWMAJOR: np.arange(K), B.BL_XQ_K16_STRIDE4: stride4_positions(K)}[layout]
+    xl = np.empty_like(xq_ref)
+    xl[:, pos] = xq_ref
+    xq = torch.from_numpy(xl).to(DEV)
+    s = torch.from_numpy(s_ref).to(DEV)
+    packed = torch.from_numpy(packed_ref).to(DEV)
+    gamma = torch.tensor([g_ref], device=DEV)
+    out = guarded_empty((M, N), torch.int32)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.bitlinear_forward_stall_test(xq, s, packed, gamma, out, err, 1_000_000, 3, path=path, layout=layout)
+    sync()
+    check_guard(out)
+    assert err.item() & B.BL_ERRBIT_TIMEOUT
+    rows = np.unique(np.r_[0, M - 1, np.random.default_rng(M).integers(0, M, 4)])
+    acc_ref = oracle.forward(xq_ref[rows], s_ref[rows], packed_ref, g_ref, K, oracle.OUT_I32)
+    for _ in range(2):
+        err.zero_()
+        acc = B.forward(xq, s, packed, gamma, torch.int32, path=path, layout=layout, err_word=err)
+        sync()
+        assert err.item() == 0
+        assert np.array_equal(acc.cpu().numpy()[rows], acc_ref)
+
+
+def test_bounded_wait_test_rejects_other_paths_and_limits():
+    xq = torch.zeros(32, 256, dtype=torch.int8, device=DEV)
+    s = torch.ones(32, device=DEV)
+    packed = torch.zeros(256, 64, dtype=torch.uint8, device=DEV)
+    gamma = torch.ones(1, device=DEV)
+    out = torch.empty(32, 256, dtype=torch.int32, device=DEV)
+    for path, limit, stall in ((B.BL_PATH_TC_2SM, 1000, 1), (B.BL_PATH_TC_1SM, 0, 1), (B.BL_PATH_TC_1SM, 1000, -1),
+                               (B.BL_PATH_TC_1SM, 3_000_000_000, 1)):
+        with pytest.raises(B.BitLinearError, match="INVALID_ARG"):
+            B.bitlinear_forward_stall_test(xq, s, packed, gamma, out, None, limit, stall, path=path)
+    with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):  # no TMA-fed GEMV at this size
+        B.bitlinear_forward_stall_test(xq[:4], s[:4], packed, gamma, out[:4], None, 1000, 1, path=B.BL_PATH_GEMV,
+                                       layout=B.BL_XQ_K16_STRIDE4)
