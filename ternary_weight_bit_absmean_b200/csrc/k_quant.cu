@@ -265,7 +265,8 @@ __device__ __forceinline__ void store_unit(uint8_t* qrow, int idx, const Unit<U>
 // registers between the absmax pass and the quantise pass (longer rows are re-read for
 // the remainder).  Short rows (G = 32) give each warp R rows, whose loads are all issued
 // before the first reduction.  Needs K % (8 U) == 0.
-template <int G, int R, int L>
+// VPT is the number of 16-byte vectors a thread keeps (NV = VPT / U units).
+template <int G, int R, int L, int VPT>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     act_quant_vec_kernel(const uint4* __restrict__ X, int64_t M, int K, float eps,
                          uint8_t* __restrict__ xq, float* __restrict__ s_out) {
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G * R;  // rows per block
     constexpr int WPG = G / 32;       // warps per row group
-    constexpr int NV = ((R > 1) ? 4 : 8) / U;
+    constexpr int NV = VPT / U;
     static_assert(R == 1 || G == 32, "several rows per group only for warp groups");
     __shared__ uint32_t red[CTA / 32];
 
@@ -587,11 +588,11 @@ cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packe
                       reinterpret_cast<const uint4*>(codes), numel, packed, err);
 }
 
-template <int G, int R, int L>
+template <int G, int R, int L, int VPT = (R > 1 ? 4 : 8)>
 static cudaError_t launch_act_g(const uint4* X4, int64_t M, int K, float eps, uint8_t* xq, float* s,
                                 cudaStream_t stream) {
     constexpr int CTA = G > 256 ? G : 256;
-    return launch_pdl(act_quant_vec_kernel<G, R, L>, dim3(grid_for(M, CTA / G * R, 1 << 30)), dim3(CTA), 0, stream,
+    return launch_pdl(act_quant_vec_kernel<G, R, L, VPT>, dim3(grid_for(M, CTA / G * R, 1 << 30)), dim3(CTA), 0, stream,
                       dim3(kNoCluster), X4, M, K, eps, xq, s);
 }
 
@@ -601,8 +602,9 @@ static cudaError_t launch_act_vec(const uint4* X4, int64_t M, int K, float eps, 
     const int nvec = K / 8;
     if (nvec <= 32) return launch_act_g<32, 4, L>(X4, M, K, eps, xq, s, stream);
     if (nvec <= 128) return launch_act_g<32, 2, L>(X4, M, K, eps, xq, s, stream);
-    if (nvec <= 256) return launch_act_g<64, 1, L>(X4, M, K, eps, xq, s, stream);
-    if (nvec <= 512) return launch_act_g<128, 1, L>(X4, M, K, eps, xq, s, stream);
+    // rows up to 4096 elements: one warp per row holding the whole row (16 vectors per
+    // lane), so the reduction needs no block barrier and a block keeps 8 rows in flight
+    if (nvec <= 512) return launch_act_g<32, 1, L, 16>(X4, M, K, eps, xq, s, stream);
     if (nvec <= 1024) return launch_act_g<256, 1, L>(X4, M, K, eps, xq, s, stream);
     return launch_act_g<512, 1, L>(X4, M, K, eps, xq, s, stream);
 }
