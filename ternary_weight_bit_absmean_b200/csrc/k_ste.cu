@@ -252,6 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
         }
     } else if (warp < kWarpB) {
         // ------------------------------------------------------------ A producers --
+        // Every global load of a stage is issued before the wait for the stage to be
+        // free, so the load latency overlaps that wait; the conversion follows.
         const int t = threadIdx.x - 32 * kWarpA;  // 0 .. 127
         int stage = 0;
         uint32_t phase = 0;
@@ -260,35 +262,39 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
             const int i0 = (tile % a.tiles_i) * kBI;
             for (int kc = 0; kc < nC; ++kc) {
                 const int c0 = kc * kBC;
-                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* ahi = gbase + sAhi(stage);
-                uint8_t* alo = gbase + sAlo(stage);
                 if constexpr (KIND == kDX) {
-                    // A[m][n] = dY[m][n]: eight threads per row, each eight consecutive n
+                    // A[m][n] = dY[m][n]: eight threads per row, each eight consecutive n;
+                    // the 16 rows of a pass are 16 apart, eight passes per stage
                     const int r_off = t >> 3, ch = t & 7;
                     const int n = c0 + 8 * ch;
                     const bool vec = (a.N & 3) == 0 && n + 8 <= a.N;
-#pragma unroll 2
+                    float x[kBI / 16][8];
+#pragma unroll
                     for (int p = 0; p < kBI / 16; ++p) {
-                        const int r = 16 * p + r_off;
-                        const int m = i0 + r;
-                        float x[8];
+                        const int m = i0 + 16 * p + r_off;
                         if (m < a.M && vec) {
                             const float4* src = reinterpret_cast<const float4*>(a.dY + static_cast<int64_t>(m) * a.N + n);
                             const float4 u = __ldg(src), v = __ldg(src + 1);
-                            x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-                            x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+                            x[p][0] = u.x; x[p][1] = u.y; x[p][2] = u.z; x[p][3] = u.w;
+                            x[p][4] = v.x; x[p][5] = v.y; x[p][6] = v.z; x[p][7] = v.w;
                         } else {
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                x[e] = (m < a.M && n + e < a.N) ? __ldg(a.dY + static_cast<int64_t>(m) * a.N + n + e)
-                                                                : 0.0f;
+                                x[p][e] = (m < a.M && n + e < a.N) ? __ldg(a.dY + static_cast<int64_t>(m) * a.N + n + e)
+                                                                   : 0.0f;
                         }
+                    }
+                    if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* ahi = gbase + sAhi(stage);
+                    uint8_t* alo = gbase + sAlo(stage);
+#pragma unroll
+                    for (int p = 0; p < kBI / 16; ++p) {
+                        const int r = 16 * p + r_off;
                         uint4 hi, lo;
-                        split8(x, hi, lo);
+                        split8(x[p], hi, lo);
                         *reinterpret_cast<uint4*>(ahi + sw128(r, ch)) = hi;
                         *reinterpret_cast<uint4*>(alo + sw128(r, ch)) = lo;
                     }
@@ -301,20 +307,28 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
                     const float rB = mB < a.M ? __frcp_rn(__ldg(a.s + mB)) : 0.0f;
                     const int n = i0 + t;
                     const bool row_ok = n < a.N;
-#pragma unroll 1
-                    for (int ch = 0; ch < kBC / 8; ++ch) {
-                        const float rsrc = ch < 4 ? rA : rB;
-                        float x[8];
+                    float x[kBC];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int m = c0 + 8 * ch + e;
-                            const float rm = __shfl_sync(0xffffffffu, rsrc, (8 * ch + e) & 31);
-                            x[e] = (row_ok && m < a.M)
-                                       ? __fmul_rn(__ldg(a.dY + static_cast<int64_t>(m) * a.N + n), rm)
-                                       : 0.0f;
-                        }
+                    for (int e = 0; e < kBC; ++e) {
+                        const int m = c0 + e;
+                        x[e] = (row_ok && m < a.M) ? __ldg(a.dY + static_cast<int64_t>(m) * a.N + n) : 0.0f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < kBC; ++e)
+                        x[e] = __fmul_rn(x[e], __shfl_sync(0xffffffffu, e < 32 ? rA : rB, e & 31));
+                    if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* ahi = gbase + sAhi(stage);
+                    uint8_t* alo = gbase + sAlo(stage);
+#pragma unroll
+                    for (int ch = 0; ch < kBC / 8; ++ch) {
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = x[8 * ch + e];
                         uint4 hi, lo;
-                        split8(x, hi, lo);
+                        split8(y, hi, lo);
                         *reinterpret_cast<uint4*>(ahi + sw128(t, ch)) = hi;
                         *reinterpret_cast<uint4*>(alo + sw128(t, ch)) = lo;
                     }
@@ -330,7 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
         }
     } else if (warp < kWarpEpi) {
         // ------------------------------------------------------------ B producers --
+        // loads first, then the wait for the stage, then the conversion (as above)
         const int t = threadIdx.x - 32 * kWarpB;  // 0 .. 255
+        constexpr int kUnits = KIND == kDX ? (BJ / 8) * 8 : (BJ / 4) * 8;  // units per stage
+        constexpr int kPer = (kUnits + 32 * kBWarps - 1) / (32 * kBWarps);   // units per thread
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -338,40 +355,64 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
             const int j0 = (tile / a.tiles_i) * BJ;
             for (int kc = 0; kc < nC; ++kc) {
                 const int c0 = kc * kBC;
-                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* bt = gbase + sB(stage);
+                uint32_t w[kPer][8];
                 if constexpr (KIND == kDX) {
                     // B[k][n] = c[n][k]: a unit is 8 consecutive k (two packed bytes per n)
                     // x 8 consecutive n; the warp's lanes take consecutive k groups of one
                     // n chunk, so each load of a warp reads one packed row contiguously
                     const int KB = a.K >> 2;
-                    for (int u = t; u < (BJ / 8) * 8; u += 32 * kBWarps) {
+#pragma unroll
+                    for (int v = 0; v < kPer; ++v) {
+                        const int u = t + 32 * kBWarps * v;
                         const int kg = u % (BJ / 8), nch = u / (BJ / 8);
                         const int k = j0 + 8 * kg, n = c0 + 8 * nch;
-                        uint32_t w[8];  // bytes k/4 and k/4 + 1 of row n + q, in bits 0..15
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            w[q] = 0;
-                            if (n + q < a.N) {
+                            w[v][q] = 0;
+                            if (u < kUnits && n + q < a.N) {
                                 const uint8_t* row = a.packed + static_cast<int64_t>(n + q) * KB;
                                 if (k + 8 <= a.K && (KB & 1) == 0) {
-                                    w[q] = __ldg(reinterpret_cast<const uint16_t*>(row + (k >> 2)));
+                                    w[v][q] = __ldg(reinterpret_cast<const uint16_t*>(row + (k >> 2)));
                                 } else {
-                                    if (k < a.K) w[q] = __ldg(row + (k >> 2));
-                                    if (k + 4 < a.K) w[q] |= static_cast<uint32_t>(__ldg(row + (k >> 2) + 1)) << 8;
+                                    if (k < a.K) w[v][q] = __ldg(row + (k >> 2));
+                                    if (k + 4 < a.K) w[v][q] |= static_cast<uint32_t>(__ldg(row + (k >> 2) + 1)) << 8;
                                 }
                             }
                         }
+                    }
+                } else {
+                    // B[k][m] = x_q[m][k]: a unit is 4 consecutive k (one word per token) x 8
+                    // consecutive m; lanes take consecutive k words of one m chunk
+#pragma unroll
+                    for (int v = 0; v < kPer; ++v) {
+                        const int u = t + 32 * kBWarps * v;
+                        const int kw = u % (BJ / 4), mch = u / (BJ / 4);
+                        const int k = j0 + 4 * kw, m = c0 + 8 * mch;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            w[v][q] = (u < kUnits && m + q < a.M && k < a.K)
+                                          ? __ldg(reinterpret_cast<const uint32_t*>(a.xq + static_cast<int64_t>(m + q) * a.K + k))
+                                          : 0u;
+                    }
+                }
+                if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* bt = gbase + sB(stage);
+#pragma unroll
+                for (int v = 0; v < kPer; ++v) {
+                    const int u = t + 32 * kBWarps * v;
+                    if (u >= kUnits) continue;
+                    if constexpr (KIND == kDX) {
+                        const int kg = u % (BJ / 8), nch = u / (BJ / 8);
                         // gather byte b (k rows 4b .. 4b + 3) of n = q into byte q % 4 of
                         // g[b][q / 4]
                         uint32_t g[2][2];
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            const uint32_t t01 = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
-                            const uint32_t t23 = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
+                            const uint32_t t01 = __byte_perm(w[v][4 * h], w[v][4 * h + 1], 0x5140);
+                            const uint32_t t23 = __byte_perm(w[v][4 * h + 2], w[v][4 * h + 3], 0x5140);
                             g[0][h] = __byte_perm(t01, t23, 0x5410);
                             g[1][h] = __byte_perm(t01, t23, 0x7632);
                         }
@@ -383,26 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
                             codes4_to_bf16((g[b][1] >> sh) & 0x03030303u, o.z, o.w);
                             *reinterpret_cast<uint4*>(bt + sw128(8 * kg + kr, nch)) = o;
                         }
-                    }
-                } else {
-                    // B[k][m] = x_q[m][k]: a unit is 4 consecutive k (one word per token) x 8
-                    // consecutive m; lanes take consecutive k words of one m chunk
-                    for (int u = t; u < (BJ / 4) * 8; u += 32 * kBWarps) {
+                    } else {
                         const int kw = u % (BJ / 4), mch = u / (BJ / 4);
-                        const int k = j0 + 4 * kw, m = c0 + 8 * mch;
-                        uint32_t w[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            w[q] = (m + q < a.M && k < a.K)
-                                       ? __ldg(reinterpret_cast<const uint32_t*>(a.xq + static_cast<int64_t>(m + q) * a.K + k))
-                                       : 0u;
 #pragma unroll
                         for (int kr = 0; kr < 4; ++kr) {
                             uint4 o;
-                            o.x = bf16x2_of_s8(w[0] >> (8 * kr), w[1] >> (8 * kr));
-                            o.y = bf16x2_of_s8(w[2] >> (8 * kr), w[3] >> (8 * kr));
-                            o.z = bf16x2_of_s8(w[4] >> (8 * kr), w[5] >> (8 * kr));
-                            o.w = bf16x2_of_s8(w[6] >> (8 * kr), w[7] >> (8 * kr));
+                            o.x = bf16x2_of_s8(w[v][0] >> (8 * kr), w[v][1] >> (8 * kr));
+                            o.y = bf16x2_of_s8(w[v][2] >> (8 * kr), w[v][3] >> (8 * kr));
+                            o.z = bf16x2_of_s8(w[v][4] >> (8 * kr), w[v][5] >> (8 * kr));
+                            o.w = bf16x2_of_s8(w[v][6] >> (8 * kr), w[v][7] >> (8 * kr));
                             *reinterpret_cast<uint4*>(bt + sw128(4 * kw + kr, mch)) = o;
                         }
                     }
