@@ -20,10 +20,11 @@
 // K in stages of 128 codes.  Per stage:
 //   warp 0 (one lane)   TMA: packed weights [128 rows x 32 B] and the x_q tile
 //                       [BT x 128 B] (128-byte swizzle) on one mbarrier;
-//   warps 2-9           expanders, two per TMEM lane quarter: each thread owns one weight
-//                       row and half the stage (64 codes), unpacks them in registers in
-//                       the order of the x_q layout and stores 16 columns of tensor
-//                       memory; after tcgen05.wait::st one lane per warp arrives;
+//   warps 2-17          expanders, four groups of four warps (one per TMEM lane quarter);
+//                       group g takes every fourth stage: each thread owns one weight row,
+//                       unpacks its 128 codes in registers in the order of the x_q layout
+//                       and stores 32 columns of tensor memory; after tcgen05.wait::st one
+//                       lane per warp arrives;
 //   warp 1 (one lane)   MMA issuer: four tcgen05.mma kind::i8 (K = 32) per stage, A from
 //                       tensor memory, B (x_q) from shared memory; tcgen05.commit frees
 //                       the stage.
@@ -53,9 +54,10 @@ namespace {
 constexpr int kRows = 128;       // weight rows per tile (MMA M)
 constexpr int kBK = 128;         // K codes per stage
 constexpr int kPBytes = kRows * (kBK / 4);  // packed weights per stage: 4 KB
-constexpr int kStages = 6;
-constexpr int kThreads = 320;    // 10 warps
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2, kExpWarps = 8;
+constexpr int kStages = 10;
+constexpr int kThreads = 576;    // 18 warps
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2;
+constexpr int kExpGroups = 4;    // expander groups, each of 4 warps (one per TMEM lane quarter)
 constexpr int kMaxCluster = 8;
 constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s
 
@@ -65,17 +67,18 @@ struct GvCfg {
     static constexpr int kXBytes = BT * kBK;
     static constexpr int kStageBytes = kPBytes + kXBytes;
     static constexpr int kACols = kBK / 4;  // TMEM columns of one expanded stage
-    // accumulator (BT columns) after the expanded stages, allocated as a power of two
+    // accumulator (BT columns) after the expanded stages; one block per SM owns all 512
     static constexpr int kTmemUsed = kStages * kACols + BT;
-    static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kTmemCols = 512;
+    static_assert(kTmemUsed <= kTmemCols, "tensor memory");
     static constexpr int kRedBytes = BT * kRows * 4;  // partial sums, aliasing the stages
     static constexpr int kBarBytes = 8 * (3 * kStages + 2) + 16;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
-    // The request also caps the blocks per SM so that their tensor memory always fits
-    // (2 x 256 or 1 x 512 columns of the SM's 512): a block that waited in tcgen05.alloc
-    // for a block of its own cluster could never be served.  An SM has 228 KB of shared
-    // memory, each block 1 KB more than it asks for.
-    static constexpr int kSmemFloor = kTmemCols == 256 ? 80 * 1024 : 116 * 1024;
+    // The request also keeps a second block off the SM, so that the block's 512 columns
+    // of tensor memory are always free: a block that waited in tcgen05.alloc for a block
+    // of its own cluster could never be served.  An SM has 228 KB of shared memory, each
+    // block 1 KB more than it asks for.
+    static constexpr int kSmemFloor = 116 * 1024;
     static constexpr int kSmemLaunch = kSmemBytes > kSmemFloor ? kSmemBytes : kSmemFloor;
     static_assert(kRedBytes <= kStages * kStageBytes, "reduction buffer");
     static_assert(kSmemLaunch <= 227 * 1024, "shared memory");
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(afull(s), kExpWarps);
+            mbar_init(afull(s), 4);
             mbar_init(empty(s), 1);
         }
         mbar_init(done_bar, 1);
@@ -248,20 +251,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- expanders --
-        // thread: weight row r (its TMEM lane) and half h of each stage (64 codes)
-        const int q = warp & 3, h = (warp - kWarpExp) >> 2;
+        // Group g expands the stages of iterations g, g + 4, ...: its thread owns weight
+        // row r (its TMEM lane) and unpacks the row's 128 codes of the stage.  Four groups
+        // keep four stages in expansion at once, so the latency of one stage's tensor
+        // memory store (waited for before the MMA may read it) does not pace the stream.
+        const int q = warp & 3, grp = (warp - kWarpExp) >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int i = 0; i < nk; ++i) {
+        for (int i = grp; i < nk; i += kExpGroups) {
+            const int stage = i % ST;
+            const uint32_t phase = static_cast<uint32_t>((i / ST) & 1);
             if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns)) break;
-            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + stage * kPBytes + r * (kBK / 4) +
-                                                            16 * h);
-            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
-            uint32_t v[16];
+            const uint8_t* prow = gbase + (sP - base) + stage * kPBytes + r * (kBK / 4);
+            const uint4 p0 = *reinterpret_cast<const uint4*>(prow);
+            const uint4 p1 = *reinterpret_cast<const uint4*>(prow + 16);
+            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            uint32_t v[32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 // 16 codes -> 16 int8 in the order of the x_q layout (natural, even/odd,
                 // or stride-4 as 64 * code)
                 if constexpr (LAY == kXqEvenOdd16)
@@ -271,18 +278,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else
                     unpack16_natural(words[c], v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
             }
-            tmem_st_32x32b_x16(tmem_base + lane_addr + static_cast<uint32_t>(stage * C::kACols + 16 * h), v);
+            tmem_st_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(stage * C::kACols), v);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(afull(stage));
-            if (++stage == ST) {
-                stage = 0;
-                phase ^= 1u;
-            }
         }
         // ------------------------------------------------------------- epilogue --
-        // both warps of a lane quarter read half of the tokens each
+        // the four warps of a lane quarter read 16-token column chunks in turn
         constexpr int kAccShift = LAY == kXqStride4K16 ? 6 : 0;
         const bool got = mbar_wait_bounded(done_bar, 0, abort_flag, a.wait_ns);
         tc_fence_after();
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
         const float grow_gamma = (a.grow && a.kind != kOutI32 && row < a.N) ? __ldg(a.gamma + row) : 0.0f;
 #pragma unroll 1
-        for (int c0 = 16 * h; c0 < BT; c0 += 32) {
+        for (int c0 = 16 * grp; c0 < BT; c0 += 16 * kExpGroups) {
             uint32_t acc[16];
             tmem_ld_32x32b_x16(tmem_base + lane_addr + acc_col + static_cast<uint32_t>(c0), acc);
             tmem_ld_wait();
@@ -386,12 +389,19 @@ cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* pack
     const int64_t row_tiles = (N + kRows - 1) / kRows;
     const int64_t tok_tiles = (M + bt - 1) / bt;
     const int nstages = static_cast<int>((K + kBK - 1) / kBK);
-    // split K over a cluster until the blocks cover every SM twice (two blocks fit an SM),
-    // keeping at least two stages per block
-    int64_t split = (2 * sms + row_tiles * tok_tiles - 1) / (row_tiles * tok_tiles);
-    if (split > kMaxCluster) split = kMaxCluster;
-    if (split > nstages / 2) split = nstages / 2;
-    if (split < 1) split = 1;
+    // split K over a cluster of up to 8 blocks (one block per SM): the split with the
+    // fewest waves x stages per block, at least two stages per block (ties: fewer blocks)
+    const int64_t tiles = row_tiles * tok_tiles;
+    int64_t split = 1, best = -1;
+    for (int64_t sp = 1; sp <= kMaxCluster && (sp == 1 || sp <= nstages / 2); ++sp) {
+        const int64_t waves = (tiles * sp + sms - 1) / sms;
+        const int64_t per = nstages - (sp - 1) * (nstages / sp);  // the last block's stages
+        const int64_t cost = waves * per;
+        if (best < 0 || cost < best) {
+            best = cost;
+            split = sp;
+        }
+    }
     if (row_tiles > 65535 || tok_tiles > 65535) return cudaErrorInvalidValue;
     CUtensorMap tx, tp;
     if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, bt, true) ||
