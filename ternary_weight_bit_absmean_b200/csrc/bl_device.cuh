@@ -74,18 +74,30 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
     return ok != 0;
 }
 
-constexpr uint32_t kSuspendHintNs = 200000;  // 0.2 ms per suspended try_wait
+// How a blocked role waits: with a suspend-time hint (the hardware parks the warp until
+// the phase completes or the hint runs out), or with the plain try_wait, whose own
+// suspension the hardware bounds; the abort flag and the clock are read every
+// kWaitCheckEvery polls.
+#ifndef BL_WAIT_HINT_NS
+#define BL_WAIT_HINT_NS 200000
+#endif
+#ifndef BL_WAIT_CHECK_EVERY
+#define BL_WAIT_CHECK_EVERY 1
+#endif
+constexpr uint32_t kSuspendHintNs = BL_WAIT_HINT_NS;
+constexpr uint32_t kWaitCheckEvery = BL_WAIT_CHECK_EVERY;
 
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up after
-// kWaitTimeoutNs, or as soon as another role of the CTA has raised *abort; returns
-// false then (and raises *abort itself on a timeout).
+// limit_ns, or as soon as another role of the CTA has raised *abort; returns false then
+// (and raises *abort itself on a timeout).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   unsigned long long limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     const uint32_t hint = limit_ns < kSuspendHintNs ? static_cast<uint32_t>(limit_ns) : kSuspendHintNs;
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    for (uint32_t it = 1;; ++it) {
+        if (kSuspendHintNs > 0 ? mbar_try_wait_sleep(bar, parity, hint) : mbar_try_wait(bar, parity)) return true;
+        if (it % kWaitCheckEvery != 0) continue;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;

@@ -390,13 +390,14 @@ cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* pack
     const int64_t tok_tiles = (M + bt - 1) / bt;
     const int nstages = static_cast<int>((K + kBK - 1) / kBK);
     // split K over a cluster of up to 8 blocks (one block per SM): the split with the
-    // fewest waves x stages per block, at least two stages per block (ties: fewer blocks)
+    // fewest waves x (stages per block + a block's fixed cost, about 16 stages: start,
+    // pipeline fill and the reduction), at least two stages per block (ties: fewer blocks)
     const int64_t tiles = row_tiles * tok_tiles;
     int64_t split = 1, best = -1;
     for (int64_t sp = 1; sp <= kMaxCluster && (sp == 1 || sp <= nstages / 2); ++sp) {
         const int64_t waves = (tiles * sp + sms - 1) / sms;
         const int64_t per = nstages - (sp - 1) * (nstages / sp);  // the last block's stages
-        const int64_t cost = waves * per;
+        const int64_t cost = waves * (per + 16);
         if (best < 0 || cost < best) {
             best = cost;
             split = sp;
