@@ -44,8 +44,21 @@ __global__ void __launch_bounds__(kAbsThreads) absmean_partials_kernel(const flo
     pdl_wait_then_release();
     double acc = 0.0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kAbsThreads;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kAbsThreads + threadIdx.x; i < n4;
-         i += stride) {
+    int64_t i = static_cast<int64_t>(blockIdx.x) * kAbsThreads + threadIdx.x;
+    // four float4 loads in flight per thread, summed in the order of the plain loop
+    for (; i + 3 * stride < n4; i += 4 * stride) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(W4 + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc += static_cast<double>(fabsf(v[u].x));
+            acc += static_cast<double>(fabsf(v[u].y));
+            acc += static_cast<double>(fabsf(v[u].z));
+            acc += static_cast<double>(fabsf(v[u].w));
+        }
+    }
+    for (; i < n4; i += stride) {
         const float4 v = __ldg(W4 + i);
         acc += static_cast<double>(fabsf(v.x));
         acc += static_cast<double>(fabsf(v.y));
@@ -396,7 +409,8 @@ __device__ __forceinline__ int norm_w_chunk(int idx, int c) {
 
 extern __shared__ float4 norm_w_sm[];
 
-template <int G, int L, int KIND>
+// VPT is the number of 16-byte vectors a thread keeps in registers (NV = VPT / U units).
+template <int G, int L, int KIND, int VPT>
 __global__ void __launch_bounds__(G > 256 ? G : 256)
     norm_act_quant_kernel(const uint4* __restrict__ X, const float* __restrict__ nw, int64_t M, int K,
                           float norm_eps, float eps, uint8_t* __restrict__ xq, float* __restrict__ s_out,
@@ -408,7 +422,7 @@ __global__ void __launch_bounds__(G > 256 ? G : 256)
     constexpr int CTA = G > 256 ? G : 256;
     constexpr int RPC = CTA / G;  // rows per block
     constexpr int WPG = G / 32;   // warps per row group
-    constexpr int NV = 8 / U;     // units kept in registers
+    constexpr int NV = VPT / U;   // units kept in registers
     __shared__ double red_d[CTA / 32];
     __shared__ float red_f[CTA / 32];
 
@@ -609,7 +623,7 @@ static cudaError_t launch_act_vec(const uint4* X4, int64_t M, int K, float eps, 
     return launch_act_g<512, 1, L>(X4, M, K, eps, xq, s, stream);
 }
 
-template <int G, int L>
+template <int G, int L, int VPT = 8>
 static cudaError_t launch_norm_g(const uint4* X4, const float* nw, int64_t M, int K, int kind, float norm_eps,
                                  float eps, uint8_t* xq, float* s, cudaStream_t stream) {
     constexpr int CTA = G > 256 ? G : 256;
@@ -617,10 +631,10 @@ static cudaError_t launch_norm_g(const uint4* X4, const float* nw, int64_t M, in
     const int stage_w = nw != nullptr && K <= kNormStageMaxK ? 1 : 0;
     const size_t smem = stage_w ? static_cast<size_t>(K) * sizeof(float) : 0;
     if (kind == 1)
-        return launch_pdl(norm_act_quant_kernel<G, L, 1>, grid, block, smem, stream, dim3(kNoCluster), X4, nw, M,
-                          K, norm_eps, eps, xq, s, stage_w);
-    return launch_pdl(norm_act_quant_kernel<G, L, 0>, grid, block, smem, stream, dim3(kNoCluster), X4, nw, M, K,
-                      norm_eps, eps, xq, s, stage_w);
+        return launch_pdl(norm_act_quant_kernel<G, L, 1, VPT>, grid, block, smem, stream, dim3(kNoCluster), X4, nw,
+                          M, K, norm_eps, eps, xq, s, stage_w);
+    return launch_pdl(norm_act_quant_kernel<G, L, 0, VPT>, grid, block, smem, stream, dim3(kNoCluster), X4, nw, M,
+                      K, norm_eps, eps, xq, s, stage_w);
 }
 
 template <int L>
@@ -628,7 +642,8 @@ static cudaError_t launch_norm_l(const uint4* X4, const float* nw, int64_t M, in
                                  float eps, uint8_t* xq, float* s, cudaStream_t stream) {
     const int nvec = K / 8;  // 16-byte vectors per row; a thread holds 8 of them
     if (nvec <= 8 * 32) return launch_norm_g<32, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
-    if (nvec <= 8 * 64) return launch_norm_g<64, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
+    // rows up to 4096 elements: one warp per row holding all of it, no block barriers
+    if (nvec <= 16 * 32) return launch_norm_g<32, L, 16>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
     if (nvec <= 8 * 128) return launch_norm_g<128, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
     if (nvec <= 8 * 256) return launch_norm_g<256, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
     return launch_norm_g<512, L>(X4, nw, M, K, kind, norm_eps, eps, xq, s, stream);
