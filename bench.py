@@ -79,7 +79,7 @@ def parse():
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
     p.add_argument("--K", type=int, default=4096)
-    p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2", "skinny", "tm"], default="auto")
+    p.add_argument("--path", choices=["auto", "gemv", "tc", "tc1", "tc2", "skinny"], default="auto")
     p.add_argument("--out-dtype", choices=["f32", "bf16", "i32"], default="bf16")
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--step-streams", choices=["branches", "serial"], default="branches",
@@ -663,8 +663,7 @@ def run_single(args):
         odt = {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32}[args.out_dtype]
         out = torch.empty(M, N, dtype=odt, device=dev)
         path = {"auto": B.BL_PATH_AUTO, "gemv": B.BL_PATH_GEMV, "tc": B.BL_PATH_TC, "tc1": B.BL_PATH_TC_1SM,
-                "tc2": B.BL_PATH_TC_2SM, "skinny": B.BL_PATH_SKINNY,
-                "tm": B.BL_PATH_TC_TMEM}[args.path]
+                "tc2": B.BL_PATH_TC_2SM, "skinny": B.BL_PATH_SKINNY}[args.path]
         lay = xq_layout_of(B, args.xq_layout)
         fn = lambda: B.bitlinear_forward(xq, s, packed, gamma, out, path=path, layout=lay)
         ops = 2 * M * N * K

@@ -84,10 +84,8 @@ typedef enum {
     BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
     BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
     BL_PATH_TC_2SM = 4, /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
-    BL_PATH_SKINNY = 5, /* the tcgen05 small-batch kernel (expanded weights in tensor memory,
-                           K split over a cluster when rows are few); K % 64 == 0 */
-    BL_PATH_TC_TMEM = 6 /* the tiled tcgen05 kernel with the expanded weights in tensor
-                           memory (one SM per tile); K % 64 == 0 */
+    BL_PATH_SKINNY = 5  /* the tcgen05 small-batch kernel (K split over a cluster when rows
+                           are few); K % 64 == 0 */
 } bl_path;
 
 /* Storage order of x_q within each row.
@@ -221,7 +219,7 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
 
 /* A test of the bounded device waits (the source pages have no counterpart): the forward
  * of bitlinear_forward_layout on one of the kernels that wait for TMA loads
- * (BL_PATH_TC_1SM, BL_PATH_TC_TMEM, BL_PATH_SKINNY, or BL_PATH_GEMV where it runs its TMA-fed form:
+ * (BL_PATH_TC_1SM, BL_PATH_SKINNY, or BL_PATH_GEMV where it runs its TMA-fed form:
  * x_q in BL_XQ_K16_STRIDE4 and a layer wide enough), in which every wait gives up after
  * wait_limit_ns (0 < wait_limit_ns <= 2 s; the forward entry points use 2 s) and the
  * load producer of each block stops after stall_after_loads loads.  The waits for the

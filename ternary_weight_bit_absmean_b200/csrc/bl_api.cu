@@ -171,7 +171,7 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32)
         return BL_ERR_INVALID_ARG;
     if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
-        path != BL_PATH_TC_2SM && path != BL_PATH_SKINNY && path != BL_PATH_TC_TMEM)
+        path != BL_PATH_TC_2SM && path != BL_PATH_SKINNY)
         return BL_ERR_INVALID_ARG;
     if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD && xq_layout != BL_XQ_K16_STRIDE4)
         return BL_ERR_INVALID_ARG;
@@ -182,8 +182,7 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return BL_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(xq) || !aligned16(s) || !aligned16(packed) || !aligned16(out)) return BL_ERR_MISALIGNED;
     const bool k64 = (K % 64) == 0;
-    const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM || path == BL_PATH_SKINNY ||
-                    path == BL_PATH_TC_TMEM;
+    const bool tc = path == BL_PATH_TC || path == BL_PATH_TC_1SM || path == BL_PATH_TC_2SM || path == BL_PATH_SKINNY;
     if (tc && !k64) return BL_ERR_UNSUPPORTED_SHAPE;
     // the tensor-core kernels expand stride-4 codes as 64 * code: 64 * 128 * K must fit
     const bool s4_big = xq_layout == BL_XQ_K16_STRIDE4 && K > (int64_t(1) << 17);
@@ -203,8 +202,6 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
         e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (path == BL_PATH_SKINNY) {
         e = bl::launch_gemv_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
-    } else if (path == BL_PATH_TC_TMEM) {
-        e = bl::launch_gemm_tm(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (k64 && M <= int64_t(65535) * 16) {
         e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else {
@@ -307,8 +304,7 @@ bl_status bitlinear_forward_stall_test(const int8_t* xq, const float* s, const u
     if (wait_limit_ns == 0 || wait_limit_ns > bl::kDefaultWaitNs || stall_after_loads < 0) return BL_ERR_INVALID_ARG;
     // only the kernels that wait on TMA loads: the single-SM tcgen05 kernel, the small-
     // batch tcgen05 kernel, and the decode GEMV where it takes its TMA-fed form
-    if (path != BL_PATH_TC_1SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV && path != BL_PATH_TC_TMEM)
-        return BL_ERR_INVALID_ARG;
+    if (path != BL_PATH_TC_1SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV) return BL_ERR_INVALID_ARG;
     if (path == BL_PATH_GEMV && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
         return BL_ERR_UNSUPPORTED_SHAPE;
     const bl::WaitTest saved = bl::g_wait_test;

@@ -81,14 +81,9 @@ cudaError_t launch_gemm_tc2(const int8_t* xq, const float* s, const uint8_t* pac
                             const float* gamma, int64_t M, int64_t N, int64_t K, void* out,
                             int kind, int32_t* err, int layout, cudaStream_t stream);
 
-// Small-batch tcgen05 kernel (expanded weights in tensor memory, K split over a cluster
-// when rows are few), K % 64 == 0, any M (token tiles of up to 128).
+// Small-batch tcgen05 kernel (K split over a cluster when rows are few), K % 64 == 0, any
+// M (token tiles of up to 128).
 cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma, int64_t M,
-                           int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout, cudaStream_t stream);
-
-// Tiled tcgen05 kernel with the expanded weights in tensor memory (persistent, one SM per
-// tile), K % 64 == 0.
-cudaError_t launch_gemm_tm(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma, int64_t M,
                            int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout, cudaStream_t stream);
 
 // The 1.6-bit (five codes per byte) weight format, K % 16 == 0 (k_tl5.cu).

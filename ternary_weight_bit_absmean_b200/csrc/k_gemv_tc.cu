@@ -1,41 +1,37 @@
 // k_gemv_tc.cu -- BitLinear forward for small and middling token counts (decode and small
-// batches, up to 128 tokens) on the tcgen05 tensor cores, with the expanded weights kept
-// in tensor memory.
+// batches, up to 128 tokens) on the tcgen05 tensor cores, with K split over a
+// thread-block cluster so that a layer with few 128-row tiles still fills the GPU.
 //
 // What is computed ("What 1.58 Bits Actually Changes", "How the low-bit linear path
 // works": +1 adds, -1 subtracts, 0 skips; "1-bit & Ternary LLMs", block "BitNet (Oct
 // 2023)": one float rescale at the end):
 //   acc[m, n] = sum_k x_q[m, k] * c[n, k],   y[m, n] = acc[m, n] * gamma / s[m].
 //
-// Why this shape of kernel.  With few tokens the work per weight byte is small and the
-// path is bound by streaming the packed weights from HBM; each SM has to turn about 22
-// packed bytes (88 codes) per cycle into tensor-core operands.  Expanding the codes into
-// shared memory (the prefill kernels) costs two shared-memory passes per expanded byte,
-// which caps the rate near half of that.  Here the expanded int8 codes go straight from
-// registers into tensor memory (tcgen05.st), and the MMA reads its A operand from there
-// (tcgen05.mma ... [a_tmem]), so shared memory carries only the packed weights and the
-// activation tile, each written once by TMA and read once.
+// With few tokens the path is bound by streaming the packed weights: per 128-code stage
+// of a 128-row tile, 4 KB of packed codes are expanded into 16 KB of int8 A operand.
+// The expansion goes through shared memory in the 128-byte-swizzled K-major layout the
+// MMA descriptor reads (as in the prefill kernels); keeping the expanded codes in tensor
+// memory instead (tcgen05.st, A operand from TMEM) was built and measured slower here:
+// the tensor-memory stores of 16 KB per stage capped the stream near 1.2 TB/s.
 //
 // Tile: 128 weight rows (MMA M, TMEM lanes) x BT tokens (MMA N; 16 to 128) x a slice of
 // K in stages of 128 codes.  Per stage:
 //   warp 0 (one lane)   TMA: packed weights [128 rows x 32 B] and the x_q tile
 //                       [BT x 128 B] (128-byte swizzle) on one mbarrier;
-//   warps 2-17          expanders, four groups of four warps (one per TMEM lane quarter);
-//                       group g takes every fourth stage: each thread owns one weight row,
-//                       unpacks its 128 codes in registers in the order of the x_q layout
-//                       and stores 32 columns of tensor memory; after tcgen05.wait::st one
-//                       lane per warp arrives;
-//   warp 1 (one lane)   MMA issuer: four tcgen05.mma kind::i8 (K = 32) per stage, A from
-//                       tensor memory, B (x_q) from shared memory; tcgen05.commit frees
-//                       the stage.
+//   warps 2-17          expanders, two groups of eight warps taking alternate stages: two
+//                       threads per weight row, each unpacking 64 codes in the order of
+//                       the x_q layout into the swizzled A tile; fence.proxy.async, then
+//                       one lane per warp arrives;
+//   warp 1 (one lane)   MMA issuer: four tcgen05.mma kind::i8 (K = 32) per stage into the
+//                       TMEM accumulator; tcgen05.commit frees the stage.
 // After the last stage the expander warps read the int32 accumulator back (one weight
-// row per thread).  When rows are few (N / 128 tiles leave SMs idle), K is split over the
-// blocks of a thread-block cluster: each block writes its partial sums to its shared
-// memory and the blocks add them through distributed shared memory, each finishing a
-// share of the tokens.  Integer sums are exact, so the split changes nothing.  Rows and
-// tokens past the edges read the TMA's zero fill and are not stored.  Every wait is
-// bounded; a block that gives up drains its copies and MMAs, sets BL_ERRBIT_TIMEOUT and
-// still takes part in the cluster barriers, so no block waits forever.
+// row per thread).  When rows are few, K is split over the blocks of a cluster: each
+// block writes its partial sums to its shared memory and the blocks add them through
+// distributed shared memory, each finishing a share of the tokens.  Integer sums are
+// exact, so the split changes nothing.  Rows and tokens past the edges read the TMA's
+// zero fill and are not stored.  Every wait is bounded; a block that gives up drains its
+// copies and MMAs, sets BL_ERRBIT_TIMEOUT and still takes part in the cluster barriers,
+// so no block waits forever.
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cuda.h>
@@ -54,10 +50,10 @@ namespace {
 constexpr int kRows = 128;       // weight rows per tile (MMA M)
 constexpr int kBK = 128;         // K codes per stage
 constexpr int kPBytes = kRows * (kBK / 4);  // packed weights per stage: 4 KB
-constexpr int kStages = 10;
+constexpr int kABytes = kRows * kBK;        // expanded weights per stage: 16 KB
 constexpr int kThreads = 576;    // 18 warps
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2;
-constexpr int kExpGroups = 4;    // expander groups, each of 4 warps (one per TMEM lane quarter)
+constexpr int kExpGroups = 2;    // expander groups of eight warps, alternate stages
 constexpr int kMaxCluster = 8;
 constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s
 
@@ -65,23 +61,17 @@ template <int BT>
 struct GvCfg {
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 128, "token tile");
     static constexpr int kXBytes = BT * kBK;
-    static constexpr int kStageBytes = kPBytes + kXBytes;
-    static constexpr int kACols = kBK / 4;  // TMEM columns of one expanded stage
-    // accumulator (BT columns) after the expanded stages; one block per SM owns all 512
-    static constexpr int kTmemUsed = kStages * kACols + BT;
-    static constexpr int kTmemCols = 512;
-    static_assert(kTmemUsed <= kTmemCols, "tensor memory");
-    static constexpr int kRedBytes = BT * kRows * 4;  // partial sums, aliasing the stages
+    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes;
+    static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+    static constexpr int kTmemCols = BT <= 32 ? 32 : BT;  // the accumulator (a power of two >= 32)
+    static constexpr int kRedBytes = BT * kRows * 4;      // partial sums, aliasing the stages
     static constexpr int kBarBytes = 8 * (3 * kStages + 2) + 16;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
-    // The request also keeps a second block off the SM, so that the block's 512 columns
-    // of tensor memory are always free: a block that waited in tcgen05.alloc for a block
-    // of its own cluster could never be served.  An SM has 228 KB of shared memory, each
-    // block 1 KB more than it asks for.
-    static constexpr int kSmemFloor = 116 * 1024;
-    static constexpr int kSmemLaunch = kSmemBytes > kSmemFloor ? kSmemBytes : kSmemFloor;
+    static_assert(kStages >= 4, "stages");
+    static_assert(BT != 48 && BT != 80 && BT != 96 && BT != 112, "power-of-two token tiles");
     static_assert(kRedBytes <= kStages * kStageBytes, "reduction buffer");
-    static_assert(kSmemLaunch <= 227 * 1024, "shared memory");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 struct GvArgs {
@@ -131,13 +121,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_p,
                    const GvArgs a) {
     using C = GvCfg<BT>;
-    constexpr int ST = kStages;
+    constexpr int ST = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
-    const uint32_t sX = base;                       // x tiles first: 1024-aligned for the swizzle
-    const uint32_t sP = sX + ST * C::kXBytes;
+    const uint32_t sX = base;  // swizzled tiles first: 1024-aligned
+    const uint32_t sA = sX + ST * C::kXBytes;
+    const uint32_t sP = sA + ST * kABytes;
     const uint32_t sBar = sP + ST * kPBytes;
     auto full = [&](int s) { return sBar + 8u * s; };
     auto afull = [&](int s) { return sBar + 8u * (ST + s); };
@@ -159,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(afull(s), 4);
+            mbar_init(afull(s), 8);
             mbar_init(empty(s), 1);
         }
         mbar_init(done_bar, 1);
@@ -178,7 +169,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const uint32_t acc_col = static_cast<uint32_t>(ST * C::kACols);
 
     if (warp == kWarpTma) {
         if (lane == 0) {
@@ -218,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // ---------------------------------------------------------- MMA issuer --
             constexpr uint32_t idesc = idesc_i8(kRows, BT);
-            const uint32_t d_tmem = tmem_base + acc_col;
+            const uint32_t d_tmem = tmem_base;
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -229,12 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_tmem = tmem_base + static_cast<uint32_t>(stage * C::kACols);
+                const uint32_t a_addr = sA + stage * kABytes;
                 const uint32_t b_addr = sX + stage * C::kXBytes;
 #pragma unroll
                 for (int kk = 0; kk < kBK / 32; ++kk)
-                    tc_mma_i8_tmem_a(d_tmem, a_tmem + 8 * kk, smem_desc_sw128(b_addr + 32 * kk), idesc,
-                                     (i | kk) != 0 ? 1u : 0u);
+                    tc_mma_i8(d_tmem, smem_desc_sw128(a_addr + 32 * kk), smem_desc_sw128(b_addr + 32 * kk), idesc,
+                              (i | kk) != 0 ? 1u : 0u);
                 tc_commit(empty(stage));
                 if (++stage == ST) {
                     stage = 0;
@@ -251,51 +241,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------- expanders --
-        // Group g expands the stages of iterations g, g + 4, ...: its thread owns weight
-        // row r (its TMEM lane) and unpacks the row's 128 codes of the stage.  Four groups
-        // keep four stages in expansion at once, so the latency of one stage's tensor
-        // memory store (waited for before the MMA may read it) does not pace the stream.
-        const int q = warp & 3, grp = (warp - kWarpExp) >> 2;
-        const int r = 32 * q + lane;
-        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        // Group g (eight warps) expands the stages of iterations g, g + 2, ...: thread e
+        // of the group owns half `half` (64 codes, 16 packed bytes) of weight row `erow`;
+        // neighbouring lanes read neighbouring 16-byte pieces and write neighbouring
+        // swizzled chunks, free of bank conflicts.
+        const int grp = (warp - kWarpExp) >> 3;
+        const int e = threadIdx.x - 32 * kWarpExp - 256 * grp;  // 0 .. 255
+        const int erow = e >> 1, half = e & 1;
+        const uint32_t sw = static_cast<uint32_t>(erow & 7);
         for (int i = grp; i < nk; i += kExpGroups) {
             const int stage = i % ST;
             const uint32_t phase = static_cast<uint32_t>((i / ST) & 1);
             if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns)) break;
-            const uint8_t* prow = gbase + (sP - base) + stage * kPBytes + r * (kBK / 4);
-            const uint4 p0 = *reinterpret_cast<const uint4*>(prow);
-            const uint4 p1 = *reinterpret_cast<const uint4*>(prow + 16);
-            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            uint32_t v[32];
+            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + stage * kPBytes + erow * (kBK / 4) +
+                                                            16 * half);
+            uint8_t* ap = gbase + (sA - base) + stage * kABytes + erow * kBK;
+            const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 // 16 codes -> 16 int8 in the order of the x_q layout (natural, even/odd,
                 // or stride-4 as 64 * code)
+                uint4 u;
                 if constexpr (LAY == kXqEvenOdd16)
-                    unpack16_evenodd(words[c], v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    unpack16_evenodd(words[c], u.x, u.y, u.z, u.w);
                 else if constexpr (LAY == kXqStride4K16)
-                    unpack16_stride4_x64(words[c], a.mul, v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    unpack16_stride4_x64(words[c], a.mul, u.x, u.y, u.z, u.w);
                 else
-                    unpack16_natural(words[c], v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    unpack16_natural(words[c], u.x, u.y, u.z, u.w);
+                const uint32_t chunk = static_cast<uint32_t>(4 * half + c);
+                *reinterpret_cast<uint4*>(ap + ((chunk ^ sw) << 4)) = u;
             }
-            tmem_st_32x32b_x32(tmem_base + lane_addr + static_cast<uint32_t>(stage * C::kACols), v);
-            tmem_st_wait();
-            tc_fence_before();
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(afull(stage));
         }
         // ------------------------------------------------------------- epilogue --
-        // the four warps of a lane quarter read 16-token column chunks in turn
+        // the four warps of a lane quarter read 16-token column chunks in turn; thread:
+        // weight row r of the tile (its TMEM lane)
         constexpr int kAccShift = LAY == kXqStride4K16 ? 6 : 0;
+        const int q = warp & 3, eg = (warp - kWarpExp) >> 2;  // lane quarter, its warp index 0..3
+        const int r = 32 * q + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
         const bool got = mbar_wait_bounded(done_bar, 0, abort_flag, a.wait_ns);
         tc_fence_after();
         const int row = n0 + r;
         const float gamma = (a.kind == kOutI32) ? 0.0f : *a.gamma;
         const float grow_gamma = (a.grow && a.kind != kOutI32 && row < a.N) ? __ldg(a.gamma + row) : 0.0f;
 #pragma unroll 1
-        for (int c0 = 16 * grp; c0 < BT; c0 += 16 * kExpGroups) {
+        for (int c0 = 16 * eg; c0 < BT; c0 += 64) {
             uint32_t acc[16];
-            tmem_ld_32x32b_x16(tmem_base + lane_addr + acc_col + static_cast<uint32_t>(c0), acc);
+            tmem_ld_32x32b_x16(tmem_base + lane_addr + static_cast<uint32_t>(c0), acc);
             tmem_ld_wait();
             if (!got) continue;
 #pragma unroll
@@ -358,10 +353,10 @@ cudaError_t launch_bt(const CUtensorMap& tx, const CUtensorMap& tp, const GvArgs
     static PerContextOnce attr;
     cudaError_t e = attr.run([] {
         return cudaFuncSetAttribute(gemv_tc_kernel<BT, LAY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemLaunch);
+                                    C::kSmemBytes);
     });
     if (e != cudaSuccess) return e;
-    return launch_pdl(gemv_tc_kernel<BT, LAY>, grid, dim3(kThreads), C::kSmemLaunch, stream,
+    return launch_pdl(gemv_tc_kernel<BT, LAY>, grid, dim3(kThreads), C::kSmemBytes, stream,
                       grid.x > 1 ? dim3(grid.x, 1, 1) : dim3(kNoCluster), tx, tp, a);
 }
 
