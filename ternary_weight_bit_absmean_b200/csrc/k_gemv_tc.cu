@@ -49,8 +49,13 @@ namespace {
 
 constexpr int kRows = 128;       // weight rows per tile (MMA M)
 constexpr int kBK = 128;         // K codes per stage
-constexpr int kPBytes = kRows * (kBK / 4);  // packed weights per stage: 4 KB
 constexpr int kABytes = kRows * kBK;        // expanded weights per stage: 16 KB
+// The packed weights come in super-tiles of 8 stages: 128 rows x 256 bytes per TMA box,
+// so every row is read in 256-byte runs (a 32-byte box per row and stage reads DRAM in
+// short scattered pieces), into a ring of two slots.
+constexpr int kSuper = 8;
+constexpr int kPSBytes = kRows * (kSuper * kBK / 4);  // 32 KB
+constexpr int kPS = 2;
 constexpr int kThreads = 576;    // 18 warps
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpExp = 2;
 constexpr int kExpGroups = 2;    // expander groups of eight warps, alternate stages
@@ -61,16 +66,16 @@ template <int BT>
 struct GvCfg {
     static_assert(BT % 16 == 0 && BT >= 16 && BT <= 128, "token tile");
     static constexpr int kXBytes = BT * kBK;
-    static constexpr int kStageBytes = kXBytes + kABytes + kPBytes;
-    static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+    static constexpr int kStageBytes = kXBytes + kABytes;
+    static constexpr int kStagesRaw = (200 * 1024 - kPS * kPSBytes) / kStageBytes;
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kTmemCols = BT <= 32 ? 32 : BT;  // the accumulator (a power of two >= 32)
     static constexpr int kRedBytes = BT * kRows * 4;      // partial sums, aliasing the stages
-    static constexpr int kBarBytes = 8 * (3 * kStages + 2) + 16;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
+    static constexpr int kBarBytes = 8 * (3 * kStages + 2 * kPS + 2) + 16;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kPS * kPSBytes + kBarBytes;
     static_assert(kStages >= 4, "stages");
     static_assert(BT != 48 && BT != 80 && BT != 96 && BT != 112, "power-of-two token tiles");
-    static_assert(kRedBytes <= kStages * kStageBytes, "reduction buffer");
+    static_assert(kRedBytes <= kStages * kStageBytes + kPS * kPSBytes, "reduction buffer");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -129,13 +134,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sX = base;  // swizzled tiles first: 1024-aligned
     const uint32_t sA = sX + ST * C::kXBytes;
     const uint32_t sP = sA + ST * kABytes;
-    const uint32_t sBar = sP + ST * kPBytes;
-    auto full = [&](int s) { return sBar + 8u * s; };
-    auto afull = [&](int s) { return sBar + 8u * (ST + s); };
-    auto empty = [&](int s) { return sBar + 8u * (2 * ST + s); };
-    const uint32_t done_bar = sBar + 8u * (3 * ST);
-    const uint32_t drain_bar = sBar + 8u * (3 * ST + 1);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (sBar - base) + 8 * (3 * ST + 2));
+    const uint32_t sBar = sP + kPS * kPSBytes;
+    auto full = [&](int s) { return sBar + 8u * s; };                // x tile landed
+    auto afull = [&](int s) { return sBar + 8u * (ST + s); };        // A tile expanded
+    auto empty = [&](int s) { return sBar + 8u * (2 * ST + s); };    // stage read by the MMA
+    auto pfull = [&](int p) { return sBar + 8u * (3 * ST + p); };    // packed super-tile landed
+    auto pempty = [&](int p) { return sBar + 8u * (3 * ST + kPS + p); };  // super-tile expanded
+    const uint32_t done_bar = sBar + 8u * (3 * ST + 2 * kPS);
+    const uint32_t drain_bar = sBar + 8u * (3 * ST + 2 * kPS + 1);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (sBar - base) + 8 * (3 * ST + 2 * kPS + 2));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* red = reinterpret_cast<int*>(gbase);  // [BT][128] partial sums, after the main loop
 
@@ -152,6 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full(s), 1);
             mbar_init(afull(s), 8);
             mbar_init(empty(s), 1);
+        }
+        for (int p = 0; p < kPS; ++p) {
+            mbar_init(pfull(p), 1);
+            mbar_init(pempty(p), 8 * kExpGroups);
         }
         mbar_init(done_bar, 1);
         mbar_init(drain_bar, 1);
@@ -175,9 +186,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ------------------------------------------------------------ producer --
             int stage = 0;
             uint32_t phase = 0;
-            long long issued = 0;
+            long long issued = 0, issued_p = 0;
             bool ok = true;
-            for (int kt = kt_begin; kt < kt_end; ++kt) {
+            for (int i = 0; i < nk; ++i) {
+                const int kt = kt_begin + i;
+                if (i % kSuper == 0) {  // the next packed super-tile
+                    const int j = i / kSuper, p = j % kPS;
+                    if (!mbar_wait_bounded(pempty(p), static_cast<uint32_t>(((j / kPS) & 1) ^ 1), abort_flag,
+                                           a.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(pfull(p), kPSBytes);
+                    tma_load_2d(sP + p * kPSBytes, &tmap_p, pfull(p), kt * (kBK / 4), n0);
+                    ++issued_p;
+                }
                 if (!mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
@@ -187,9 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(full(stage), C::kXBytes + kPBytes);
+                mbar_arrive_expect_tx(full(stage), C::kXBytes);
                 tma_load_2d(sX + stage * C::kXBytes, &tmap_x, full(stage), kt * kBK, t0);
-                tma_load_2d(sP + stage * kPBytes, &tmap_p, full(stage), kt * (kBK / 4), n0);
                 ++issued;
                 if (++stage == ST) {
                     stage = 0;
@@ -198,9 +220,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) {
                 // wait for every load still in flight before the block may go on
-                for (int s = 0; s < ST; ++s) {
-                    const long long fills = (issued - s + ST - 1) / ST;
-                    if (fills > 0) drain_wait(full(s), static_cast<uint32_t>((fills - 1) & 1));
+                for (int q = 0; q < ST; ++q) {
+                    const long long fills = (issued - q + ST - 1) / ST;
+                    if (fills > 0) drain_wait(full(q), static_cast<uint32_t>((fills - 1) & 1));
+                }
+                for (int q = 0; q < kPS; ++q) {
+                    const long long fills = (issued_p - q + kPS - 1) / kPS;
+                    if (fills > 0) drain_wait(pfull(q), static_cast<uint32_t>((fills - 1) & 1));
                 }
             }
         }
@@ -252,8 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = grp; i < nk; i += kExpGroups) {
             const int stage = i % ST;
             const uint32_t phase = static_cast<uint32_t>((i / ST) & 1);
-            if (!mbar_wait_bounded(full(stage), phase, abort_flag, a.wait_ns)) break;
-            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + stage * kPBytes + erow * (kBK / 4) +
+            const int j = i / kSuper, pslot = j % kPS;
+            // the packed super-tile has landed, and the MMA is done with this stage's A tile
+            if (!mbar_wait_bounded(pfull(pslot), static_cast<uint32_t>((j / kPS) & 1), abort_flag, a.wait_ns) ||
+                !mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns))
+                break;
+            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + pslot * kPSBytes +
+                                                            erow * (kSuper * kBK / 4) + (i % kSuper) * (kBK / 4) +
                                                             16 * half);
             uint8_t* ap = gbase + (sA - base) + stage * kABytes + erow * kBK;
             const uint32_t words[4] = {p.x, p.y, p.z, p.w};
@@ -273,7 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(afull(stage));
+            if (lane == 0) {
+                mbar_arrive(afull(stage));
+                // the group's last stage of this super-tile frees the slot
+                if (i + kExpGroups >= (j + 1) * kSuper || i + kExpGroups >= nk) mbar_arrive(pempty(pslot));
+            }
         }
         // ------------------------------------------------------------- epilogue --
         // the four warps of a lane quarter read 16-token column chunks in turn; thread:
@@ -398,15 +433,20 @@ cudaError_t launch_gemv_tc(const int8_t* xq, const float* s, const uint8_t* pack
             split = sp;
         }
     }
+    // blocks start on packed super-tile boundaries where that keeps the split (a super-tile
+    // that runs past a block's K range would load bytes the block never reads)
+    int64_t sps = (nstages + split - 1) / split;
+    if (sps >= kSuper) sps = (sps + kSuper - 1) / kSuper * kSuper;
+    split = (nstages + sps - 1) / sps;
     if (row_tiles > 65535 || tok_tiles > 65535) return cudaErrorInvalidValue;
     CUtensorMap tx, tp;
     if (!encode_tmap_u8_2d(&tx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kBK, bt, true) ||
-        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kBK / 4, kRows,
-                           false))
+        !encode_tmap_u8_2d(&tp, packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), kSuper * kBK / 4,
+                           kRows, false))
         return cudaErrorInvalidValue;
     const WaitTest wt = wait_test();
     GvArgs a{s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-             static_cast<int>(nstages / split), nstages, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind),
+             static_cast<int>(sps), nstages, out, out_kind_of(kind), err, s4_mul(), gamma_rows_of(kind),
              wt.wait_ns, wt.stall_after};
     const dim3 grid(static_cast<unsigned>(split), static_cast<unsigned>(row_tiles), static_cast<unsigned>(tok_tiles));
     switch (layout) {

@@ -42,12 +42,19 @@
 // leaves its output incomplete).
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "bl_device.cuh"
 #include "bl_internal.h"
 
 namespace bl {
+
+bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer, bool swizzle128);
+bool encode_tmap_f32_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                        uint32_t box_outer);
+
 namespace {
 
 constexpr int kBI = 128;           // rows per tile (MMA M)
@@ -499,6 +506,350 @@ __global__ void __launch_bounds__(kThreads, 1) ste_tc_kernel(const SteArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------------
+// The same GEMM with the raw operands staged by TMA (shapes whose rows are 16-byte
+// aligned: N % 4 == 0, and K % 64 == 0 for dX / K % 16 == 0 for dW).  One thread loads
+// each stage's raw tiles -- dY as fp32 and the packed codes (dX) or x_q (dW) as bytes --
+// into a ring of raw stages, several stages ahead; the converter warps turn a raw stage
+// into the bf16 operand tiles of a converted stage (shared to shared, no global latency
+// on their path) and release the raw stage; the MMA issuer consumes converted stages as
+// before.
+//   warp 0 (one lane)  TMA producer;  warp 1 (one lane)  MMA issuer;
+//   warps 2-5          A converters;  warps 6-13  B converters;  warps 14-17  epilogue.
+constexpr int kThreadsT = 576;  // 18 warps
+constexpr int kWarpTmaT = 0, kWarpMmaT = 1, kWarpAT = 2, kWarpBT = 6, kWarpEpiT = 14;
+constexpr int kAWarpsT = kWarpBT - kWarpAT, kBWarpsT = kWarpEpiT - kWarpBT;
+
+template <int KIND, int BJ>
+struct SteTCfg {
+    static constexpr int kATile = kBI * kRowBytes;
+    static constexpr int kBTile = BJ * kRowBytes;
+    static constexpr int kConvBytes = 2 * kATile + kBTile;
+    static constexpr int kRawA = kBI * kBC * 4;                          // 128 x 64 fp32 either way
+    static constexpr int kRawB = KIND == kDX ? kBC * (BJ / 4) : kBC * BJ;  // 64 rows of codes or x_q
+    static constexpr int kRawBytes = kRawA + kRawB;
+    static constexpr int kCS = 2;  // converted stages
+    static constexpr int kRSRaw = (227 * 1024 - 1024 - 512 - kCS * kConvBytes) / kRawBytes;
+    static constexpr int kRS = kRSRaw > 4 ? 4 : kRSRaw;  // raw stages
+    static constexpr int kTmemCols = 2 * BJ;
+    static constexpr int kBarCount = 2 * kRS + 2 * kCS + 5;
+    static constexpr int kSmemBytes = 1024 + kCS * kConvBytes + kRS * kRawBytes + 8 * kBarCount + 16;
+    static_assert(kRS >= 2, "raw stages");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+template <int KIND, int BJ>
+__global__ void __launch_bounds__(kThreadsT, 1)
+    ste_tma_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                   const SteArgs a) {
+    using Cfg = SteTCfg<KIND, BJ>;
+    constexpr int CS = Cfg::kCS, RS = Cfg::kRS;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw0 = smem_u32(smem_raw);
+    const uint32_t base = (raw0 + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw0);
+    // converted stages first (1024-aligned swizzled tiles), then the raw stages
+    auto cAhi = [&](int c) { return static_cast<uint32_t>(c * Cfg::kConvBytes); };
+    auto cAlo = [&](int c) { return static_cast<uint32_t>(c * Cfg::kConvBytes + Cfg::kATile); };
+    auto cB = [&](int c) { return static_cast<uint32_t>(c * Cfg::kConvBytes + 2 * Cfg::kATile); };
+    auto rA = [&](int r) { return static_cast<uint32_t>(CS * Cfg::kConvBytes + r * Cfg::kRawBytes); };
+    auto rB = [&](int r) { return static_cast<uint32_t>(CS * Cfg::kConvBytes + r * Cfg::kRawBytes + Cfg::kRawA); };
+    const uint32_t sBar = base + CS * Cfg::kConvBytes + RS * Cfg::kRawBytes;
+    auto rfull = [&](int r) { return sBar + 8u * r; };
+    auto rempty = [&](int r) { return sBar + 8u * (RS + r); };
+    auto cfull = [&](int c) { return sBar + 8u * (2 * RS + c); };
+    auto cempty = [&](int c) { return sBar + 8u * (2 * RS + CS + c); };
+    auto tfull = [&](int b) { return sBar + 8u * (2 * RS + 2 * CS + b); };
+    auto tempty = [&](int b) { return sBar + 8u * (2 * RS + 2 * CS + 2 + b); };
+    const uint32_t drain_bar = sBar + 8u * (2 * RS + 2 * CS + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + (sBar - base) + 8 * Cfg::kBarCount);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int r = 0; r < RS; ++r) {
+            mbar_init(rfull(r), 1);
+            mbar_init(rempty(r), kAWarpsT + kBWarpsT);
+        }
+        for (int c = 0; c < CS; ++c) {
+            mbar_init(cfull(c), kAWarpsT + kBWarpsT);
+            mbar_init(cempty(c), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        tma_prefetch_desc(&tmap_a);
+        tma_prefetch_desc(&tmap_b);
+    }
+    pdl_wait_then_release();
+    if (warp == kWarpMmaT) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nC = (a.C + kBC - 1) / kBC;
+    const int my_tiles = a.num_tiles > static_cast<int>(blockIdx.x)
+                             ? (a.num_tiles - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
+                             : 0;
+    const int total = my_tiles * nC;  // stages this block runs, across its tiles
+
+    if (warp == kWarpTmaT) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ producer --
+            int r = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+                const int i0 = (tile % a.tiles_i) * kBI, j0 = (tile / a.tiles_i) * BJ;
+                for (int kc = 0; kc < nC; ++kc) {
+                    const int c0 = kc * kBC;
+                    if (!mbar_wait_bounded(rempty(r), phase ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(rfull(r), Cfg::kRawBytes);
+                    if constexpr (KIND == kDX) {
+                        tma_load_2d(base + rA(r), &tmap_a, rfull(r), c0, i0);       // dY[i0 .., c0 ..]
+                        tma_load_2d(base + rB(r), &tmap_b, rfull(r), j0 / 4, c0);   // packed[c0 .., j0/4 ..]
+                    } else {
+                        tma_load_2d(base + rA(r), &tmap_a, rfull(r), i0, c0);       // dY[c0 .., i0 ..]
+                        tma_load_2d(base + rB(r), &tmap_b, rfull(r), j0, c0);       // x_q[c0 .., j0 ..]
+                    }
+                    ++issued;
+                    if (++r == RS) {
+                        r = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                for (int q = 0; q < RS; ++q) {
+                    const long long fills = (issued - q + RS - 1) / RS;
+                    if (fills > 0) mbar_drain_ste(rfull(q), static_cast<uint32_t>((fills - 1) & 1));
+                }
+            }
+        }
+    } else if (warp == kWarpMmaT) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- MMA issuer --
+            constexpr uint32_t idesc = idesc_bf16(kBI, BJ);
+            int c = 0, buf = 0;
+            uint32_t phase = 0, bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
+                if (!mbar_wait_bounded(tempty(buf), bphase ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BJ);
+                for (int kc = 0; kc < nC; ++kc) {
+                    if (!mbar_wait_bounded(cfull(c), phase, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBC / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(base + cB(c) + 32 * kk);
+                        tc_mma_bf16(d_tmem, smem_desc_sw128(base + cAhi(c) + 32 * kk), bd, idesc,
+                                    (kc | kk) != 0 ? 1u : 0u);
+                        tc_mma_bf16(d_tmem, smem_desc_sw128(base + cAlo(c) + 32 * kk), bd, idesc, 1u);
+                    }
+                    tc_commit(cempty(c));
+                    if (++c == CS) {
+                        c = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(tfull(buf));
+                if (++buf == 2) {
+                    buf = 0;
+                    bphase ^= 1u;
+                }
+            }
+            if (!ok) {
+                tc_commit(drain_bar);
+                mbar_drain_ste(drain_bar, 0);
+            }
+        }
+    } else if (warp < kWarpEpiT) {
+        // ------------------------------------------------------------- converters --
+        // every converter warp takes part in every stage: wait for its raw stage and a
+        // free converted stage, convert its share, release the raw stage, then mark the
+        // converted stage full
+        const bool is_a = warp < kWarpBT;
+        const int t = is_a ? threadIdx.x - 32 * kWarpAT : threadIdx.x - 32 * kWarpBT;
+        for (int i = 0; i < total; ++i) {
+            const int r = i % RS, c = i % CS;
+            const uint32_t rph = static_cast<uint32_t>((i / RS) & 1), cph = static_cast<uint32_t>((i / CS) & 1);
+            const int kc = i % nC;
+            const int c0 = kc * kBC;
+            // dW: the stage's 64 reciprocals 1/s_m (two per lane), fetched before the waits
+            float rA_ = 0.0f, rB_ = 0.0f;
+            if constexpr (KIND == kDW) {
+                if (is_a) {
+                    const int mA = c0 + lane, mB = c0 + 32 + lane;
+                    rA_ = mA < a.M ? __frcp_rn(__ldg(a.s + mA)) : 0.0f;
+                    rB_ = mB < a.M ? __frcp_rn(__ldg(a.s + mB)) : 0.0f;
+                }
+            }
+            if (!mbar_wait_bounded(rfull(r), rph, abort_flag) || !mbar_wait_bounded(cempty(c), cph ^ 1u, abort_flag))
+                break;
+            const uint8_t* ra = gbase + rA(r);
+            const uint8_t* rb = gbase + rB(r);
+            if (is_a) {
+                uint8_t* ahi = gbase + cAhi(c);
+                uint8_t* alo = gbase + cAlo(c);
+                if constexpr (KIND == kDX) {
+                    // raw [128 tokens][64 n] fp32 -> A[m][n]: eight threads per row
+                    const int r_off = t >> 3, ch = t & 7;
+#pragma unroll
+                    for (int p = 0; p < kBI / 16; ++p) {
+                        const int row = 16 * p + r_off;
+                        const float4* src = reinterpret_cast<const float4*>(ra + row * (kBC * 4) + ch * 32);
+                        const float4 u = src[0], v = src[1];
+                        const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+                        uint4 hi, lo;
+                        split8(x, hi, lo);
+                        *reinterpret_cast<uint4*>(ahi + sw128(row, ch)) = hi;
+                        *reinterpret_cast<uint4*>(alo + sw128(row, ch)) = lo;
+                    }
+                } else {
+                    // raw [64 tokens][128 n] fp32 -> A[n][m] = dY[m][n] / s[m]: thread = row n
+                    const float* rf = reinterpret_cast<const float*>(ra);
+#pragma unroll
+                    for (int ch = 0; ch < kBC / 8; ++ch) {
+                        float x[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int m = 8 * ch + e;
+                            x[e] = __fmul_rn(rf[m * kBI + t], __shfl_sync(0xffffffffu, m < 32 ? rA_ : rB_, m & 31));
+                        }
+                        uint4 hi, lo;
+                        split8(x, hi, lo);
+                        *reinterpret_cast<uint4*>(ahi + sw128(t, ch)) = hi;
+                        *reinterpret_cast<uint4*>(alo + sw128(t, ch)) = lo;
+                    }
+                }
+            } else {
+                uint8_t* bt = gbase + cB(c);
+                if constexpr (KIND == kDX) {
+                    // raw packed [64 n][BJ/4 bytes] -> B[k][n]: units of 8 k x 8 n
+                    constexpr int kUnits = (BJ / 8) * 8;
+                    for (int u = t; u < kUnits; u += 32 * kBWarpsT) {
+                        const int kg = u % (BJ / 8), nch = u / (BJ / 8);
+                        uint32_t w[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            w[q] = *reinterpret_cast<const uint16_t*>(rb + (8 * nch + q) * (BJ / 4) + 2 * kg);
+                        uint32_t g[2][2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t t01 = __byte_perm(w[4 * h], w[4 * h + 1], 0x5140);
+                            const uint32_t t23 = __byte_perm(w[4 * h + 2], w[4 * h + 3], 0x5140);
+                            g[0][h] = __byte_perm(t01, t23, 0x5410);
+                            g[1][h] = __byte_perm(t01, t23, 0x7632);
+                        }
+#pragma unroll
+                        for (int kr = 0; kr < 8; ++kr) {
+                            const int b = kr >> 2, sh = 2 * (kr & 3);
+                            uint4 o;
+                            codes4_to_bf16((g[b][0] >> sh) & 0x03030303u, o.x, o.y);
+                            codes4_to_bf16((g[b][1] >> sh) & 0x03030303u, o.z, o.w);
+                            *reinterpret_cast<uint4*>(bt + sw128(8 * kg + kr, nch)) = o;
+                        }
+                    }
+                } else {
+                    // raw x_q [64 tokens][BJ bytes] -> B[k][m]: units of 4 k x 8 m
+                    constexpr int kUnits = (BJ / 4) * 8;
+                    for (int u = t; u < kUnits; u += 32 * kBWarpsT) {
+                        const int kw = u % (BJ / 4), mch = u / (BJ / 4);
+                        uint32_t w[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            w[q] = *reinterpret_cast<const uint32_t*>(rb + (8 * mch + q) * BJ + 4 * kw);
+#pragma unroll
+                        for (int kr = 0; kr < 4; ++kr) {
+                            uint4 o;
+                            o.x = bf16x2_of_s8(w[0] >> (8 * kr), w[1] >> (8 * kr));
+                            o.y = bf16x2_of_s8(w[2] >> (8 * kr), w[3] >> (8 * kr));
+                            o.z = bf16x2_of_s8(w[4] >> (8 * kr), w[5] >> (8 * kr));
+                            o.w = bf16x2_of_s8(w[6] >> (8 * kr), w[7] >> (8 * kr));
+                            *reinterpret_cast<uint4*>(bt + sw128(4 * kw + kr, mch)) = o;
+                        }
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(rempty(r));
+                mbar_arrive(cfull(c));
+            }
+        }
+    } else {
+        // -------------------------------------------------------------- epilogue --
+        const int q = warp & 3;
+        const float g = *a.gamma;
+        const bool vec = (a.J & 3) == 0;
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+            const int i0 = (tile % a.tiles_i) * kBI, j0 = (tile / a.tiles_i) * BJ;
+            if (!mbar_wait_bounded(tfull(buf), bphase, abort_flag)) break;
+            tc_fence_after();
+            const int i = i0 + 32 * q + lane;
+            float* orow = a.out + static_cast<int64_t>(i) * a.J;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BJ; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
+                                       static_cast<uint32_t>(buf * BJ + c0),
+                                   r);
+                tmem_ld_wait();
+                if (i >= a.I) continue;
+                const int j = j0 + c0;
+                if (vec && j + 32 <= a.J) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(orow + j + e) =
+                            make_float4(__fmul_rn(g, __uint_as_float(r[e])), __fmul_rn(g, __uint_as_float(r[e + 1])),
+                                        __fmul_rn(g, __uint_as_float(r[e + 2])),
+                                        __fmul_rn(g, __uint_as_float(r[e + 3])));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j + e < a.J) orow[j + e] = __fmul_rn(g, __uint_as_float(r[e]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty(buf));
+            if (++buf == 2) {
+                buf = 0;
+                bphase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMmaT) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
 int sm_count_ste() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -539,10 +890,41 @@ cudaError_t launch_ste_bj(SteArgs a, int sms, cudaStream_t stream) {
                       dim3(kNoCluster), a);
 }
 
+template <int KIND, int BJ>
+cudaError_t launch_ste_tma_bj(SteArgs a, int sms, cudaStream_t stream) {
+    using Cfg = SteTCfg<KIND, BJ>;
+    CUtensorMap ta, tb;
+    // dY is [M, N] fp32 for both; the raw box is 64 x 128 (dX: n-inner) or 128 x 64 (dW)
+    const bool ok_a = KIND == kDX
+                          ? encode_tmap_f32_2d(&ta, a.dY, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M), kBC, kBI)
+                          : encode_tmap_f32_2d(&ta, a.dY, static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M), kBI, kBC);
+    const bool ok_b = KIND == kDX
+                          ? encode_tmap_u8_2d(&tb, a.packed, static_cast<uint64_t>(a.K / 4), static_cast<uint64_t>(a.N),
+                                              BJ / 4, kBC, false)
+                          : encode_tmap_u8_2d(&tb, a.xq, static_cast<uint64_t>(a.K), static_cast<uint64_t>(a.M), BJ, kBC,
+                                              false);
+    if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+    static PerContextOnce attr;
+    cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(ste_tma_kernel<KIND, BJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    Cfg::kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
+    a.tiles_i = (a.I + kBI - 1) / kBI;
+    a.num_tiles = a.tiles_i * ((a.J + BJ - 1) / BJ);
+    const int grid = a.num_tiles < sms ? a.num_tiles : sms;
+    return launch_pdl(ste_tma_kernel<KIND, BJ>, dim3(grid), dim3(kThreadsT), Cfg::kSmemBytes, stream,
+                      dim3(kNoCluster), ta, tb, a);
+}
+
 template <int KIND>
 cudaError_t launch_ste(SteArgs a, cudaStream_t stream) {
     const int sms = sm_count_ste();
-    if (ste_tile(a.I, a.J, sms) == 256) return launch_ste_bj<KIND, 256>(a, sms, stream);
+    const int bj = ste_tile(a.I, a.J, sms);
+    // TMA needs 16-byte row pitches: dY rows (N % 4), packed rows (K % 64) or x_q rows (K % 16)
+    const bool staged = (a.N % 4) == 0 && (KIND == kDX ? a.K % 64 == 0 : a.K % 16 == 0);
+    if (staged) return bj == 256 ? launch_ste_tma_bj<KIND, 256>(a, sms, stream) : launch_ste_tma_bj<KIND, 128>(a, sms, stream);
+    if (bj == 256) return launch_ste_bj<KIND, 256>(a, sms, stream);
     return launch_ste_bj<KIND, 128>(a, sms, stream);
 }
 
