@@ -16,8 +16,9 @@
 //
 // Tile: 128 weight rows (MMA M, TMEM lanes) x BT tokens (MMA N; 16 to 128) x a slice of
 // K in stages of 128 codes.  Per stage:
-//   warp 0 (one lane)   TMA: packed weights [128 rows x 32 B] and the x_q tile
-//                       [BT x 128 B] (128-byte swizzle) on one mbarrier;
+//   warp 0 (one lane)   TMA: the x_q tile [BT x 128 B] (128-byte swizzle) per stage,
+//                       and the packed weights of eight stages at a time [128 rows x
+//                       256 B] into a two-slot ring with its own mbarriers;
 //   warps 2-17          expanders, two groups of eight warps taking alternate stages: two
 //                       threads per weight row, each unpacking 64 codes in the order of
 //                       the x_q layout into the swizzled A tile; fence.proxy.async, then

@@ -1,5 +1,5 @@
-"""Parity of the small-batch tcgen05 forward (BL_PATH_SKINNY: expanded weights in tensor
-memory, K split over a thread-block cluster when rows are few) with the oracle: ragged
+"""Parity of the small-batch tcgen05 forward (BL_PATH_SKINNY: weights expanded to int8 in
+shared memory, K split over a thread-block cluster when rows are few) with the oracle: ragged
 shapes in every x_q layout and output kind, the LLaMA-70B decode shapes at 17 to 64
 tokens (the automatic dispatch's range for this kernel), the largest accumulators,
 per-row weight scales, undefined code 11, and repeated launches.
