@@ -84,8 +84,16 @@ typedef enum {
     BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
     BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
     BL_PATH_TC_2SM = 4, /* the tcgen05 path forced to SM-pair (cta_group::2) tiles (testing) */
-    BL_PATH_SKINNY = 5  /* the tcgen05 small-batch kernel (K split over a cluster when rows
+    BL_PATH_SKINNY = 5, /* the tcgen05 small-batch kernel (K split over a cluster when rows
                            are few); K % 64 == 0 */
+    BL_PATH_GEMV_STREAM = 6, /* the GEMV kernel fed by per-thread asynchronous copies (testing):
+                                M <= 16, x_q in BL_XQ_K16_STRIDE4, K % 64 == 0, K <= 2^17, and
+                                between 1 and 64 sixteen-row tiles of N per SM; other shapes
+                                return BL_ERR_UNSUPPORTED_SHAPE */
+    BL_PATH_GEMV_TMA = 7     /* the persistent TMA-fed GEMV kernel (testing): M <= 16, x_q in
+                                BL_XQ_K16_STRIDE4, K % 128 == 0, K <= 2^17, and between 1 and
+                                32 sixteen-row tiles of N per SM; other shapes return
+                                BL_ERR_UNSUPPORTED_SHAPE */
 } bl_path;
 
 /* Storage order of x_q within each row.
@@ -219,8 +227,8 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
 
 /* A test of the bounded device waits (the source pages have no counterpart): the forward
  * of bitlinear_forward_layout on one of the kernels that wait for TMA loads
- * (BL_PATH_TC_1SM, BL_PATH_SKINNY, or BL_PATH_GEMV where it runs its TMA-fed form:
- * x_q in BL_XQ_K16_STRIDE4 and a layer wide enough), in which every wait gives up after
+ * (BL_PATH_TC_1SM, BL_PATH_SKINNY, or BL_PATH_GEMV_TMA -- BL_PATH_GEMV is read as
+ * BL_PATH_GEMV_TMA here -- with its shape conditions), in which every wait gives up after
  * wait_limit_ns (0 < wait_limit_ns <= 2 s; the forward entry points use 2 s) and the
  * load producer of each block stops after stall_after_loads loads.  The waits for the
  * next load then run out: the kernel stops its other roles, lets every copy and MMA in
@@ -228,7 +236,7 @@ BL_API bl_status bitlinear_forward_path(const int8_t *xq, const float *s, const 
  * returns; the output is left incomplete.  If a block needs no more loads than
  * stall_after_loads it finishes normally.  The next call on the stream runs as usual.
  * Errors: those of bitlinear_forward_layout; BL_ERR_INVALID_ARG for another path or a
- * limit out of range, BL_ERR_UNSUPPORTED_SHAPE for a GEMV shape without the TMA form. */
+ * limit out of range, BL_ERR_UNSUPPORTED_SHAPE for a shape the TMA-fed GEMV does not take. */
 BL_API bl_status bitlinear_forward_stall_test(const int8_t *xq, const float *s, const uint8_t *packed,
                                               const float *gamma, int64_t M, int64_t N, int64_t K, void *out,
                                               bl_dtype out_dtype, int32_t *err_word, bl_xq_layout xq_layout,

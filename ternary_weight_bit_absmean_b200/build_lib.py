@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbitlinear.so")
-SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemv_tc.cu", "k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_noalloc.cu", "k_tl5.cu", "k_ste.cu"]
+SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemv_tc.cu", "k_gemv_stream.cu", "k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_noalloc.cu", "k_tl5.cu", "k_ste.cu"]
 HEADERS = ["bl_device.cuh", "bl_internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

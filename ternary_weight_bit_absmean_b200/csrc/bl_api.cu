@@ -171,7 +171,7 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     if (out_dtype != BL_OUT_F32 && out_dtype != BL_OUT_BF16 && out_dtype != BL_OUT_I32)
         return BL_ERR_INVALID_ARG;
     if (path != BL_PATH_AUTO && path != BL_PATH_GEMV && path != BL_PATH_TC && path != BL_PATH_TC_1SM &&
-        path != BL_PATH_TC_2SM && path != BL_PATH_SKINNY)
+        path != BL_PATH_TC_2SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV_STREAM && path != BL_PATH_GEMV_TMA)
         return BL_ERR_INVALID_ARG;
     if (xq_layout != BL_XQ_ROWMAJOR && xq_layout != BL_XQ_K16_EVENODD && xq_layout != BL_XQ_K16_STRIDE4)
         return BL_ERR_INVALID_ARG;
@@ -187,6 +187,11 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
     // the tensor-core kernels expand stride-4 codes as 64 * code: 64 * 128 * K must fit
     const bool s4_big = xq_layout == BL_XQ_K16_STRIDE4 && K > (int64_t(1) << 17);
     if (tc && s4_big) return BL_ERR_UNSUPPORTED_SHAPE;
+    if (path == BL_PATH_GEMV_STREAM &&
+        (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_stream_applicable(M, N, K)))
+        return BL_ERR_UNSUPPORTED_SHAPE;
+    if (path == BL_PATH_GEMV_TMA && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
+        return BL_ERR_UNSUPPORTED_SHAPE;
     if (path == BL_PATH_AUTO)
         path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : (M <= 64 ? BL_PATH_SKINNY : BL_PATH_TC);
     if (gamma_per_row && !aligned16(gamma)) return BL_ERR_MISALIGNED;
@@ -202,6 +207,10 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
         e = bl::launch_gemm_tc2(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else if (path == BL_PATH_SKINNY) {
         e = bl::launch_gemv_tc(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
+    } else if (path == BL_PATH_GEMV_STREAM) {
+        e = bl::launch_gemv_stream(xq, s, packed, gamma, M, N, K, out, kind, st);
+    } else if (path == BL_PATH_GEMV_TMA) {
+        e = bl::launch_gemv_tma(xq, s, packed, gamma, M, N, K, out, kind, err_word, st);
     } else if (k64 && M <= int64_t(65535) * 16) {
         e = bl::launch_gemv(xq, s, packed, gamma, M, N, K, out, kind, err_word, lay, st);
     } else {
@@ -303,9 +312,11 @@ bl_status bitlinear_forward_stall_test(const int8_t* xq, const float* s, const u
     BL_RANGE("bitlinear_forward_stall_test");
     if (wait_limit_ns == 0 || wait_limit_ns > bl::kDefaultWaitNs || stall_after_loads < 0) return BL_ERR_INVALID_ARG;
     // only the kernels that wait on TMA loads: the single-SM tcgen05 kernel, the small-
-    // batch tcgen05 kernel, and the decode GEMV where it takes its TMA-fed form
-    if (path != BL_PATH_TC_1SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV) return BL_ERR_INVALID_ARG;
-    if (path == BL_PATH_GEMV && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
+    // batch tcgen05 kernel, and the TMA-fed decode GEMV (BL_PATH_GEMV names it here)
+    if (path != BL_PATH_TC_1SM && path != BL_PATH_SKINNY && path != BL_PATH_GEMV && path != BL_PATH_GEMV_TMA)
+        return BL_ERR_INVALID_ARG;
+    if (path == BL_PATH_GEMV) path = BL_PATH_GEMV_TMA;
+    if (path == BL_PATH_GEMV_TMA && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
         return BL_ERR_UNSUPPORTED_SHAPE;
     const bl::WaitTest saved = bl::g_wait_test;
     bl::g_wait_test = bl::WaitTest{wait_limit_ns, stall_after_loads};

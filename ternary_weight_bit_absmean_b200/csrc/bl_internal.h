@@ -64,6 +64,11 @@ bool gemv_tma_applicable(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_gemv_tma(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                             int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err,
                             cudaStream_t stream);
+// The GEMV fed by per-thread asynchronous copies (k_gemv_stream.cu), x_q in the
+// stride-4 k16 layout; gemv_stream_applicable states its shape conditions.
+bool gemv_stream_applicable(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_stream(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
+                               int64_t M, int64_t N, int64_t K, void* out, int kind, cudaStream_t stream);
 // Plain fallback for K % 64 != 0 (one output per thread).
 cudaError_t launch_gemv_generic(const int8_t* xq, const float* s, const uint8_t* packed,
                                 const float* gamma, int64_t M, int64_t N, int64_t K, void* out,

@@ -120,6 +120,8 @@ def test_other_entry_points_validation(L):
     for p in (2, 3, 4):  # every tcgen05 variant needs K % 64 == 0
         assert path(FAKE, FAKE, FAKE, FAKE, 40, 8, 96, FAKE, 0, None, p, None) == SHAPE
     assert path(FAKE, FAKE, FAKE, FAKE, 4, 8, 64, FAKE, 0, None, 9, None) == INVALID
+    for p in (6, 7):  # the two forced decode GEMV kernels read x_q in the stride-4 layout only
+        assert path(FAKE, FAKE, FAKE, FAKE, 4, 8192, 256, FAKE, 0, None, p, None) == SHAPE
     assert L.bitlinear_status_string(3) == b"BL_ERR_MISALIGNED"
     lay = L.bitlinear_forward_layout
     for k16 in (1, 2):  # the k16 layouts need K % 16 == 0
