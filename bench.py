@@ -73,9 +73,10 @@ def parse():
     p.add_argument("--weight-format", choices=["2bit", "tl5"], default="2bit",
                    help="--sweep: the 2-bit forward, or the five-codes-per-byte decode forward (M <= 16 shapes)")
     p.add_argument("--single", choices=["forward", "quantize_act", "norm_quantize_act", "quantize_weights", "pack",
-                                        "forward_tl5", "repack_tl5", "ste_input", "ste_weight", "copy"],
+                                        "forward_tl5", "repack_tl5", "ste_input", "ste_weight", "copy", "read"],
                    help="time one entry point on one shape instead of the step (kernel study, ncu); "
-                        "'copy' times a device-to-device copy of the packed weights' size as a reference")
+                        "'copy' times a device-to-device copy of the packed weights' size, 'read' a max-reduction "
+                        "over that many bytes, as references")
     p.add_argument("--M", type=int, default=4096)
     p.add_argument("--N", type=int, default=4096)
     p.add_argument("--K", type=int, default=4096)
@@ -738,6 +739,19 @@ def run_single(args):
         copies = max(2, -(-3 * L2_BYTES // nbytes))
         pairs = [(src, dst)] + [(src.clone(), torch.empty_like(src)) for _ in range(copies - 1)]
         rot_fns = [(lambda p=p: p[1].copy_(p[0])) for p in pairs]
+    elif args.single == "read":
+        # reference for one launch's reachable read-only bandwidth: a plain streaming read
+        # (every 16-byte chunk once, full occupancy, four loads in flight per thread) of as
+        # many bytes as the packed weights of an N x K matrix
+        rk = read_kernel()
+        src = torch.ones(N * K // 4, dtype=torch.uint8, device=dev)
+        sink = torch.zeros(4, dtype=torch.int32, device=dev)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        fn = lambda: rk.stream_read(src, sink, 4 * sms)
+        ops, nbytes = 0, src.numel()
+        copies = max(2, -(-3 * L2_BYTES // nbytes))
+        srcs = [src] + [src.clone() for _ in range(copies - 1)]
+        rot_fns = [(lambda x=x: rk.stream_read(x, sink, 4 * sms)) for x in srcs]
     elif args.single == "quantize_weights":
         W = torch.randn(N, K, device=dev) * 0.02
         gamma = torch.empty(1, device=dev)
@@ -752,7 +766,7 @@ def run_single(args):
         ops, nbytes = 0, N * K + N * K // 4
     ts = time_calls(fn, flusher, args.iters)
     t = statistics.median(ts) * 1e-3
-    t_b2b = time_back_to_back(rot_fns, flusher, 4) if args.single in ("forward", "copy") else None
+    t_b2b = time_back_to_back(rot_fns, flusher, 4) if args.single in ("forward", "copy", "read") else None
     rec = {"single": args.single, "M": M, "N": N, "K": K, "path": args.path, "out_dtype": args.out_dtype,
            "xq_layout": args.xq_layout,
            "us_median": round(t * 1e6, 2), "us_min": round(min(ts) * 1e3, 2),
@@ -773,6 +787,40 @@ def run_single(args):
         else:
             rec["int8_frac"] = round(ops / t / 1e12 / (2.0 * P["bf16_tflops"]), 4)
     print(json.dumps(rec), flush=True)
+
+
+READ_KERNEL_SRC = r"""
+#include <torch/extension.h>
+#include <c10/cuda/CUDAStream.h>
+__global__ void __launch_bounds__(512, 4) stream_read_kernel(const uint4* __restrict__ w, long long n, int* sink) {
+    uint4 acc = make_uint4(0, 0, 0, 0);
+    const long long step = (long long)gridDim.x * blockDim.x;
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * step < n; i += 4 * step) {
+        const uint4 a = __ldcs(w + i), b = __ldcs(w + i + step), c = __ldcs(w + i + 2 * step), d = __ldcs(w + i + 3 * step);
+        acc.x ^= a.x ^ b.x ^ c.x ^ d.x; acc.y ^= a.y ^ b.y ^ c.y ^ d.y;
+        acc.z ^= a.z ^ b.z ^ c.z ^ d.z; acc.w ^= a.w ^ b.w ^ c.w ^ d.w;
+    }
+    for (; i < n; i += step) { const uint4 a = __ldcs(w + i); acc.x ^= a.x; acc.y ^= a.y; acc.z ^= a.z; acc.w ^= a.w; }
+    if ((acc.x ^ acc.y ^ acc.z ^ acc.w) == 0x9E3779B9u) sink[0] = 1;  // keeps the loads
+}
+void stream_read(torch::Tensor w, torch::Tensor sink, int64_t blocks) {
+    stream_read_kernel<<<(unsigned)blocks, 512, 0, c10::cuda::getCurrentCUDAStream()>>>(
+        reinterpret_cast<const uint4*>(w.data_ptr()), w.numel() / 16, sink.data_ptr<int>());
+}
+"""
+
+
+def read_kernel():
+    """The streaming-read reference kernel of `--single read`, compiled on first use."""
+    import tempfile
+    from torch.utils.cpp_extension import load_inline
+    build = os.path.join(tempfile.gettempdir(), "bitlinear_bench_read")
+    os.makedirs(build, exist_ok=True)
+    return load_inline("bitlinear_bench_read", cpp_sources="void stream_read(torch::Tensor w, torch::Tensor sink, "
+                       "int64_t blocks);", cuda_sources=READ_KERNEL_SRC, functions=["stream_read"],
+                       extra_cuda_cflags=["-O3", "-gencode", "arch=compute_100a,code=sm_100a"],
+                       build_directory=build, verbose=False)
 
 
 def time_calls(fn, flusher, iters):
