@@ -55,8 +55,9 @@ inline int out_kind_of(int kind) { return kind & 0xFF; }
 inline int gamma_rows_of(int kind) { return (kind & kGammaPerRow) ? 1 : 0; }
 
 // Decode GEMV: register unpack + mma.sync, any M (token groups of 16), K % 64 == 0.
-// With x_q in the stride-4 k16 layout and a shape gemv_tma_applicable accepts, it runs
-// the persistent TMA-fed kernel (k_gemv_tma.cu).
+// With x_q in the stride-4 k16 layout it runs the kernel fed by per-thread asynchronous
+// copies (k_gemv_stream.cu) where gemv_stream_applicable accepts the shape, else the
+// persistent TMA-fed kernel (k_gemv_tma.cu) where gemv_tma_applicable does.
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed,
                         const float* gamma, int64_t M, int64_t N, int64_t K, void* out, int kind,
                         int32_t* err, int layout, cudaStream_t stream);

@@ -411,6 +411,8 @@ cudaError_t launch_gemv_mt(GemvArgs a, int S, int64_t row_blocks, int64_t token_
 cudaError_t launch_gemv(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                         int64_t M, int64_t N, int64_t K, void* out, int kind, int32_t* err, int layout,
                         cudaStream_t stream) {
+    if (layout == kXqStride4K16 && gemv_stream_applicable(M, N, K))
+        return launch_gemv_stream(xq, s, packed, gamma, M, N, K, out, kind, stream);
     if (layout == kXqStride4K16 && gemv_tma_applicable(M, N, K))
         return launch_gemv_tma(xq, s, packed, gamma, M, N, K, out, kind, err, stream);
     const int grow = gamma_rows_of(kind);

@@ -14,17 +14,19 @@
 // and the weights stream at about a third of the copy rate.  Here every thread copies
 // the bytes it will itself unpack (cp.async, 16 bytes, L1 bypassed, with a 256-byte L2
 // prefetch so DRAM still sees long runs) into a private ring of stages in shared memory:
-// no barrier between warps in the main loop, 24 warps per SM, and several kilobytes per
-// warp in flight.
+// no barrier between warps in the main loop, 24-32 warps per SM, and 96 KB per SM in
+// flight.
 //
 // Work split.  One block per SM owns a contiguous, balanced run of 16-row tiles over the
 // whole of K.  A unit is one tile's 16 rows x one 256-code quarter of K (1 KB of packed
 // weights).  The block's units are ordered quarter-major (all tiles of quarter 0, then
 // quarter 1, ...) and cut into equal contiguous chunks, one per warp, so a warp holds one
-// quarter's activations in registers for a run of tiles.  After each unit the warp adds
-// its int32 partial tile into a shared-memory accumulator of the block with shared
-// atomics (integer sums are exact in any order); after a block barrier the block scales
-// and stores its rows, coalesced along N.
+// quarter's activations in registers for a run of tiles (read from the block's copy of
+// the activations in shared memory when they fit there, else from global memory).  After
+// each unit the warp adds its int32 partial tile into a shared-memory accumulator of the
+// block with shared atomics (integer sums are exact in any order); after a block barrier
+// the block scales and stores its rows, coalesced along N.  (A tile-major order, each
+// warp walking along K, was measured slower: it reloads the activations every unit.)
 //
 // Thread (g, t) of a warp (g = lane / 4, t = lane % 4) owns, in every unit, rows g and
 // g + 8 of the tile at bytes 64 q + 16 t of the quarter q (16-groups 4 (4q + t) + i,
@@ -41,12 +43,21 @@ namespace bl {
 
 namespace {
 
-constexpr int kWarps = 24;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;                      // units in flight per warp
+// Warps per block and units in flight per warp, per token-tile count: one token tile
+// fits 64 registers, so 32 warps x 3 stages; two need more, so 24 warps x 4 stages
+// (measured on the LLaMA-70B decode shapes).  Either way 96 KB of copies per SM.
+template <int MT>
+struct StreamCfg {
+    static constexpr int W = MT == 1 ? 32 : 24;
+    static constexpr int S = MT == 1 ? 3 : 4;
+};
 constexpr int kWarpStage = 1024;                // bytes per warp and stage: [row g | row g + 8][lane][16 B]
-constexpr int kRingBytes = kWarps * kStages * kWarpStage;  // 96 KB
+constexpr int kRingBytes = 96 * 1024;
+static_assert(StreamCfg<1>::W * StreamCfg<1>::S * kWarpStage == kRingBytes, "ring size");
+static_assert(StreamCfg<2>::W * StreamCfg<2>::S * kWarpStage == kRingBytes, "ring size");
 constexpr int kMaxTiles = 64;                   // 16-row tiles per block
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kXPad = 16;                       // bytes after each staged activation row
 constexpr int kTokStride = 20;                  // ints per token row of a tile's accumulator
 constexpr int64_t kMaxK = int64_t(1) << 17;     // keeps 64 * 128 * K below 2^31
 
@@ -61,6 +72,8 @@ struct GsArgs {
     void* out;
     int kind;
     int grow;  // gamma holds one scale per output row
+    int tmax;  // the most tiles a block owns (sizes the accumulator)
+    int xs;    // the activations are staged in shared memory (M rows of K + kXPad bytes)
     S4Mul mul;
 };
 
@@ -72,6 +85,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
@@ -131,24 +150,43 @@ __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int ac
 
 // Shared memory: the block accumulator [tile][token][kTokStride ints: 16 rows + 4 pad]
 // (the pad puts the eight row groups and four token pairs of a warp's atomics in 32
-// distinct banks), then the copy ring [warp][stage][row g, row g + 8][lane][16 B], so
-// that each of a warp's two shared loads per unit reads 512 contiguous bytes.
+// distinct banks), the copy ring [warp][stage][row g, row g + 8][lane][16 B] (each of a
+// warp's two shared loads per unit reads 512 contiguous bytes), and, when they fit, the
+// block's copy of the activations [token][K + kXPad bytes] (the pad spreads the tokens'
+// rows over the banks).
+__host__ __device__ constexpr uint32_t red_bytes_of(int tmax, int MT) {
+    return (static_cast<uint32_t>(tmax) * 8 * MT * kTokStride * 4 + 15u) & ~15u;
+}
+
 template <int MT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const GsArgs a) {
+__global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(const GsArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     constexpr int TOK = 8 * MT;
+    constexpr int kWarps = StreamCfg<MT>::W, kStages = StreamCfg<MT>::S, kThreads = 32 * kWarps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int t_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * a.ntiles) / gridDim.x);
     const int t_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * a.ntiles) / gridDim.x);
     const int T = t_end - t_begin;
     int* red = reinterpret_cast<int*>(smem);
-    const uint32_t red_bytes = static_cast<uint32_t>(kMaxTiles * TOK * kTokStride * sizeof(int));
+    const uint32_t red_bytes = red_bytes_of(a.tmax, MT);
     const uint32_t ring = smem_u32(smem) + red_bytes + static_cast<uint32_t>(warp * kStages * kWarpStage) +
                           static_cast<uint32_t>(16 * lane);
+    const uint32_t xsm = smem_u32(smem) + red_bytes + kRingBytes;
+    const int xstride = a.K + kXPad;
 
     for (int i = threadIdx.x; i < T * TOK * kTokStride; i += kThreads) red[i] = 0;
     pdl_wait_then_release();
+    if (a.xs) {
+        const int cpr = a.K / 16;  // 16-byte chunks per activation row
+        for (int c = threadIdx.x; c < a.M * cpr; c += kThreads) {
+            const int r = c / cpr, k = c - r * cpr;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<int64_t>(r) * a.K) + k);
+            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(xsm + r * xstride + 16 * k), "r"(v.x),
+                         "r"(v.y), "r"(v.z), "r"(v.w)
+                         : "memory");
+        }
+    }
     __syncthreads();
 
     const int U = T * a.Q;
@@ -157,20 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const GsArgs a
     const int64_t rs = a.K / 4;  // packed bytes per row
     const int rowg = 16 * t_begin + g;
 
-    // unit (q, tile): copy rows g and g + 8 of the tile at bytes 64 q + 16 t
-    auto issue = [&](int q, int tile, int stage) {
-        const int off = 64 * q + 16 * t;
-        const bool in_k = 4 * off < a.K;
-        const int r0 = rowg + 16 * tile, r1 = r0 + 8;
-        const bool v0 = in_k && r0 < a.N, v1 = in_k && r1 < a.N;
-        const uint8_t* p0 = a.packed + (v0 ? static_cast<int64_t>(r0) * rs + off : 0);
-        const uint8_t* p1 = a.packed + (v1 ? static_cast<int64_t>(r1) * rs + off : 0);
-        const uint32_t dst = ring + static_cast<uint32_t>(stage * kWarpStage);
-        cp_async_16(dst, p0, v0 ? 16u : 0u);
-        cp_async_16(dst + kWarpStage / 2, p1, v1 ? 16u : 0u);
-    };
     // unit u is (q, tile) = (u / T, u % T); the issue and compute positions advance by
-    // one tile at a time
+    // one tile at a time.  The issue position keeps the byte offset of row g of its tile
+    // at its quarter (row g + 8 is 8 rows further), moved by one tile (16 rows) per unit.
     int iq = u0 / T, itile = u0 - iq * T;
     const int cq0 = iq, ctile0 = itile;
     auto advance = [&](int& q, int& tile) {
@@ -179,12 +206,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const GsArgs a
             ++q;
         }
     };
+    const int64_t tile_bytes = 16 * rs;
+    int64_t ioff = (rowg + 16 * static_cast<int64_t>(itile)) * rs + 64 * iq + 16 * t;
+    bool iin_k = 256 * iq + 64 * t < a.K;
+    // copy rows g and g + 8 of the issue position's unit into the stage, then advance it
+    auto issue_next = [&](int stage) {
+        const int r0 = rowg + 16 * itile;
+        const bool v0 = iin_k && r0 < a.N, v1 = iin_k && r0 + 8 < a.N;
+        const uint32_t dst = ring + static_cast<uint32_t>(stage * kWarpStage);
+        cp_async_16(dst, a.packed + (v0 ? ioff : 0), v0 ? 16u : 0u);
+        cp_async_16(dst + kWarpStage / 2, a.packed + (v1 ? ioff + 8 * rs : 0), v1 ? 16u : 0u);
+        ioff += tile_bytes;
+        if (++itile == T) {
+            itile = 0;
+            ++iq;
+            ioff += 64 - T * tile_bytes;
+            iin_k = 256 * iq + 64 * t < a.K;
+        }
+    };
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
-        if (u0 + s < u1) {
-            issue(iq, itile, s);
-            advance(iq, itile);
-        }
+        if (u0 + s < u1) issue_next(s);
         cp_async_commit();
     }
 
@@ -208,11 +250,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const GsArgs a
             const bool in_k = 256 * q + 64 * t < a.K;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                b[i] = (in_k && g < a.M) ? __ldg(reinterpret_cast<const uint4*>(x0 + 256 * q + 16 * i))
-                                         : make_uint4(0, 0, 0, 0);
-                if constexpr (MT == 2)
-                    bb[i] = (in_k && g + 8 < a.M) ? __ldg(reinterpret_cast<const uint4*>(x1 + 256 * q + 16 * i))
-                                                  : make_uint4(0, 0, 0, 0);
+                b[i] = bb[i] = make_uint4(0, 0, 0, 0);
+                if (a.xs) {
+                    if (in_k && g < a.M) b[i] = lds128(xsm + g * xstride + 256 * q + 64 * t + 16 * i);
+                    if (MT == 2 && in_k && g + 8 < a.M)
+                        bb[i] = lds128(xsm + (g + 8) * xstride + 256 * q + 64 * t + 16 * i);
+                } else {
+                    if (in_k && g < a.M) b[i] = __ldg(reinterpret_cast<const uint4*>(x0 + 256 * q + 16 * i));
+                    if (MT == 2 && in_k && g + 8 < a.M)
+                        bb[i] = __ldg(reinterpret_cast<const uint4*>(x1 + 256 * q + 16 * i));
+                }
             }
         }
         cp_async_wait<kStages - 1>();
@@ -234,10 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_stream_kernel(const GsArgs a
                 s4_group2(acc[i & 1], acc2[i & 1], word_of(wg, i), word_of(wh, i), b[i], bb[i], mul);
         }
         // the MMAs have consumed the stage's words: refill it with the unit kStages ahead
-        if (u + kStages < u1) {
-            issue(iq, itile, stage);
-            advance(iq, itile);
-        }
+        if (u + kStages < u1) issue_next(stage);
         cp_async_commit();
         if (++stage == kStages) stage = 0;
         // fragment: rows g (e = 0, 1) and g + 8 (e = 2, 3), tokens 2t + (e & 1)
@@ -274,7 +318,13 @@ int sm_count() {
     return sms;
 }
 
-size_t smem_bytes(int MT) { return static_cast<size_t>(kMaxTiles) * 8 * MT * kTokStride * sizeof(int) + kRingBytes; }
+// Shared memory of a launch, and whether the activations are staged in it.
+size_t smem_bytes(int MT, int tmax, int64_t M, int64_t K, bool* xs) {
+    const size_t base = red_bytes_of(tmax, MT) + static_cast<size_t>(kRingBytes);
+    const size_t xbytes = static_cast<size_t>(M) * static_cast<size_t>(K + kXPad);
+    *xs = base + xbytes <= static_cast<size_t>(kSmemLimit);
+    return *xs ? base + xbytes : base;
+}
 
 }  // namespace
 
@@ -292,20 +342,26 @@ cudaError_t launch_gemv_stream(const int8_t* xq, const float* s, const uint8_t* 
     if (!gemv_stream_applicable(M, N, K)) return cudaErrorInvalidValue;
     const int sms = sm_count();
     const int MT = M <= 8 ? 1 : 2;
+    const int64_t ntiles = (N + 15) / 16;
+    const int tmax = static_cast<int>((ntiles + sms - 1) / sms);
+    bool xs = false;
+    const size_t smem = smem_bytes(MT, tmax, M, K, &xs);
     GsArgs a{packed, xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-             static_cast<int>((N + 15) / 16), static_cast<int>((K + 255) / 256), out, out_kind_of(kind),
-             gamma_rows_of(kind), s4_mul()};
+             static_cast<int>(ntiles), static_cast<int>((K + 255) / 256), out, out_kind_of(kind),
+             gamma_rows_of(kind), tmax, xs ? 1 : 0, s4_mul()};
     static PerContextOnce attr[2];
     cudaError_t e = attr[MT - 1].run([MT] {
         return MT == 1 ? cudaFuncSetAttribute(gemv_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(smem_bytes(1)))
+                                              kSmemLimit)
                        : cudaFuncSetAttribute(gemv_stream_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(smem_bytes(2)));
+                                              kSmemLimit);
     });
     if (e != cudaSuccess) return e;
     if (MT == 1)
-        return launch_pdl(gemv_stream_kernel<1>, dim3(sms), dim3(kThreads), smem_bytes(1), stream, dim3(kNoCluster), a);
-    return launch_pdl(gemv_stream_kernel<2>, dim3(sms), dim3(kThreads), smem_bytes(2), stream, dim3(kNoCluster), a);
+        return launch_pdl(gemv_stream_kernel<1>, dim3(sms), dim3(32 * StreamCfg<1>::W), smem, stream,
+                          dim3(kNoCluster), a);
+    return launch_pdl(gemv_stream_kernel<2>, dim3(sms), dim3(32 * StreamCfg<2>::W), smem, stream, dim3(kNoCluster),
+                      a);
 }
 
 }  // namespace bl

@@ -88,8 +88,9 @@ def run(xq_ref, s_ref, packed_ref, gamma, dtypes=ALL, rows=None, path=ST, gamma_
     return outs
 
 
-# (M, N, K): one token tile (M <= 8) and two (9..16); N from just over 148 tiles (blocks of
-# one or two tiles, a ragged last tile) up; K from one quarter to 40, with partial quarters
+# (M, N, K): one token tile (M <= 8) and two (9..16); N from just over one tile per SM
+# (blocks of one or two tiles, a ragged last tile) up; K from one quarter to 40, with
+# partial quarters; activations staged in shared memory or read from global memory
 SHAPES = [(1, 2368, 64), (3, 2353, 192), (8, 2400, 320), (9, 3000, 1024), (16, 4737, 640), (2, 5000, 2112),
           (7, 9000, 4160), (12, 2400, 10048)]
 
@@ -126,14 +127,14 @@ def test_stream_llama70b_decode(M, N, K):
 
 
 def test_stream_most_tiles_per_block():
-    """64 tiles per block on 148 SMs (N = 148 * 64 * 16 rows), the kernel's limit, and one
-    row more is refused."""
+    """64 tiles per block on every SM (N = SMs * 64 * 16 rows), the kernel's limit, and
+    one tile more is refused."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     N, K, M = sms * 64 * 16, 128, 5
     g, packed, xq, s = problem(M, N, K, seed=3)
     run(xq, s, packed, g, dtypes=(torch.int32, torch.float32))
     xd = torch.zeros(M, K, dtype=torch.int8, device=DEV)
-    big = torch.zeros(N + 1, K // 4, dtype=torch.uint8, device=DEV)
+    big = torch.zeros(N + 16, K // 4, dtype=torch.uint8, device=DEV)
     with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):
         B.forward(xd, torch.ones(M, device=DEV), big, torch.ones(1, device=DEV), torch.int32, path=ST, layout=S4)
 
