@@ -78,8 +78,10 @@ typedef enum {
 } bl_dtype;
 
 typedef enum {
-    BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core paths cannot tile), the
-                           small-batch tcgen05 kernel for 16 < M <= 64, else tiled tcgen05 */
+    BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core paths cannot tile); for
+                           16 < M <= 64 the GEMV fed by asynchronous copies up to 32 tokens
+                           (stride-4 x_q, wide enough layers), else the small-batch tcgen05
+                           kernel; tiled tcgen05 above 64 tokens */
     BL_PATH_GEMV = 1,   /* register-unpack GEMV, any M (token tiles of 16) */
     BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
     BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
@@ -87,9 +89,9 @@ typedef enum {
     BL_PATH_SKINNY = 5, /* the tcgen05 small-batch kernel (K split over a cluster when rows
                            are few); K % 64 == 0 */
     BL_PATH_GEMV_STREAM = 6, /* the GEMV kernel fed by per-thread asynchronous copies (testing):
-                                M <= 16, x_q in BL_XQ_K16_STRIDE4, K % 64 == 0, K <= 2^17, and
-                                between 1 and 64 sixteen-row tiles of N per SM (2353 to
-                                151552 rows on a B200); other shapes return
+                                M <= 64, x_q in BL_XQ_K16_STRIDE4, K % 64 == 0, K <= 2^17, and
+                                between 1 and 64 (48 for M > 16) sixteen-row tiles of N per SM
+                                (N from 2353 rows on a B200); other shapes return
                                 BL_ERR_UNSUPPORTED_SHAPE */
     BL_PATH_GEMV_TMA = 7     /* the persistent TMA-fed GEMV kernel (testing): M <= 16, x_q in
                                 BL_XQ_K16_STRIDE4, K % 128 == 0, K <= 2^17, and between 1 and
@@ -212,9 +214,10 @@ BL_API bl_status bitlinear_norm_quantize_act(const uint16_t *X, const float *nor
  *   out     out : [M, N] of out_dtype, device.
  *   err_word out: optional; BL_ERRBIT_TIMEOUT if a bounded device wait gave up (the
  *                 output is then incomplete).
- * M <= 16 runs the register-unpack GEMV; 16 < M <= 64 the small-batch tcgen05 kernel and
- * larger M the tiled tcgen05 kind::i8 path, when K % 64 == 0 (else the GEMV).  K * 127
- * must stay below 2^31.
+ * M <= 16 runs the register-unpack GEMV; 16 < M <= 64 the small-batch tcgen05 kernel (up
+ * to 32 tokens with x_q in BL_XQ_K16_STRIDE4, the GEMV fed by asynchronous copies where its
+ * shape conditions hold) and larger M the tiled tcgen05 kind::i8 path, when K % 64 == 0
+ * (else the GEMV).  K * 127 must stay below 2^31.
  * Errors: BL_ERR_INVALID_ARG, BL_ERR_UNSUPPORTED_SHAPE, BL_ERR_MISALIGNED, BL_ERR_CUDA. */
 BL_API bl_status bitlinear_forward(const int8_t *xq, const float *s, const uint8_t *packed,
                             const float *gamma, int64_t M, int64_t N, int64_t K, void *out,

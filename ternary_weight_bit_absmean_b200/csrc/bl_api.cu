@@ -192,8 +192,14 @@ static bl_status forward_impl(const int8_t* xq, const float* s, const uint8_t* p
         return BL_ERR_UNSUPPORTED_SHAPE;
     if (path == BL_PATH_GEMV_TMA && (xq_layout != BL_XQ_K16_STRIDE4 || !bl::gemv_tma_applicable(M, N, K)))
         return BL_ERR_UNSUPPORTED_SHAPE;
-    if (path == BL_PATH_AUTO)
-        path = (M <= 16 || !k64 || s4_big) ? BL_PATH_GEMV : (M <= 64 ? BL_PATH_SKINNY : BL_PATH_TC);
+    if (path == BL_PATH_AUTO) {
+        if (M <= 16 || !k64 || s4_big)
+            path = BL_PATH_GEMV;
+        else if (M <= 32 && xq_layout == BL_XQ_K16_STRIDE4 && bl::gemv_stream_applicable(M, N, K))
+            path = BL_PATH_GEMV_STREAM;  // measured faster than the small-batch kernel up to 32 tokens
+        else
+            path = M <= 64 ? BL_PATH_SKINNY : BL_PATH_TC;
+    }
     if (gamma_per_row && !aligned16(gamma)) return BL_ERR_MISALIGNED;
     const int kind = static_cast<int>(out_dtype) | (gamma_per_row ? bl::kGammaPerRow : 0);
     const int lay = static_cast<int>(xq_layout);

@@ -43,19 +43,25 @@ namespace bl {
 
 namespace {
 
-// Warps per block and units in flight per warp, per token-tile count: one token tile
-// fits 64 registers, so 32 warps x 3 stages; two need more, so 24 warps x 4 stages
-// (measured on the LLaMA-70B decode shapes).  Either way 96 KB of copies per SM.
+// Warps per block and units in flight per warp, per token-tile count MT (tiles of 8
+// tokens): one token tile fits 64 registers, so 32 warps x 3 stages; two need more, so 24
+// warps x 4 stages (measured on the LLaMA-70B decode shapes); four hold 64 activation
+// registers, so 16 warps x 6 stages.  Either way 96 KB of copies per SM.  NS accumulator
+// sets alternate between the 16-groups of a unit (two independent MMA chains) where the
+// registers allow.  A block takes at most kMaxTiles 16-row tiles (fewer with four token
+// tiles, whose accumulator is larger).
 template <int MT>
 struct StreamCfg {
-    static constexpr int W = MT == 1 ? 32 : 24;
-    static constexpr int S = MT == 1 ? 3 : 4;
+    static constexpr int W = MT == 1 ? 32 : MT == 2 ? 24 : 16;
+    static constexpr int S = MT == 1 ? 3 : MT == 2 ? 4 : 6;
+    static constexpr int NS = MT == 4 ? 1 : 2;
+    static constexpr int kMaxTiles = MT == 4 ? 48 : 64;
 };
 constexpr int kWarpStage = 1024;                // bytes per warp and stage: [row g | row g + 8][lane][16 B]
 constexpr int kRingBytes = 96 * 1024;
 static_assert(StreamCfg<1>::W * StreamCfg<1>::S * kWarpStage == kRingBytes, "ring size");
 static_assert(StreamCfg<2>::W * StreamCfg<2>::S * kWarpStage == kRingBytes, "ring size");
-constexpr int kMaxTiles = 64;                   // 16-row tiles per block
+static_assert(StreamCfg<4>::W * StreamCfg<4>::S * kWarpStage == kRingBytes, "ring size");
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kXPad = 16;                       // bytes after each staged activation row
 constexpr int kTokStride = 20;                  // ints per token row of a tile's accumulator
@@ -73,7 +79,7 @@ struct GsArgs {
     int kind;
     int grow;  // gamma holds one scale per output row
     int tmax;  // the most tiles a block owns (sizes the accumulator)
-    int xs;    // the activations are staged in shared memory (M rows of K + kXPad bytes)
+    int xs;    // the block's tokens' activations are staged in shared memory (K + kXPad bytes a row)
     S4Mul mul;
 };
 
@@ -97,44 +103,25 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-#define BL_MMA(D, A, B) "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 " D ", " A ", " B ", " D ";\n\t"
-
-// One 16-group of the thread's two rows (words wg: row g, wh: row g + 8) against one
-// token tile's activations b (16 bytes in stride-4 order): two MMAs into acc.
-__device__ __forceinline__ void s4_group(int (&acc)[4], uint32_t wg, uint32_t wh, uint4 b, const S4Mul& k) {
-    asm volatile(
-        "{\n\t.reg .b32 ta, tx, ty, tv, tt;\n\t"
-        ".reg .b32 p0,p1,p2,p3,q0,q1,q2,q3;\n\t"
-        BL_S4_UNPACK("%4", "p0", "p1", "p2", "p3", "%10", "%11", "%12", "%13", "%14")
-        BL_S4_UNPACK("%5", "q0", "q1", "q2", "q3", "%10", "%11", "%12", "%13", "%14")
-        BL_MMA("{%0,%1,%2,%3}", "{p0,q0,p1,q1}", "{%6,%7}")
-        BL_MMA("{%0,%1,%2,%3}", "{p2,q2,p3,q3}", "{%8,%9}")
+// One 16-group of the thread's two rows (words wg: row g, wh: row g + 8) unpacked into
+// the A fragments of two MMAs, {p0, q0, p1, q1} and {p2, q2, p3, q3}.
+__device__ __forceinline__ void unpack_pair(uint32_t wg, uint32_t wh, uint32_t (&p)[4], uint32_t (&q)[4],
+                                            const S4Mul& k) {
+    asm("{\n\t.reg .b32 ta, tx, ty, tv, tt;\n\t"
+        BL_S4_UNPACK("%8", "%0", "%1", "%2", "%3", "%10", "%11", "%12", "%13", "%14")
+        BL_S4_UNPACK("%9", "%4", "%5", "%6", "%7", "%10", "%11", "%12", "%13", "%14")
         "}\n"
-        : "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3])
-        : "r"(wg), "r"(wh), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(k.hi1), "r"(k.two), "r"(k.m4), "r"(k.m16),
-          "r"(k.m64));
+        : "=&r"(p[0]), "=&r"(p[1]), "=&r"(p[2]), "=&r"(p[3]), "=&r"(q[0]), "=&r"(q[1]), "=&r"(q[2]), "=&r"(q[3])
+        : "r"(wg), "r"(wh), "r"(k.hi1), "r"(k.two), "r"(k.m4), "r"(k.m16), "r"(k.m64));
 }
 
-// The same for two token tiles sharing the unpacked words (tokens 0-7 into acc, 8-15
-// into acc2).
-__device__ __forceinline__ void s4_group2(int (&acc)[4], int (&acc2)[4], uint32_t wg, uint32_t wh, uint4 b,
-                                          uint4 bb, const S4Mul& k) {
-    asm volatile(
-        "{\n\t.reg .b32 ta, tx, ty, tv, tt;\n\t"
-        ".reg .b32 p0,p1,p2,p3,q0,q1,q2,q3;\n\t"
-        BL_S4_UNPACK("%8", "p0", "p1", "p2", "p3", "%18", "%19", "%20", "%21", "%22")
-        BL_S4_UNPACK("%9", "q0", "q1", "q2", "q3", "%18", "%19", "%20", "%21", "%22")
-        BL_MMA("{%0,%1,%2,%3}", "{p0,q0,p1,q1}", "{%10,%11}")
-        BL_MMA("{%0,%1,%2,%3}", "{p2,q2,p3,q3}", "{%12,%13}")
-        BL_MMA("{%4,%5,%6,%7}", "{p0,q0,p1,q1}", "{%14,%15}")
-        BL_MMA("{%4,%5,%6,%7}", "{p2,q2,p3,q3}", "{%16,%17}")
-        "}\n"
-        : "+r"(acc[0]), "+r"(acc[1]), "+r"(acc[2]), "+r"(acc[3]), "+r"(acc2[0]), "+r"(acc2[1]), "+r"(acc2[2]),
-          "+r"(acc2[3])
-        : "r"(wg), "r"(wh), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w), "r"(bb.x), "r"(bb.y), "r"(bb.z), "r"(bb.w),
-          "r"(k.hi1), "r"(k.two), "r"(k.m4), "r"(k.m16), "r"(k.m64));
+// d += A (16 rows x 32 codes) * B (32 codes x 8 tokens), s8 x s8 -> s32.
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-#undef BL_MMA
 
 __device__ __forceinline__ void store_y(void* out, int kind, int64_t idx, int acc, float fac) {
     if (kind == kOutI32) {
@@ -158,30 +145,36 @@ __host__ __device__ constexpr uint32_t red_bytes_of(int tmax, int MT) {
     return (static_cast<uint32_t>(tmax) * 8 * MT * kTokStride * 4 + 15u) & ~15u;
 }
 
+// grid: x = one block per SM (a run of 16-row tiles each), y = groups of 8 MT tokens.
 template <int MT>
 __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(const GsArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     constexpr int TOK = 8 * MT;
-    constexpr int kWarps = StreamCfg<MT>::W, kStages = StreamCfg<MT>::S, kThreads = 32 * kWarps;
+    constexpr int kWarps = StreamCfg<MT>::W, kStages = StreamCfg<MT>::S, NS = StreamCfg<MT>::NS;
+    constexpr int kThreads = 32 * kWarps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int t_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * a.ntiles) / gridDim.x);
     const int t_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * a.ntiles) / gridDim.x);
     const int T = t_end - t_begin;
+    // this block's tokens: m0 .. m0 + Mg - 1
+    const int m0 = TOK * static_cast<int>(blockIdx.y);
+    const int Mg = a.M - m0 < TOK ? a.M - m0 : TOK;
     int* red = reinterpret_cast<int*>(smem);
     const uint32_t red_bytes = red_bytes_of(a.tmax, MT);
     const uint32_t ring = smem_u32(smem) + red_bytes + static_cast<uint32_t>(warp * kStages * kWarpStage) +
                           static_cast<uint32_t>(16 * lane);
     const uint32_t xsm = smem_u32(smem) + red_bytes + kRingBytes;
     const int xstride = a.K + kXPad;
+    const int8_t* xblk = a.xq + static_cast<int64_t>(m0) * a.K;
 
     for (int i = threadIdx.x; i < T * TOK * kTokStride; i += kThreads) red[i] = 0;
     pdl_wait_then_release();
     if (a.xs) {
         const int cpr = a.K / 16;  // 16-byte chunks per activation row
-        for (int c = threadIdx.x; c < a.M * cpr; c += kThreads) {
+        for (int c = threadIdx.x; c < Mg * cpr; c += kThreads) {
             const int r = c / cpr, k = c - r * cpr;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.xq + static_cast<int64_t>(r) * a.K) + k);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xblk + static_cast<int64_t>(r) * a.K) + k);
             asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(xsm + r * xstride + 16 * k), "r"(v.x),
                          "r"(v.y), "r"(v.z), "r"(v.w)
                          : "memory");
@@ -235,13 +228,12 @@ __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(c
     asm volatile("mov.b32 %0, %5;\n\tmov.b32 %1, %6;\n\tmov.b32 %2, %7;\n\tmov.b32 %3, %8;\n\tmov.b32 %4, %9;"
                  : "=r"(mul.hi1), "=r"(mul.two), "=r"(mul.m4), "=r"(mul.m16), "=r"(mul.m64)
                  : "r"(a.mul.hi1), "r"(a.mul.two), "r"(a.mul.m4), "r"(a.mul.m16), "r"(a.mul.m64));
-    // activation rows of tokens g and g + 8; a token past M, or a quarter piece past K,
-    // holds zeros (its products are never stored, or meet zero-filled weights)
-    const int8_t* x0 = a.xq + static_cast<int64_t>(g) * a.K + 64 * t;
-    const int8_t* x1 = a.xq + static_cast<int64_t>(g + 8) * a.K + 64 * t;
-    uint4 b[4], bb[4];
+    // b[m][i]: the activations of token g + 8 m of the group at the thread's 16-group i of
+    // the current quarter; a token past the group, or a piece past K, holds zeros (its
+    // products are never stored, or meet zero-filled weights)
+    uint4 b[MT][4];
     int qcur = -1;
-    int acc[2][4], acc2[2][4];
+    int acc[NS][MT][4];
     int stage = 0;
     int q = cq0, tile = ctile0;
     for (int u = u0; u < u1; ++u, advance(q, tile)) {
@@ -249,65 +241,67 @@ __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(c
             qcur = q;
             const bool in_k = 256 * q + 64 * t < a.K;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                b[i] = bb[i] = make_uint4(0, 0, 0, 0);
-                if (a.xs) {
-                    if (in_k && g < a.M) b[i] = lds128(xsm + g * xstride + 256 * q + 64 * t + 16 * i);
-                    if (MT == 2 && in_k && g + 8 < a.M)
-                        bb[i] = lds128(xsm + (g + 8) * xstride + 256 * q + 64 * t + 16 * i);
-                } else {
-                    if (in_k && g < a.M) b[i] = __ldg(reinterpret_cast<const uint4*>(x0 + 256 * q + 16 * i));
-                    if (MT == 2 && in_k && g + 8 < a.M)
-                        bb[i] = __ldg(reinterpret_cast<const uint4*>(x1 + 256 * q + 16 * i));
+            for (int m = 0; m < MT; ++m) {
+                const bool ok = in_k && g + 8 * m < Mg;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int off = 256 * q + 64 * t + 16 * i;
+                    b[m][i] = !ok ? make_uint4(0, 0, 0, 0)
+                              : a.xs ? lds128(xsm + (g + 8 * m) * xstride + off)
+                                     : __ldg(reinterpret_cast<const uint4*>(
+                                           xblk + static_cast<int64_t>(g + 8 * m) * a.K + off));
                 }
             }
         }
         cp_async_wait<kStages - 1>();
         const uint32_t src = ring + static_cast<uint32_t>(stage * kWarpStage);
-        uint4 wg, wh;
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(wg.x), "=r"(wg.y), "=r"(wg.z), "=r"(wg.w) : "r"(src));
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(wh.x), "=r"(wh.y), "=r"(wh.z), "=r"(wh.w)
-                     : "r"(src + kWarpStage / 2));
+        const uint4 wg = lds128(src), wh = lds128(src + kWarpStage / 2);
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < NS; ++j)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[j][e] = acc2[j][e] = 0;
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[j][m][e] = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if constexpr (MT == 1)
-                s4_group(acc[i & 1], word_of(wg, i), word_of(wh, i), b[i], mul);
-            else
-                s4_group2(acc[i & 1], acc2[i & 1], word_of(wg, i), word_of(wh, i), b[i], bb[i], mul);
+            uint32_t pa[4], qa[4];
+            unpack_pair(word_of(wg, i), word_of(wh, i), pa, qa, mul);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                mma_s8(acc[i % NS][m], pa[0], qa[0], pa[1], qa[1], b[m][i].x, b[m][i].y);
+                mma_s8(acc[i % NS][m], pa[2], qa[2], pa[3], qa[3], b[m][i].z, b[m][i].w);
+            }
         }
         // the MMAs have consumed the stage's words: refill it with the unit kStages ahead
         if (u + kStages < u1) issue_next(stage);
         cp_async_commit();
         if (++stage == kStages) stage = 0;
-        // fragment: rows g (e = 0, 1) and g + 8 (e = 2, 3), tokens 2t + (e & 1)
+        // fragment: rows g (e = 0, 1) and g + 8 (e = 2, 3), tokens 8 m + 2t + (e & 1)
         int* rt = red + tile * TOK * kTokStride;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int idx = (2 * t + (e & 1)) * kTokStride + g + 8 * (e >> 1);
-            atomicAdd(rt + idx, acc[0][e] + acc[1][e]);
-            if constexpr (MT == 2) atomicAdd(rt + 8 * kTokStride + idx, acc2[0][e] + acc2[1][e]);
-        }
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int idx = (8 * m + 2 * t + (e & 1)) * kTokStride + g + 8 * (e >> 1);
+                int v = acc[0][m][e];
+                if constexpr (NS == 2) v += acc[NS - 1][m][e];
+                atomicAdd(rt + idx, v);
+            }
     }
     cp_async_wait<0>();
     __syncthreads();
 
     // epilogue: consecutive threads take consecutive rows of one token
     const int rows = 16 * T;
-    const int mt = a.M < TOK ? a.M : TOK;
     const float gamma = (a.kind == kOutI32 || a.grow) ? 0.0f : *a.gamma;
-    for (int i = threadIdx.x; i < mt * rows; i += kThreads) {
+    for (int i = threadIdx.x; i < Mg * rows; i += kThreads) {
         const int tok = i / rows, rl = i - tok * rows;
         const int64_t n = 16 * static_cast<int64_t>(t_begin) + rl;
         if (n >= a.N) continue;
         const int acc_v = red[((rl >> 4) * TOK + tok) * kTokStride + (rl & 15)] >> 6;
         float fac = 0.0f;
-        if (a.kind != kOutI32) fac = __fdiv_rn(a.grow ? a.gamma[n] : gamma, a.s[tok]);
-        store_y(a.out, a.kind, static_cast<int64_t>(tok) * a.N + n, acc_v, fac);
+        if (a.kind != kOutI32) fac = __fdiv_rn(a.grow ? a.gamma[n] : gamma, a.s[m0 + tok]);
+        store_y(a.out, a.kind, static_cast<int64_t>(m0 + tok) * a.N + n, acc_v, fac);
     }
 }
 
@@ -318,50 +312,60 @@ int sm_count() {
     return sms;
 }
 
-// Shared memory of a launch, and whether the activations are staged in it.
-size_t smem_bytes(int MT, int tmax, int64_t M, int64_t K, bool* xs) {
+// Shared memory of a launch with token groups of mg tokens, and whether the activations
+// are staged in it.
+size_t smem_bytes(int MT, int tmax, int64_t mg, int64_t K, bool* xs) {
     const size_t base = red_bytes_of(tmax, MT) + static_cast<size_t>(kRingBytes);
-    const size_t xbytes = static_cast<size_t>(M) * static_cast<size_t>(K + kXPad);
+    const size_t xbytes = static_cast<size_t>(mg) * static_cast<size_t>(K + kXPad);
     *xs = base + xbytes <= static_cast<size_t>(kSmemLimit);
     return *xs ? base + xbytes : base;
 }
 
+// Token tiles of 8 per block: 1 or 2 up to 16 tokens, else groups of 32 tokens (4 tiles).
+int token_tiles(int64_t M) { return M <= 8 ? 1 : M <= 16 ? 2 : 4; }
+
+int max_tiles(int MT) {
+    return MT == 1 ? StreamCfg<1>::kMaxTiles : MT == 2 ? StreamCfg<2>::kMaxTiles : StreamCfg<4>::kMaxTiles;
+}
+
+template <int MT>
+cudaError_t launch_mt(const GsArgs& a, int sms, int groups, size_t smem, cudaStream_t stream) {
+    static PerContextOnce attr;
+    const cudaError_t e = attr.run([] {
+        return cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    });
+    if (e != cudaSuccess) return e;
+    return launch_pdl(gemv_stream_kernel<MT>, dim3(sms, groups), dim3(32 * StreamCfg<MT>::W), smem, stream,
+                      dim3(kNoCluster), a);
+}
+
 }  // namespace
 
-// M <= 16, K % 64 == 0 (16-byte aligned packed rows), K <= 2^17, and between one and
-// kMaxTiles 16-row tiles per SM.
+// M <= 64 (token groups of up to 32), K % 64 == 0 (16-byte aligned packed rows),
+// K <= 2^17, and between one and 64 (48 above 16 tokens) 16-row tiles per SM.
 bool gemv_stream_applicable(int64_t M, int64_t N, int64_t K) {
-    if (M < 1 || M > 16 || K < 64 || K % 64 != 0 || K > kMaxK || N < 1) return false;
+    if (M < 1 || M > 64 || K < 64 || K % 64 != 0 || K > kMaxK || N < 1) return false;
     const int64_t sms = sm_count();
     const int64_t ntiles = (N + 15) / 16;
-    return ntiles >= sms && (ntiles + sms - 1) / sms <= kMaxTiles;
+    return ntiles >= sms && (ntiles + sms - 1) / sms <= max_tiles(token_tiles(M));
 }
 
 cudaError_t launch_gemv_stream(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
                                int64_t M, int64_t N, int64_t K, void* out, int kind, cudaStream_t stream) {
     if (!gemv_stream_applicable(M, N, K)) return cudaErrorInvalidValue;
     const int sms = sm_count();
-    const int MT = M <= 8 ? 1 : 2;
+    const int MT = token_tiles(M);
+    const int groups = static_cast<int>((M + 8 * MT - 1) / (8 * MT));
     const int64_t ntiles = (N + 15) / 16;
     const int tmax = static_cast<int>((ntiles + sms - 1) / sms);
     bool xs = false;
-    const size_t smem = smem_bytes(MT, tmax, M, K, &xs);
-    GsArgs a{packed, xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-             static_cast<int>(ntiles), static_cast<int>((K + 255) / 256), out, out_kind_of(kind),
-             gamma_rows_of(kind), tmax, xs ? 1 : 0, s4_mul()};
-    static PerContextOnce attr[2];
-    cudaError_t e = attr[MT - 1].run([MT] {
-        return MT == 1 ? cudaFuncSetAttribute(gemv_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              kSmemLimit)
-                       : cudaFuncSetAttribute(gemv_stream_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              kSmemLimit);
-    });
-    if (e != cudaSuccess) return e;
-    if (MT == 1)
-        return launch_pdl(gemv_stream_kernel<1>, dim3(sms), dim3(32 * StreamCfg<1>::W), smem, stream,
-                          dim3(kNoCluster), a);
-    return launch_pdl(gemv_stream_kernel<2>, dim3(sms), dim3(32 * StreamCfg<2>::W), smem, stream, dim3(kNoCluster),
-                      a);
+    const size_t smem = smem_bytes(MT, tmax, M < 8 * MT ? M : 8 * MT, K, &xs);
+    const GsArgs a{packed, xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                   static_cast<int>(ntiles), static_cast<int>((K + 255) / 256), out, out_kind_of(kind),
+                   gamma_rows_of(kind), tmax, xs ? 1 : 0, s4_mul()};
+    if (MT == 1) return launch_mt<1>(a, sms, groups, smem, stream);
+    if (MT == 2) return launch_mt<2>(a, sms, groups, smem, stream);
+    return launch_mt<4>(a, sms, groups, smem, stream);
 }
 
 }  // namespace bl

@@ -1,7 +1,9 @@
 """Parity of the decode GEMV fed by per-thread asynchronous copies (BL_PATH_GEMV_STREAM) with
-the oracle, and agreement with the TMA-fed GEMV (BL_PATH_GEMV_TMA) where both apply.
+the oracle, and agreement with the TMA-fed GEMV (BL_PATH_GEMV_TMA) and the small-batch
+tcgen05 kernel where they apply.
 
-Shapes span one and two token tiles (M = 1..16), ragged rows (N not a multiple of 16,
+Shapes span one, two and four token tiles (M = 1..16, then groups of 32 tokens up to
+M = 64, with a ragged last group), ragged rows (N not a multiple of 16,
 blocks with unequal tile counts), K with a partial last 256-code quarter (K % 256 = 64,
 128, 192), the most tiles a block takes, the largest accumulators, per-row weight
 scales and the undefined code 11.  Integers bit-exact, fp32 within 1e-5 relative /
@@ -92,7 +94,8 @@ def run(xq_ref, s_ref, packed_ref, gamma, dtypes=ALL, rows=None, path=ST, gamma_
 # (blocks of one or two tiles, a ragged last tile) up; K from one quarter to 40, with
 # partial quarters; activations staged in shared memory or read from global memory
 SHAPES = [(1, 2368, 64), (3, 2353, 192), (8, 2400, 320), (9, 3000, 1024), (16, 4737, 640), (2, 5000, 2112),
-          (7, 9000, 4160), (12, 2400, 10048)]
+          (7, 9000, 4160), (12, 2400, 10048), (17, 2400, 1024), (32, 2368, 640), (33, 3000, 2112),
+          (50, 2353, 320), (64, 4737, 1024)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -109,11 +112,11 @@ def _layer_weights(N, K):
 
 
 @pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672), (8192, 8192)])
-@pytest.mark.parametrize("M", [1, 4, 8, 16])
+@pytest.mark.parametrize("M", [1, 4, 8, 16, 32, 64])
 def test_stream_llama70b_decode(M, N, K):
     """The LLaMA-70B layer's wide projections at decode token counts: every row in int32
-    against the oracle for M = 1, sampled rows otherwise, and equality with the TMA-fed
-    GEMV on every element."""
+    against the oracle for M = 1, sampled rows otherwise, and equality on every element
+    with the TMA-fed GEMV (M <= 16) or the small-batch tcgen05 kernel (M > 16)."""
     g, packed = _layer_weights(N, K)
     X = synth.activations(M, K, seed=N + K + M, outlier_frac=0.01, outlier_scale=20.0)
     xq, s = oracle.quantize_act(bits(X), EPS)
@@ -121,7 +124,8 @@ def test_stream_llama70b_decode(M, N, K):
     outs = run(xq, s, packed, np.float32(g), dtypes=(torch.int32, torch.bfloat16), rows=rows)
     xd = torch.from_numpy(stride4(xq)).to(DEV)
     other = B.forward(xd, torch.from_numpy(s).to(DEV), torch.from_numpy(packed).to(DEV),
-                      torch.tensor([g], device=DEV), torch.int32, path=B.BL_PATH_GEMV_TMA, layout=S4)
+                      torch.tensor([g], device=DEV), torch.int32,
+                      path=B.BL_PATH_GEMV_TMA if M <= 16 else B.BL_PATH_SKINNY, layout=S4)
     torch.cuda.synchronize()
     assert torch.equal(outs[torch.int32], other)
 
@@ -204,6 +208,6 @@ def test_stream_refuses_other_layouts_and_shapes():
     for packed, layout, M in ((wide, B.BL_XQ_ROWMAJOR, 4), (wide, B.BL_XQ_K16_EVENODD, 4), (narrow, S4, 4)):
         with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):
             B.forward(xq[:M], s[:M], packed, gamma, torch.int32, path=ST, layout=layout)
-    x17 = torch.zeros(17, 256, dtype=torch.int8, device=DEV)
+    x65 = torch.zeros(65, 256, dtype=torch.int8, device=DEV)
     with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):
-        B.forward(x17, torch.ones(17, device=DEV), wide, gamma, torch.int32, path=ST, layout=S4)
+        B.forward(x65, torch.ones(65, device=DEV), wide, gamma, torch.int32, path=ST, layout=S4)

@@ -121,8 +121,9 @@ def test_skinny_ragged(M, N, K, layout):
                                       ("down", 8192, 28672)])
 def test_skinny_llama70b_decode_batches(name, N, K):
     """The LLaMA-70B layer's projections at 17-64 tokens through the automatic dispatch
-    with x_q in the stride-4 layout (as the benchmark runs them): sampled token rows
-    against the oracle, every row through linearity."""
+    with x_q in the stride-4 layout, as the benchmark runs them (the asynchronous-copy
+    GEMV up to 32 tokens, this kernel above): sampled token rows against the oracle,
+    every row through linearity; and the forced small-batch kernel at 32 tokens."""
     W = synth.weight(N, K, seed=N + K)
     g, _, packed = oracle.quantize_weights(W.numpy(), EPS)
     del W
@@ -131,6 +132,8 @@ def test_skinny_llama70b_decode_batches(name, N, K):
         xq, s = oracle.quantize_act(bits(X), EPS)
         rows = np.unique(np.r_[0, M - 1, np.random.default_rng(M).integers(0, M, 1)])
         run(xq, s, packed, g, B.BL_XQ_K16_STRIDE4, ALL, rows=rows, path=B.BL_PATH_AUTO)
+        if M == 32:
+            run(xq, s, packed, g, B.BL_XQ_K16_STRIDE4, (torch.int32,), rows=rows, path=SK)
 
 
 def test_skinny_extreme_accumulators():
