@@ -90,9 +90,8 @@ typedef enum {
                            are few); K % 64 == 0 */
     BL_PATH_GEMV_STREAM = 6, /* the GEMV kernel fed by per-thread asynchronous copies (testing):
                                 M <= 64, x_q in BL_XQ_K16_STRIDE4, K % 64 == 0, K <= 2^17, and
-                                between 1 and 64 (48 for M > 16) sixteen-row tiles of N per SM
-                                (N from 2353 rows on a B200); other shapes return
-                                BL_ERR_UNSUPPORTED_SHAPE */
+                                at most 64 (48 for M > 16) sixteen-row tiles of N per SM; other
+                                shapes return BL_ERR_UNSUPPORTED_SHAPE */
     BL_PATH_GEMV_TMA = 7     /* the persistent TMA-fed GEMV kernel (testing): M <= 16, x_q in
                                 BL_XQ_K16_STRIDE4, K % 128 == 0, K <= 2^17, and between 1 and
                                 32 sixteen-row tiles of N per SM; other shapes return

@@ -18,7 +18,8 @@
 // flight.
 //
 // Work split.  One block per SM owns a contiguous, balanced run of 16-row tiles over the
-// whole of K.  A unit is one tile's 16 rows x one 256-code quarter of K (1 KB of packed
+// whole of K (a layer with fewer tiles than SMs gives each tile to a cluster of 2 to 8
+// blocks that split its K and add their partial sums through distributed shared memory).  A unit is one tile's 16 rows x one 256-code quarter of K (1 KB of packed
 // weights).  The block's units are ordered quarter-major (all tiles of quarter 0, then
 // quarter 1, ...) and cut into equal contiguous chunks, one per warp, so a warp holds one
 // quarter's activations in registers for a run of tiles (read from the block's copy of
@@ -79,6 +80,7 @@ struct GsArgs {
     int kind;
     int grow;  // gamma holds one scale per output row
     int tmax;  // the most tiles a block owns (sizes the accumulator)
+    int ksplit;  // blocks (a cluster) sharing each run of tiles, splitting its K
     int xs;    // the block's tokens' activations are staged in shared memory (K + kXPad bytes a row)
     S4Mul mul;
 };
@@ -91,6 +93,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -145,8 +153,9 @@ __host__ __device__ constexpr uint32_t red_bytes_of(int tmax, int MT) {
     return (static_cast<uint32_t>(tmax) * 8 * MT * kTokStride * 4 + 15u) & ~15u;
 }
 
-// grid: x = one block per SM (a run of 16-row tiles each), y = groups of 8 MT tokens.
-template <int MT>
+// grid: x = one block per SM (a run of 16-row tiles each) or, for layers with fewer tiles
+// than SMs, a cluster of a.ksplit blocks per tile (SPLIT); y = groups of 8 MT tokens.
+template <int MT, bool SPLIT>
 __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(const GsArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     constexpr int TOK = 8 * MT;
@@ -154,8 +163,13 @@ __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(c
     constexpr int kThreads = 32 * kWarps;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int t_begin = static_cast<int>((static_cast<int64_t>(blockIdx.x) * a.ntiles) / gridDim.x);
-    const int t_end = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * a.ntiles) / gridDim.x);
+    // a.ksplit blocks (one cluster when more than one) own the same run of tiles, each a
+    // contiguous share of its units (a range of K, the units being quarter-major)
+    const int S = SPLIT ? a.ksplit : 1;
+    const int rank = SPLIT ? static_cast<int>(cluster_ctarank()) : 0;
+    const int cid = blockIdx.x / S, ncl = gridDim.x / S;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(cid) * a.ntiles) / ncl);
+    const int t_end = static_cast<int>((static_cast<int64_t>(cid + 1) * a.ntiles) / ncl);
     const int T = t_end - t_begin;
     // this block's tokens: m0 .. m0 + Mg - 1
     const int m0 = TOK * static_cast<int>(blockIdx.y);
@@ -183,8 +197,10 @@ __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(c
     __syncthreads();
 
     const int U = T * a.Q;
-    const int u0 = static_cast<int>((static_cast<int64_t>(warp) * U) / kWarps);
-    const int u1 = static_cast<int>((static_cast<int64_t>(warp + 1) * U) / kWarps);
+    const int bu0 = static_cast<int>((static_cast<int64_t>(rank) * U) / S);
+    const int bu1 = static_cast<int>((static_cast<int64_t>(rank + 1) * U) / S);
+    const int u0 = bu0 + static_cast<int>((static_cast<int64_t>(warp) * (bu1 - bu0)) / kWarps);
+    const int u1 = bu0 + static_cast<int>((static_cast<int64_t>(warp + 1) * (bu1 - bu0)) / kWarps);
     const int64_t rs = a.K / 4;  // packed bytes per row
     const int rowg = 16 * t_begin + g;
 
@@ -290,19 +306,33 @@ __global__ void __launch_bounds__(32 * StreamCfg<MT>::W, 1) gemv_stream_kernel(c
     }
     cp_async_wait<0>();
     __syncthreads();
+    // with a K split, every block's partial sums are complete and visible across the
+    // cluster after this barrier; each block then finishes its share of the rows, adding
+    // all blocks' partials through distributed shared memory in rank order (integer sums:
+    // exact in any order), and the second barrier keeps each block's shared memory alive
+    // until the others have read it
+    if constexpr (SPLIT) cluster_sync_all();
 
     // epilogue: consecutive threads take consecutive rows of one token
     const int rows = 16 * T;
+    const int r_begin = (rows * rank) / S, nr = (rows * (rank + 1)) / S - r_begin;
     const float gamma = (a.kind == kOutI32 || a.grow) ? 0.0f : *a.gamma;
-    for (int i = threadIdx.x; i < Mg * rows; i += kThreads) {
-        const int tok = i / rows, rl = i - tok * rows;
+    const uint32_t red_addr = smem_u32(red);
+    for (int i = threadIdx.x; i < Mg * nr; i += kThreads) {
+        const int tok = i / nr, rl = r_begin + (i - tok * nr);
         const int64_t n = 16 * static_cast<int64_t>(t_begin) + rl;
         if (n >= a.N) continue;
-        const int acc_v = red[((rl >> 4) * TOK + tok) * kTokStride + (rl & 15)] >> 6;
+        const int idx = ((rl >> 4) * TOK + tok) * kTokStride + (rl & 15);
+        int sum = red[idx];
+        if constexpr (SPLIT)
+            for (int b = 0; b < S; ++b)
+                if (b != rank) sum += static_cast<int>(ld_cluster_u32(mapa_shared(red_addr + 4u * idx, b)));
+        const int acc_v = sum >> 6;
         float fac = 0.0f;
         if (a.kind != kOutI32) fac = __fdiv_rn(a.grow ? a.gamma[n] : gamma, a.s[m0 + tok]);
         store_y(a.out, a.kind, static_cast<int64_t>(m0 + tok) * a.N + n, acc_v, fac);
     }
+    if constexpr (SPLIT) cluster_sync_all();
 }
 
 int sm_count() {
@@ -328,26 +358,47 @@ int max_tiles(int MT) {
     return MT == 1 ? StreamCfg<1>::kMaxTiles : MT == 2 ? StreamCfg<2>::kMaxTiles : StreamCfg<4>::kMaxTiles;
 }
 
-template <int MT>
-cudaError_t launch_mt(const GsArgs& a, int sms, int groups, size_t smem, cudaStream_t stream) {
+template <int MT, bool SPLIT>
+cudaError_t launch_split(const GsArgs& a, int blocks, int groups, size_t smem, cudaStream_t stream) {
     static PerContextOnce attr;
     const cudaError_t e = attr.run([] {
-        return cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+        return cudaFuncSetAttribute(gemv_stream_kernel<MT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kSmemLimit);
     });
     if (e != cudaSuccess) return e;
-    return launch_pdl(gemv_stream_kernel<MT>, dim3(sms, groups), dim3(32 * StreamCfg<MT>::W), smem, stream,
-                      dim3(kNoCluster), a);
+    return launch_pdl(gemv_stream_kernel<MT, SPLIT>, dim3(blocks, groups), dim3(32 * StreamCfg<MT>::W), smem, stream,
+                      SPLIT ? dim3(a.ksplit, 1, 1) : dim3(kNoCluster), a);
+}
+
+template <int MT>
+cudaError_t launch_mt(const GsArgs& a, int blocks, int groups, size_t smem, cudaStream_t stream) {
+    return a.ksplit > 1 ? launch_split<MT, true>(a, blocks, groups, smem, stream)
+                        : launch_split<MT, false>(a, blocks, groups, smem, stream);
+}
+
+// Work split: with at least one 16-row tile per SM, one block per SM over a balanced run
+// of tiles; with fewer tiles, one tile per run and K split over a cluster of S blocks (a
+// power of two up to 8, S x tiles <= SMs, at most one 256-code quarter per block less).
+struct StreamPlan {
+    int blocks, ksplit, tmax;
+};
+StreamPlan plan_stream(int64_t ntiles, int64_t K, int sms) {
+    if (ntiles >= sms) return {sms, 1, static_cast<int>((ntiles + sms - 1) / sms)};
+    const int64_t Q = (K + 255) / 256;
+    int S = 1;
+    while (S < 8 && 2 * S * ntiles <= sms && 2 * S <= Q) S *= 2;
+    return {static_cast<int>(S * ntiles), S, 1};
 }
 
 }  // namespace
 
 // M <= 64 (token groups of up to 32), K % 64 == 0 (16-byte aligned packed rows),
-// K <= 2^17, and between one and 64 (48 above 16 tokens) 16-row tiles per SM.
+// K <= 2^17, and at most 64 (48 above 16 tokens) 16-row tiles per SM.
 bool gemv_stream_applicable(int64_t M, int64_t N, int64_t K) {
     if (M < 1 || M > 64 || K < 64 || K % 64 != 0 || K > kMaxK || N < 1) return false;
     const int64_t sms = sm_count();
     const int64_t ntiles = (N + 15) / 16;
-    return ntiles >= sms && (ntiles + sms - 1) / sms <= max_tiles(token_tiles(M));
+    return (ntiles + sms - 1) / sms <= max_tiles(token_tiles(M));
 }
 
 cudaError_t launch_gemv_stream(const int8_t* xq, const float* s, const uint8_t* packed, const float* gamma,
@@ -357,15 +408,15 @@ cudaError_t launch_gemv_stream(const int8_t* xq, const float* s, const uint8_t* 
     const int MT = token_tiles(M);
     const int groups = static_cast<int>((M + 8 * MT - 1) / (8 * MT));
     const int64_t ntiles = (N + 15) / 16;
-    const int tmax = static_cast<int>((ntiles + sms - 1) / sms);
+    const StreamPlan p = plan_stream(ntiles, K, sms);
     bool xs = false;
-    const size_t smem = smem_bytes(MT, tmax, M < 8 * MT ? M : 8 * MT, K, &xs);
+    const size_t smem = smem_bytes(MT, p.tmax, M < 8 * MT ? M : 8 * MT, K, &xs);
     const GsArgs a{packed, xq, s, gamma, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
                    static_cast<int>(ntiles), static_cast<int>((K + 255) / 256), out, out_kind_of(kind),
-                   gamma_rows_of(kind), tmax, xs ? 1 : 0, s4_mul()};
-    if (MT == 1) return launch_mt<1>(a, sms, groups, smem, stream);
-    if (MT == 2) return launch_mt<2>(a, sms, groups, smem, stream);
-    return launch_mt<4>(a, sms, groups, smem, stream);
+                   gamma_rows_of(kind), p.tmax, p.ksplit, xs ? 1 : 0, s4_mul()};
+    if (MT == 1) return launch_mt<1>(a, p.blocks, groups, smem, stream);
+    if (MT == 2) return launch_mt<2>(a, p.blocks, groups, smem, stream);
+    return launch_mt<4>(a, p.blocks, groups, smem, stream);
 }
 
 }  // namespace bl

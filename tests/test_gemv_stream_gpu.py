@@ -3,8 +3,9 @@ the oracle, and agreement with the TMA-fed GEMV (BL_PATH_GEMV_TMA) and the small
 tcgen05 kernel where they apply.
 
 Shapes span one, two and four token tiles (M = 1..16, then groups of 32 tokens up to
-M = 64, with a ragged last group), ragged rows (N not a multiple of 16,
-blocks with unequal tile counts), K with a partial last 256-code quarter (K % 256 = 64,
+M = 64, with a ragged last group), ragged rows (N not a multiple of 16, blocks with
+unequal tile counts, and layers with fewer tiles than SMs, whose K is split over a
+cluster of blocks that add their partial sums through distributed shared memory), K with a partial last 256-code quarter (K % 256 = 64,
 128, 192), the most tiles a block takes, the largest accumulators, per-row weight
 scales and the undefined code 11.  Integers bit-exact, fp32 within 1e-5 relative /
 1e-6 absolute, bf16 equal up to rounding-midpoint cases, and no write outside the
@@ -90,12 +91,16 @@ def run(xq_ref, s_ref, packed_ref, gamma, dtypes=ALL, rows=None, path=ST, gamma_
     return outs
 
 
-# (M, N, K): one token tile (M <= 8) and two (9..16); N from just over one tile per SM
-# (blocks of one or two tiles, a ragged last tile) up; K from one quarter to 40, with
-# partial quarters; activations staged in shared memory or read from global memory
+# (M, N, K): one token tile (M <= 8), two (9..16) and groups of 32; N from one row (one
+# tile, K split over a cluster) through fewer tiles than SMs to several tiles per SM
+# (ragged last tiles); K from one quarter to 40, with partial quarters; activations
+# staged in shared memory or read from global memory
 SHAPES = [(1, 2368, 64), (3, 2353, 192), (8, 2400, 320), (9, 3000, 1024), (16, 4737, 640), (2, 5000, 2112),
           (7, 9000, 4160), (12, 2400, 10048), (17, 2400, 1024), (32, 2368, 640), (33, 3000, 2112),
-          (50, 2353, 320), (64, 4737, 1024)]
+          (50, 2353, 320), (64, 4737, 1024),
+          # fewer tiles than SMs: one tile per run, K split over a cluster of 2 to 8 blocks
+          (1, 1024, 8192), (4, 16, 2048), (9, 300, 640), (1, 1536, 1536), (32, 1024, 8192), (17, 40, 256),
+          (2, 1, 4096)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -204,8 +209,7 @@ def test_stream_refuses_other_layouts_and_shapes():
     s = torch.ones(4, device=DEV)
     gamma = torch.ones(1, device=DEV)
     wide = torch.zeros(4096, 64, dtype=torch.uint8, device=DEV)
-    narrow = torch.zeros(1024, 64, dtype=torch.uint8, device=DEV)  # fewer tiles than SMs
-    for packed, layout, M in ((wide, B.BL_XQ_ROWMAJOR, 4), (wide, B.BL_XQ_K16_EVENODD, 4), (narrow, S4, 4)):
+    for packed, layout, M in ((wide, B.BL_XQ_ROWMAJOR, 4), (wide, B.BL_XQ_K16_EVENODD, 4)):
         with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):
             B.forward(xq[:M], s[:M], packed, gamma, torch.int32, path=ST, layout=layout)
     x65 = torch.zeros(65, 256, dtype=torch.int8, device=DEV)
