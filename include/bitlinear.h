@@ -80,8 +80,8 @@ typedef enum {
 typedef enum {
     BL_PATH_AUTO = 0,   /* GEMV for M <= 16 (or shapes the tensor-core paths cannot tile); for
                            16 < M <= 64 the GEMV fed by asynchronous copies up to 32 tokens
-                           (stride-4 x_q, wide enough layers), else the small-batch tcgen05
-                           kernel; tiled tcgen05 above 64 tokens */
+                           (stride-4 x_q), else the small-batch tcgen05 kernel; tiled tcgen05
+                           above 64 tokens */
     BL_PATH_GEMV = 1,   /* register-unpack GEMV, any M (token tiles of 16) */
     BL_PATH_TC = 2,     /* tcgen05 kind::i8 tiled path (single SM or SM pair, by shape); K % 64 == 0 */
     BL_PATH_TC_1SM = 3, /* the tcgen05 path forced to single-SM tiles (testing) */
