@@ -539,7 +539,7 @@ def run_ours(args):
         m1 = dec["by_M"]["1"]
         result["decode_70b"] = dec["by_M"]
         result["roofline_decode"] = {
-            "kernel": "decode forward (gemv_stream for the wide projections, gemv for k/v), the 70B layer's 7 projections at M=1 as one graph",
+            "kernel": "decode forward (gemv_stream; K split over a cluster for the narrow k/v), the 70B layer's 7 projections at M=1 as one graph",
             "bound": "hbm", "achieved": m1["fwd_gbs"], "peak": P["hbm_gbs"], "unit": "GB/s",
             "frac": round(m1["fwd_gbs"] / P["hbm_gbs"], 4), "weight_gbs": m1["weight_gbs"],
             "weight_frac": round(m1["weight_gbs"] / P["hbm_gbs"], 4),
