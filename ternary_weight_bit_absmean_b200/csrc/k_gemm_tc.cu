@@ -33,6 +33,7 @@
 // TMEM is freed and BL_ERRBIT_TIMEOUT is OR-ed into the caller's error word.
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -378,32 +379,91 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // 2-D uint8 tensor map over a row-major [outer, inner] byte matrix with a
 // [box_outer, box_inner] box; 128-byte swizzle or none.
+namespace {
+
+// Encoded tensor maps of recent calls.  A map is a pure function of the arguments that
+// describe it (address, element type, extents, box, swizzle), so a stored copy is valid
+// for any later call with the same arguments, whatever the memory holds; repeated calls
+// on the same buffers (a decode loop) then skip the driver's encoding.
+struct TmapKey {
+    const void* ptr;
+    uint64_t inner, outer;
+    uint32_t box_inner, box_outer, kind;  // kind: element type and swizzle
+    bool operator==(const TmapKey& o) const {
+        return ptr == o.ptr && inner == o.inner && outer == o.outer && box_inner == o.box_inner &&
+               box_outer == o.box_outer && kind == o.kind;
+    }
+};
+constexpr int kTmapCacheSlots = 64;
+struct TmapEntry {
+    TmapKey key;
+    CUtensorMap map;
+    bool used;
+};
+std::mutex g_tmap_mu;
+TmapEntry g_tmap_cache[kTmapCacheSlots];
+
+int tmap_slot(const TmapKey& k) {
+    uint64_t h = reinterpret_cast<uint64_t>(k.ptr) ^ (k.inner * 0x9E3779B97F4A7C15ull) ^ (k.outer << 17) ^
+                 (static_cast<uint64_t>(k.box_inner) << 40) ^ (static_cast<uint64_t>(k.box_outer) << 28) ^ k.kind;
+    h ^= h >> 29;
+    h *= 0xBF58476D1CE4E5B9ull;
+    h ^= h >> 32;
+    return static_cast<int>(h % kTmapCacheSlots);
+}
+
+// Looks the map up, else encodes it with `encode` and stores it.
+template <typename F>
+bool cached_tmap(CUtensorMap* map, const TmapKey& key, F encode) {
+    const int slot = tmap_slot(key);
+    {
+        std::lock_guard<std::mutex> lock(g_tmap_mu);
+        const TmapEntry& e = g_tmap_cache[slot];
+        if (e.used && e.key == key) {
+            *map = e.map;
+            return true;
+        }
+    }
+    if (!encode(map)) return false;
+    std::lock_guard<std::mutex> lock(g_tmap_mu);
+    g_tmap_cache[slot] = TmapEntry{key, *map, true};
+    return true;
+}
+
+}  // namespace
+
 bool encode_tmap_u8_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                        uint32_t box_outer, bool swizzle128) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
-    if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const TmapKey key{ptr, inner, outer, box_inner, box_outer, swizzle128 ? 1u : 0u};
+    return cached_tmap(map, key, [&](CUtensorMap* m) {
+        PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
+        if (fn == nullptr) return false;
+        const cuuint64_t dims[2] = {inner, outer};
+        const cuuint64_t strides[1] = {inner};
+        const cuuint32_t box[2] = {box_inner, box_outer};
+        const cuuint32_t estr[2] = {1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    });
 }
 
 // 2-D tensor map over a row-major [outer, inner] matrix of 4-byte elements (fp32), no
 // swizzle, zero fill outside the matrix.
 bool encode_tmap_f32_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                         uint32_t box_outer) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
-    if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner * 4};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const TmapKey key{ptr, inner, outer, box_inner, box_outer, 2u};
+    return cached_tmap(map, key, [&](CUtensorMap* m) {
+        PFN_cuTensorMapEncodeTiled_v12000 fn = get_encode_fn();
+        if (fn == nullptr) return false;
+        const cuuint64_t dims[2] = {inner, outer};
+        const cuuint64_t strides[1] = {inner * 4};
+        const cuuint32_t box[2] = {box_inner, box_outer};
+        const cuuint32_t estr[2] = {1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    });
 }
 
 namespace {

@@ -914,3 +914,27 @@ def test_bounded_wait_test_rejects_other_paths_and_limits():
     with pytest.raises(B.BitLinearError, match="UNSUPPORTED_SHAPE"):  # no TMA-fed GEMV at this size
         B.bitlinear_forward_stall_test(xq[:4], s[:4], packed, gamma, out[:4], None, 1000, 1, path=B.BL_PATH_GEMV,
                                        layout=B.BL_XQ_K16_STRIDE4)
+
+
+# ------------------------------------------------- reused buffers, other shapes --
+
+def test_tensor_core_paths_reuse_buffers_with_other_shapes():
+    """The same device buffers viewed with different shapes in turn (the launchers keep
+    recently encoded tensor maps, keyed by address and shape): every call matches the
+    oracle, including a shape repeated after another one used the same addresses."""
+    xbuf = torch.empty(1 << 20, dtype=torch.int8, device=DEV)
+    pbuf = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
+    shapes = [(300, 256, 1024), (200, 512, 512), (300, 256, 1024), (129, 384, 640)]
+    for i, (M, N, K) in enumerate(shapes):
+        g_ref, packed_ref, xq_ref, s_ref = make_problem(M, N, K, seed=40 + i)
+        xq = xbuf[:M * K].view(M, K)
+        xq.copy_(torch.from_numpy(xq_ref))
+        packed = pbuf[:N * K // 4].view(N, K // 4)
+        packed.copy_(torch.from_numpy(packed_ref))
+        s = torch.from_numpy(s_ref).to(DEV)
+        gamma = torch.tensor([g_ref], device=DEV)
+        acc_ref = oracle.forward(xq_ref, s_ref, packed_ref, g_ref, K, oracle.OUT_I32)
+        for path in (B.BL_PATH_TC_1SM, B.BL_PATH_TC_2SM, B.BL_PATH_SKINNY):
+            acc = B.forward(xq, s, packed, gamma, torch.int32, path=path)
+            sync()
+            assert np.array_equal(acc.cpu().numpy(), acc_ref), (M, N, K, path)
