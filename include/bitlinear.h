@@ -67,9 +67,12 @@ typedef enum {
     BL_ERR_BAD_CODE = 7           /* (err_word bit) an input code outside {-1, 0, +1} */
 } bl_status;
 
-/* Bits OR-ed into the optional device err_word. */
+/* Bits OR-ed into the optional device err_word.  BL_ERRBIT_INDEX is set only by a library
+ * built with device index checks (BL_DEBUG_CHECKS=1, a debugging build): a kernel found an
+ * index outside its buffer, recorded it here and skipped that access. */
 #define BL_ERRBIT_BAD_CODE 0x1
 #define BL_ERRBIT_TIMEOUT 0x2
+#define BL_ERRBIT_INDEX 0x4
 
 typedef enum {
     BL_OUT_F32 = 0,  /* y as fp32 */

@@ -24,7 +24,7 @@ BL_OK = 0
 BL_OUT_F32, BL_OUT_BF16, BL_OUT_I32 = 0, 1, 2
 (BL_PATH_AUTO, BL_PATH_GEMV, BL_PATH_TC, BL_PATH_TC_1SM, BL_PATH_TC_2SM, BL_PATH_SKINNY, BL_PATH_GEMV_STREAM,
  BL_PATH_GEMV_TMA) = range(8)
-BL_ERRBIT_BAD_CODE, BL_ERRBIT_TIMEOUT = 0x1, 0x2
+BL_ERRBIT_BAD_CODE, BL_ERRBIT_TIMEOUT, BL_ERRBIT_INDEX = 0x1, 0x2, 0x4
 BL_XQ_ROWMAJOR, BL_XQ_K16_EVENODD, BL_XQ_K16_STRIDE4 = 0, 1, 2
 BL_NORM_RMS, BL_NORM_LAYER = 0, 1
 

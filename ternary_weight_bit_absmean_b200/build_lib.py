@@ -1,6 +1,10 @@
 """Build ``libbitlinear.so`` (the CUDA kernels and the C ABI) in-tree for sm_100a.
 
-``python -m ternary_weight_bit_absmean_b200.build_lib [--force] [--verbose]``
+``python -m ternary_weight_bit_absmean_b200.build_lib [--force] [--verbose] [--debug]``
+
+``--debug`` builds ``libbitlinear_debug.so`` instead: the same library with the device
+index checks on (``BL_DEBUG_CHECKS=1``; a failed check ORs ``BL_ERRBIT_INDEX`` into the
+caller's error word and skips the access), for debugging without a sanitizer.
 
 The library is compiled with nvcc for ``sm_100a`` only, position independent, with the
 CUDA runtime linked statically (no dependency on the runtime that PyTorch ships) and
@@ -16,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbitlinear.so")
+DEBUG_LIB = os.path.join(PKG, "libbitlinear_debug.so")
 SOURCES = ["bl_api.cu", "k_quant.cu", "k_gemv.cu", "k_gemv_tma.cu", "k_gemv_tc.cu", "k_gemv_stream.cu", "k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_noalloc.cu", "k_tl5.cu", "k_ste.cu"]
 HEADERS = ["bl_device.cuh", "bl_internal.h"]
 
@@ -47,32 +52,34 @@ def source_digest(files=None) -> str:
 PREFILL_KERNEL_FILES = ["k_gemm_tc.cu", "k_gemm_tc2.cu", "bl_device.cuh"]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(PKG, "_build")
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    objdir = os.path.join(PKG, "_build_debug" if debug else "_build")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [NVCC, *FLAGS, *(["-DBL_DEBUG_CHECKS=1"] if debug else []), "-I", INCLUDE, "-I", CSRC, "-c",
+               os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
                     *objs, "-o", tmp], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

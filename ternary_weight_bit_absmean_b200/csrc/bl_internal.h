@@ -33,6 +33,33 @@ cudaError_t launch_ternarise_pack(const float* W, int64_t numel, const float* ga
 cudaError_t launch_pack_codes(const int8_t* codes, int64_t numel, uint8_t* packed, int32_t* err,
                               cudaStream_t stream);
 
+// Device index checks of a debugging build (BL_DEBUG_CHECKS=1; compute-sanitizer is not
+// available on the GPUs this was built for): bl_check(cond, err) returns cond and, when it
+// is false, ORs BL_ERRBIT_INDEX (0x4) into the error word, so that the caller skips the
+// access instead of trapping.  In a normal build it is `true` and costs nothing.
+#ifndef BL_DEBUG_CHECKS
+#define BL_DEBUG_CHECKS 0
+#endif
+constexpr int kErrBitIndex = 0x4;
+#ifdef __CUDACC__
+__device__ __forceinline__ bool bl_check(bool cond, int32_t* err) {
+#if BL_DEBUG_CHECKS
+    if (!cond && err != nullptr) atomicOr(err, kErrBitIndex);
+    return cond;
+#else
+    (void)cond;
+    (void)err;
+    return true;
+#endif
+}
+// Bytes of dynamic shared memory of the running launch.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+    uint32_t v;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+    return v;
+}
+#endif
+
 // Layouts of x_q (mirror bl_xq_layout).
 enum XqLayout : int { kXqRowMajor = 0, kXqEvenOdd16 = 1, kXqStride4K16 = 2 };
 

@@ -284,10 +284,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait_bounded(pfull(pslot), static_cast<uint32_t>((j / kPS) & 1), abort_flag, a.wait_ns) ||
                 !mbar_wait_bounded(empty(stage), phase ^ 1u, abort_flag, a.wait_ns))
                 break;
-            const uint4 p = *reinterpret_cast<const uint4*>(gbase + (sP - base) + pslot * kPSBytes +
-                                                            erow * (kSuper * kBK / 4) + (i % kSuper) * (kBK / 4) +
-                                                            16 * half);
+            const uint8_t* pp = gbase + (sP - base) + pslot * kPSBytes + erow * (kSuper * kBK / 4) +
+                                (i % kSuper) * (kBK / 4) + 16 * half;
             uint8_t* ap = gbase + (sA - base) + stage * kABytes + erow * kBK;
+            // a debugging build checks that the piece read and the row written lie in the
+            // launch's shared memory
+            const uint32_t dyn = dynamic_smem_bytes();
+            const bool ok_p = bl_check(pp + 16 <= smem_raw + dyn, a.err);
+            const bool ok_a = bl_check(ap + kBK <= smem_raw + dyn, a.err);
+            const uint4 p = ok_p ? *reinterpret_cast<const uint4*>(pp) : make_uint4(0, 0, 0, 0);
             const uint32_t words[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else
                     unpack16_natural(words[c], u.x, u.y, u.z, u.w);
                 const uint32_t chunk = static_cast<uint32_t>(4 * half + c);
-                *reinterpret_cast<uint4*>(ap + ((chunk ^ sw) << 4)) = u;
+                if (ok_a) *reinterpret_cast<uint4*>(ap + ((chunk ^ sw) << 4)) = u;
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -333,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 16; ++j) {
                 const int v = static_cast<int>(acc[j]) >> kAccShift;
                 if (nsplit > 1) {
-                    red[(c0 + j) * kRows + r] = v;
+                    if (bl_check((c0 + j) * kRows + r < BT * kRows, a.err)) red[(c0 + j) * kRows + r] = v;
                 } else {
                     const int tok = t0 + c0 + j;
                     if (tok < a.M && row < a.N) {
@@ -361,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int tok = t0 + tt;
             if (tok >= a.M || row >= a.N) continue;
             int sum = 0;
+            if (!bl_check(tt * kRows + rr < BT * kRows, a.err)) continue;
             for (int b = 0; b < nsplit; ++b)
                 sum += static_cast<int>(ld_shared_cluster_u32(mapa_shared(red_addr + 4u * (tt * kRows + rr), b)));
             const float fac = a.kind == kOutI32 ? 0.0f : __fdiv_rn(gamma, __ldg(a.s + tok));
